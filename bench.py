@@ -1,0 +1,516 @@
+"""Benchmark of the B200 CodeQuant LUT MoE linear layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: the Qwen3-4B-shaped dense SwiGLU FFN decode layer (hidden
+2560, intermediate 9728, gate/up 2560->9728, down 9728->2560) in all six
+published variants -- M in {1, 4, 16} tokens x {A4W4, A8W4}.  One step runs
+each variant once (42 tokens) on its own copy of the weights, so a step
+streams 6 x 38 MB of packed indices + codebooks (> the 126 MB L2) and no
+variant finds its weights in L2 from the previous step.
+
+Reported (one JSON line from rank 0):
+  value       tokens/s of the whole job (sum over ranks / max time), device
+              timed with CUDA events, inputs resident in HBM; the step is
+              replayed from a CUDA graph (the decode serving path)
+  e2e         the same metric through the C-ABI calls with host buffers: the
+              step's activations copied from pinned host memory and the
+              outputs copied back inside the timed region
+  roofline    the dominant kernel (the LUT GEMM): algorithmic bytes over its
+              CUDA-event-timed launches, against the measured HBM copy peak
+  cpu_baseline  the CPU oracle on the host cores, on a bounded token sample
+Multi-GPU: replicas only (each rank runs the whole workload on its own GPU);
+the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "MoE-FFN tokens/s (LUT-GEMV effective GB/s and HBM roofline fraction in roofline)"
+
+
+# ---------------------------------------------------------------------------
+# workloads
+
+
+def workload_shapes(name):
+    import synth
+    if name == "qwen3_4b_ffn_decode":
+        return [synth.cfg1(M, b) for (M, b) in synth.CFG1_VARIANTS]
+    if name == "qwen3_30b_a3b_moe_decode":
+        return [synth.CFG2]
+    if name == "mixtral_8x7b_moe":
+        return [synth.CFG3]
+    if name == "prefill_moe_e64_s2":
+        return [synth.CFG4]
+    if name == "linear_m1_k2048":
+        return None
+    raise SystemExit(f"unknown workload {name}")
+
+
+WORKLOADS = ["qwen3_4b_ffn_decode", "qwen3_30b_a3b_moe_decode", "mixtral_8x7b_moe",
+             "prefill_moe_e64_s2", "linear_m1_k2048"]
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def lut_alg_bytes(M, N, K, bits):
+    """Algorithmic bytes of one LUT product: packed indices + codebooks +
+    activation codes + scales + fp32 output."""
+    return N * K // 2 + 32 * N + M * K * bits // 8 + 4 * M + 4 * M * N
+
+
+def layer_alg(shape, counts=None):
+    """(algorithmic bytes, flops) of one MoE / dense FFN layer call.  Only
+    experts that receive at least one token count for weights."""
+    s = shape
+    T, H, I = s.T, s.H, s.I
+    nbytes = 2 * T * H + 4 * T * H      # x in, out
+    flops = 0
+    groups = []
+    if s.E:
+        nbytes += 4 * T * s.E            # router logits
+        for c in counts:
+            if c > 0:
+                groups.append((int(c), I))
+    for _ in range(s.n_shared):
+        groups.append((T, s.I_shared))
+    for (m, i) in groups:
+        nbytes += 2 * (i * H // 2 + 32 * i) + (H * i // 2 + 32 * H)
+        flops += 2 * m * (2 * i * H + H * i)
+    return nbytes, flops
+
+
+def lut_launch_bytes(shape, counts=None):
+    """Algorithmic bytes of every LUT GEMM launch in one layer call, in
+    launch order (gate/up routed, gate/up shared, down routed, down shared)."""
+    s = shape
+    T, H, I, bits = s.T, s.H, s.I, s.act_bits
+    out = []
+    gu, dn = [], []
+    if s.E:
+        b_gu = b_dn = 0
+        for c in counts:
+            if c > 0:
+                b_gu += lut_alg_bytes(int(c), 2 * I, H, bits)
+                b_dn += lut_alg_bytes(int(c), H, I, bits)
+        gu.append(b_gu)
+        dn.append(b_dn)
+    if s.n_shared:
+        gu.append(s.n_shared * lut_alg_bytes(T, 2 * s.I_shared, H, bits))
+        dn.append(s.n_shared * lut_alg_bytes(T, H, s.I_shared, bits))
+    out = gu + dn
+    return out
+
+
+# ---------------------------------------------------------------------------
+# helpers
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="clk", suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        for line in Path(self.path).read_text().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                 power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 200] or rows
+        reasons = set()
+        for r in load:
+            for k, nm in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                          ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[k].lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "samples_under_load": len(load)}
+
+
+def profile_traffic(kernel_src: Path, profile: Path):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (its sha256 is recorded in the summary)."""
+    if not profile.exists():
+        return None
+    txt = profile.read_text()
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    m_b = re.search(r"dram_bytes_per_launch_full:\s*([0-9.eE+]+)", txt)
+    if not (m_sha and m_b):
+        return None
+    sha = hashlib.sha256(kernel_src.read_bytes()).hexdigest()
+    if sha != m_sha.group(1):
+        return None
+    return float(m_b.group(1))
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline leg and reference arm)
+
+WEIGHT_FIELDS = ("gate_idx", "up_idx", "down_idx", "gate_cb", "up_cb", "down_cb", "sh_gate_idx",
+                 "sh_up_idx", "sh_down_idx", "sh_gate_cb", "sh_up_cb", "sh_down_cb")
+
+
+def workload_inputs(name):
+    """Host inputs of every layer call of one step, keyed by shape name."""
+    import synth
+    shapes = workload_shapes(name)
+    out = {}
+    if name == "qwen3_4b_ffn_decode":
+        # one k-means weight set shared by the six variants (each variant gets
+        # its own device copy in the timed loop)
+        base = synth.moe_inputs(synth.cfg1(16, 4))
+        for s in shapes:
+            x = synth.activations(s.T, s.H, seed=0, name=f"{s.name}.x")
+            out[s.name] = synth.MoEInputs(s, x, None, **{k: getattr(base, k) for k in WEIGHT_FIELDS})
+    else:
+        for s in shapes:
+            out[s.name] = synth.moe_inputs(s)
+    return shapes, out
+
+
+def oracle_threads():
+    try:
+        return int(os.environ.get("OMP_NUM_THREADS") or len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_sample(shapes, inputs, budget_s):
+    """Run the CPU oracle layer on single tokens, cycling through the
+    workload's layer calls, until budget_s has elapsed (at least one call).
+    Returns (tokens, seconds, description)."""
+    import oracle
+    import synth
+    oracle.build()
+    t0 = time.perf_counter()
+    ntok, names = 0, []
+    while True:
+        for s in shapes:
+            inp = inputs[s.name]
+            one = synth.MoEShape(**{**s.__dict__, "T": 1})
+            sub = synth.MoEInputs(one, inp.x[:1],
+                                  inp.logits[:1] if inp.logits is not None else None,
+                                  **{k: getattr(inp, k) for k in WEIGHT_FIELDS})
+            oracle.moe_ffn(sub, one)
+            ntok += 1
+            names.append(s.name)
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"{ntok} single-token layer calls ({', '.join(sorted(set(names)))}) "
+            f"of the C oracle, {dt:.1f} s")
+    return ntok, dt, desc
+
+
+def run_reference(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    if args.workload == "linear_m1_k2048":
+        raise SystemExit("the reference arm runs the FFN / MoE workloads")
+    shapes, inputs = workload_inputs(args.workload)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(shapes, inputs, 0.0)
+    tok = sec = 0.0
+    for _ in range(args.steps):
+        n, dt, desc = cpu_oracle_sample(shapes, inputs, args.ref_step_seconds)
+        tok += n
+        sec += dt
+    v = tok / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sec / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: single-token oracle layer calls for "
+                                   f"~{args.ref_step_seconds:.0f} s, cycling through the "
+                                   f"workload's layer calls"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+
+class DeviceLayer:
+    """One layer call with every tensor resident on the device, plus pinned
+    host copies of its activations / logits / output for the e2e leg."""
+
+    def __init__(self, cq, inp, dev):
+        import torch
+        s = inp.shape
+        self.s = s
+        self.cfg = cq.MoEConfig(H=s.H, I=s.I, E=s.E, top_k=s.top_k, n_shared=s.n_shared,
+                                I_shared=s.I_shared, act_bits=s.act_bits,
+                                had_block_h=s.had_block_h, had_block_i=s.had_block_i,
+                                had_block_i_shared=s.had_block_i_shared,
+                                renormalize=s.renormalize)
+        self.w = {k: torch.from_numpy(np.ascontiguousarray(getattr(inp, k))).to(dev)
+                  for k in WEIGHT_FIELDS if getattr(inp, k) is not None}
+        self.x = torch.from_numpy(inp.x).to(dev)
+        self.lg = torch.from_numpy(inp.logits).to(dev) if s.E else None
+        self.out = torch.empty((s.T, s.H), dtype=torch.float32, device=dev)
+        self.call = cq.MoELayer(self.cfg, s.T, self.w, dev)
+        self.x_h = torch.from_numpy(inp.x).pin_memory()
+        self.lg_h = torch.from_numpy(inp.logits).pin_memory() if s.E else None
+        self.out_h = torch.empty((s.T, s.H), dtype=torch.float32).pin_memory()
+        self.h2d = self.x_h.numel() * 2 + (self.lg_h.numel() * 4 if s.E else 0)
+        self.d2h = self.out_h.numel() * 4
+
+    def run(self):
+        self.call(self.x, self.lg, self.out)
+
+    def run_e2e(self):
+        self.x.copy_(self.x_h, non_blocking=True)
+        if self.lg is not None:
+            self.lg.copy_(self.lg_h, non_blocking=True)
+        self.call(self.x, self.lg, self.out)
+        self.out_h.copy_(self.out, non_blocking=True)
+
+    def counts(self, dev):
+        """Per-expert token counts of this call (for the byte accounting)."""
+        import torch
+        if not self.s.E:
+            return None
+        c = torch.zeros((self.s.E,), dtype=torch.int32, device=dev)
+        self.call(self.x, self.lg, self.out, debug={"counts": c})
+        return c.cpu().numpy()
+
+
+def timed(fn, steps, dist, world):
+    """Device time (ms) of `steps` calls of fn on the current stream,
+    bracketed by barrier + synchronize on both sides; max over ranks."""
+    import torch
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        fn()
+    e1.record(st)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="qwen3_4b_ffn_decode", choices=WORKLOADS)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-graph", action="store_true", help="time eager calls, not a CUDA graph")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    import lut_clustered_weight_b200 as cq
+
+    peak_gbs, peak_tf, peak_kind = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+
+    shapes, inputs = workload_inputs(args.workload)
+    layers = [DeviceLayer(cq, inputs[s.name], dev) for s in shapes]
+    tokens_per_step = sum(s.T for s in shapes)
+
+    def step():
+        for L in layers:
+            L.run()
+
+    # byte / flop accounting (routing counts of the synthetic inputs)
+    counts = [L.counts(dev) for L in layers]
+    lut_bytes_step = sum(sum(lut_launch_bytes(L.s, c)) for L, c in zip(layers, counts))
+    lut_launches_step = sum(len(lut_launch_bytes(L.s, c)) for L, c in zip(layers, counts))
+    alg_bytes_step = sum(layer_alg(L.s, c)[0] for L, c in zip(layers, counts))
+    alg_flops_step = sum(layer_alg(L.s, c)[1] for L, c in zip(layers, counts))
+
+    # ---- warm-up (eager), launch count of one step
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n0 = cq.cq_launch_count()
+    step()
+    torch.cuda.synchronize()
+    launches_per_step = cq.cq_launch_count() - n0
+
+    # ---- timed region: device-resident inputs, CUDA-graph replay of the step
+    use_graph = not args.no_graph
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        run = graph.replay
+    else:
+        run = step
+    for _ in range(args.warmup):
+        run()
+    with ClockSampler(local) as clk:
+        ms = timed(run, args.steps, dist, world)
+    clocks = clk.summary()
+    ms_step = ms / args.steps
+    value = tokens_per_step * args.steps * world / (ms / 1e3)
+
+    # ---- the LUT GEMM kernel, CUDA-event timed launch by launch (eager steps)
+    cq.cq_timing_enable(True)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    cq.cq_timing_enable(False)
+    n_lut, lut_ms = cq.cq_timing_read()
+    assert n_lut == args.steps * lut_launches_step, (n_lut, lut_launches_step)
+    lut_gbs = args.steps * lut_bytes_step / (lut_ms / 1e3) / 1e9
+    traffic = profile_traffic(ROOT / "lut_clustered_weight_b200" / "csrc" / "kernels_lut.cu",
+                              ROOT / "profiles" / f"lut_gemm_{args.workload}.md")
+    roofline = {"bound": "hbm", "achieved": lut_gbs, "peak": peak_gbs, "unit": "GB/s",
+                "frac": lut_gbs / peak_gbs, "peak_source": f"{peak_kind} hbm_gbs",
+                "traffic": traffic, "kernel": "k_lut_mma",
+                "alg_bytes_per_launch": lut_bytes_step / lut_launches_step,
+                "avg_launch_us": 1e3 * lut_ms / n_lut, "launches_timed": n_lut,
+                "lut_share_of_step": (lut_ms / args.steps) / ms_step}
+
+    # ---- e2e: host buffers through the C-ABI, copies inside the timed region
+    def step_e2e():
+        for L in layers:
+            L.run_e2e()
+    for _ in range(args.warmup):
+        step_e2e()
+    ms_e2e = timed(step_e2e, args.steps, dist, world)
+    e2e = {"value": tokens_per_step * args.steps * world / (ms_e2e / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": sum(L.h2d for L in layers),
+           "d2h_bytes_per_step": sum(L.d2h for L in layers),
+           "ms_per_step": ms_e2e / args.steps}
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        n, dt, desc = cpu_oracle_sample(shapes, inputs, args.cpu_seconds)
+        cpu = {"value": n / dt, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+               "sample": desc}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16", "data": "synthetic",
+            "config": {"workload": args.workload,
+                       "layers_per_step": [s.name for s in shapes],
+                       "tokens_per_step": tokens_per_step, "cuda_graph": use_graph,
+                       "l2": "no flush: each step streams "
+                             f"{alg_bytes_step / 1e6:.0f} MB of distinct weights (> 126 MB L2)",
+                       "parallelism": f"replicas x{world}"},
+            "effective_gbs": alg_bytes_step / (ms_step / 1e3) / 1e9,
+            "alg_bytes_per_step": alg_bytes_step, "alg_flops_per_step": alg_flops_step,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+            "dtype_note": "int4/int8 codes and 4-bit indices; LUT weights as fp16 into "
+                          "mma.sync with fp32 accumulation; rotation exact in fp64",
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

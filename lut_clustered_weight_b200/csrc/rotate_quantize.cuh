@@ -1,0 +1,161 @@
+// rotate_quantize.cuh -- exact block Walsh-Hadamard rotation and per-token
+// absmax quantization of one row held in shared memory (one CTA per row).
+//
+// The rotated values are kept in fp64.  fp16 inputs are multiples of 2^-24
+// and every butterfly sum stays below 65504 * 8192 < 2^29, so all of them are
+// integers below 2^53 in units of 2^-24: the fp64 butterflies are exact and
+// the order of the levels does not matter.  The quantization decision
+// round_half_even(qmax * v / A) is then taken exactly with int64 arithmetic.
+#pragma once
+
+#include "cq_common.cuh"
+
+namespace cq {
+
+// In-place Walsh-Hadamard transform (Sylvester order) of every contiguous
+// block of b = 2^log2b elements of buf[0, K).  K % 8 == 0, K % b == 0.
+//   levels 0..4 (index bits 0-4): lanes of a warp, via shuffles
+//   levels 5..7 (bits 5-7):       8 registers per lane (stride 32)
+//   levels 8..  (bits 8..):       one thread per column, stride 256
+template <int THREADS>
+__device__ void block_fwht(double *buf, int K, int log2b) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int NW = THREADS / 32;
+    const int lv1 = log2b < 8 ? log2b : 8;
+    if (lv1 > 0) {
+        for (int base = warp * 256; base < K; base += NW * 256) {
+            double v[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                int k = base + lane + 32 * j;
+                v[j] = k < K ? buf[k] : 0.0;
+            }
+            // bits 0..4: across lanes
+            for (int L = 0; L < (lv1 < 5 ? lv1 : 5); L++) {
+                const int bit = 1 << L;
+                const bool upper = lane & bit;
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    double p = __shfl_xor_sync(0xffffffffu, v[j], bit);
+                    v[j] = upper ? (p - v[j]) : (v[j] + p);
+                }
+            }
+            // bits 5..7: inside the thread
+            for (int L = 5; L < lv1; L++) {
+                const int h = 1 << (L - 5);
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    if ((j & h) == 0) {
+                        double a = v[j], c = v[j + h];
+                        v[j] = a + c;
+                        v[j + h] = a - c;
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                int k = base + lane + 32 * j;
+                if (k < K) buf[k] = v[j];
+            }
+        }
+        __syncthreads();
+    }
+    if (log2b > 8) {
+        const int R = 1 << (log2b - 8);  // 2..32 elements per column
+        const int ncols = K >> (log2b - 8);
+        for (int col = threadIdx.x; col < ncols; col += THREADS) {
+            const int blk = col >> 8, c = col & 255;
+            double *p = buf + ((size_t)blk << log2b) + c;
+            double v[32];
+#pragma unroll
+            for (int r = 0; r < 32; r++)
+                if (r < R) v[r] = p[256 * r];
+#pragma unroll
+            for (int h = 1; h < 32; h <<= 1) {
+                if (h < R) {
+#pragma unroll
+                    for (int r = 0; r < 32; r++) {
+                        if (r < R && (r & h) == 0) {
+                            double a = v[r], d = v[r + h];
+                            v[r] = a + d;
+                            v[r + h] = a - d;
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 32; r++)
+                if (r < R) p[256 * r] = v[r];
+        }
+        __syncthreads();
+    }
+}
+
+// max |buf[k]| over the row, returned to every thread.  red: >= 32 doubles.
+template <int THREADS>
+__device__ double block_absmax(const double *buf, int K, double *red) {
+    double m = 0.0;
+    for (int k = threadIdx.x; k < K; k += THREADS) m = fmax(m, fabs(buf[k]));
+    m = warp_max_d(m);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (warp == 0) {
+        double v = lane < THREADS / 32 ? red[lane] : 0.0;
+        v = warp_max_d(v);
+        if (lane == 0) red[32] = v;
+    }
+    __syncthreads();
+    double A = red[32];
+    __syncthreads();  // red may be reused by the caller
+    return A;
+}
+
+// round_half_even(qmax * v / A) for v, A multiples of 2^-24 (|.| < 2^29), A > 0.
+CQ_DEV int quantize_exact(double v, long long Ai, int qmax) {
+    const long long vi = __double2ll_rn(v * 16777216.0);  // exact integer
+    const long long av = vi < 0 ? -vi : vi;
+    const long long num = (long long)qmax * av;            // < 2^60
+    // fp64 estimate of the quotient, then exact integer correction
+    long long q0 = (long long)floor(__ddiv_rn((double)num, (double)Ai));
+    long long r = num - q0 * Ai;
+    if (r < 0) { q0 -= 1; r += Ai; }
+    if (r >= Ai) { q0 += 1; r -= Ai; }
+    if (2 * r > Ai || (2 * r == Ai && (q0 & 1))) q0 += 1;
+    return (int)(vi < 0 ? -q0 : q0);
+}
+
+// s = (float)((A / sqrt(b)) / qmax), each step IEEE round-to-nearest fp64.
+CQ_DEV float quant_scale(double A, int log2b, int qmax) {
+    return __double2float_rn(__ddiv_rn(__ddiv_rn(A, __dsqrt_rn((double)(1 << log2b))),
+                                       (double)qmax));
+}
+
+// Quantize the rotated row and store its codes: bits 4 -> K/2 packed bytes
+// (low nibble = even k), bits 8 -> K int8.  Writes the scale through s_out.
+template <int THREADS>
+__device__ void block_quantize_store(const double *buf, int K, int log2b, int bits, double A,
+                                     uint8_t *qrow, float *s_out) {
+    const int qmax = (1 << (bits - 1)) - 1;
+    const long long Ai = __double2ll_rn(A * 16777216.0);
+    const double2 *b2 = reinterpret_cast<const double2 *>(buf);
+    for (int p = threadIdx.x; p < K / 2; p += THREADS) {
+        double2 v = b2[p];
+        int q0 = 0, q1 = 0;
+        if (Ai > 0) {
+            q0 = quantize_exact(v.x, Ai, qmax);
+            q1 = quantize_exact(v.y, Ai, qmax);
+        }
+        if (bits == 4) {
+            qrow[p] = (uint8_t)((q0 & 15) | ((q1 & 15) << 4));
+        } else {
+            char2 c;
+            c.x = (char)q0;
+            c.y = (char)q1;
+            reinterpret_cast<char2 *>(qrow)[p] = c;
+        }
+    }
+    if (threadIdx.x == 0) *s_out = Ai > 0 ? quant_scale(A, log2b, qmax) : 0.0f;
+}
+
+}  // namespace cq

@@ -1,0 +1,207 @@
+"""GPU parity of the CUDA path (through the C ABI) against the CPU oracle."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from moe_check import check_moe, moe_inputs_cached, run_moe
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def cq():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import lut_clustered_weight_b200 as m
+    return m
+
+
+def _codes_to_dev(q, bits):
+    return torch.from_numpy(oracle.pack_codes(q, bits)).to(DEV)
+
+
+# ---------------------------------------------------------------------------
+# rotate + quantize
+
+
+RQ_CASES = [
+    # (M, K, b, bits, outliers)
+    (1, 2048, 2048, 4, 4),
+    (3, 2560, 512, 4, 4),
+    (5, 2560, 512, 8, 4),
+    (7, 9728, 256, 4, 4),
+    (2, 9728, 256, 8, 0),
+    (4, 1408, 128, 4, 8),
+    (2, 768, 256, 8, 0),
+    (2, 4096, 4096, 8, 4),
+    (2, 14336, 2048, 8, 4),
+    (2, 8192, 8192, 4, 4),
+    (3, 16384, 16, 4, 2),
+    (6, 8, 8, 4, 0),
+    (5, 24, 1, 8, 1),
+    (33, 64, 4, 4, 0),
+    (0, 256, 256, 4, 0),
+]
+
+
+@pytest.mark.parametrize("M,K,b,bits,outl", RQ_CASES)
+def test_rotate_quantize_bit_exact(cq, M, K, b, bits, outl):
+    x = synth.activations(M, K, seed=1, name=f"rq{M}.{K}.{b}", n_outliers=min(outl, K))
+    if M >= 3:
+        x[1] = 0                        # zero row
+        x[2, : min(K, 7)] = 65504.0      # largest fp16
+        x[2, min(K, 7):] *= np.float16(1e-3)
+    xd = torch.from_numpy(x).to(DEV)
+    q, s = cq.cq_rotate_quantize(xd, b, bits)
+    torch.cuda.synchronize()
+    qr, sr = oracle.rotate_quantize(x, b, bits)
+    qg = oracle.unpack_codes(q.cpu().numpy(), K, bits)
+    assert np.array_equal(qg, qr)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), sr.view(np.uint32))
+
+
+def test_rotate_quantize_exact_ties(cq):
+    # b = 1: x_rot = x; with A = 14 every odd x lands on a tie for int4
+    x = np.array([[14, 1, 3, 5, -7, 9, -11, 13] * 4], dtype=np.float16)
+    for bits in (4, 8):
+        q, s = cq.cq_rotate_quantize(torch.from_numpy(x).to(DEV), 1, bits)
+        qr, sr = oracle.rotate_quantize(x, 1, bits)
+        assert np.array_equal(oracle.unpack_codes(q.cpu().numpy(), 32, bits), qr)
+        assert s.item() == sr[0]
+
+
+# ---------------------------------------------------------------------------
+# LUT GEMM
+
+
+LUT_CASES = [
+    # (M, K, N, bits)
+    (1, 2048, 2048, 4),
+    (1, 32, 64, 4),
+    (3, 96, 128, 8),
+    (8, 160, 64, 4),
+    (9, 2560, 256, 4),
+    (16, 2560, 512, 8),
+    (17, 1408, 192, 4),
+    (40, 768, 128, 8),
+    (5, 9728, 128, 4),
+    (2, 14336, 64, 8),
+]
+
+
+def _lut_inputs(M, K, N, bits, seed):
+    g = np.random.default_rng(seed)
+    qmax = 2 ** (bits - 1) - 1
+    q = g.integers(-qmax, qmax + 1, (M, K)).astype(np.int8)
+    q[0, : min(K, 5)] = qmax
+    if M > 2:
+        q[2] = 0
+    s = (g.random(M) * 0.05 + 1e-3).astype(np.float32)
+    w_idx, cb = synth.lut_weights(N, K, seed=seed, name=f"lut{M}.{K}.{N}")
+    return q, s, w_idx, cb
+
+
+@pytest.mark.parametrize("M,K,N,bits", LUT_CASES)
+def test_lut_gemm_parity(cq, M, K, N, bits):
+    q, s, w_idx, cb = _lut_inputs(M, K, N, bits, seed=M * 7 + K + N)
+    y, S = cq.cq_lut_gemm(_codes_to_dev(q, bits), torch.from_numpy(s).to(DEV), K, bits,
+                          torch.from_numpy(w_idx).to(DEV), torch.from_numpy(cb).to(DEV),
+                          centroid_sums=True)
+    torch.cuda.synchronize()
+    yr, mag, Sr = oracle.lut_gemm(q, s, w_idx, cb, centroid_sums=True)
+    err = np.abs(y.cpu().numpy().astype(np.float64) - yr)
+    tol = oracle.lut_tolerance(mag)
+    assert np.all(err <= tol), f"max excess {(err - tol).max()}, worst ratio {(err / tol).max()}"
+    assert np.array_equal(S.cpu().numpy(), Sr)
+
+
+def test_lut_gemm_config0_full(cq):
+    """Linear M=1, K=N=2048, A4W4 with the real rotate+quantize front end."""
+    s = synth.CFG0
+    x, w_idx, cb = synth.linear_inputs(s)
+    xd = torch.from_numpy(x).to(DEV)
+    q, sx = cq.cq_rotate_quantize(xd, s.had_block, s.act_bits)
+    y = cq.cq_lut_gemm(q, sx, s.K, s.act_bits, torch.from_numpy(w_idx).to(DEV),
+                       torch.from_numpy(cb).to(DEV))
+    torch.cuda.synchronize()
+    qr, sr = oracle.rotate_quantize(x, s.had_block, s.act_bits)
+    assert np.array_equal(oracle.unpack_codes(q.cpu().numpy(), s.K, 4), qr)
+    yr, mag, _ = oracle.lut_gemm(qr, sr, w_idx, cb)
+    err = np.abs(y.cpu().numpy() - yr)
+    assert np.all(err <= oracle.lut_tolerance(mag))
+
+
+def test_lut_gemm_repeatable(cq):
+    """Split-K partials are reduced in a fixed order: bitwise repeatable."""
+    q, s, w_idx, cb = _lut_inputs(4, 9728, 128, 4, seed=3)
+    args = (_codes_to_dev(q, 4), torch.from_numpy(s).to(DEV), 9728, 4,
+            torch.from_numpy(w_idx).to(DEV), torch.from_numpy(cb).to(DEV))
+    y1 = cq.cq_lut_gemm(*args).cpu().numpy()
+    y2 = cq.cq_lut_gemm(*args).cpu().numpy()
+    assert np.array_equal(y1.view(np.uint32), y2.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# MoE / dense FFN, small shapes: every row and token checked
+
+
+SMALL_MOE = [
+    synth.MoEShape("dense_small", H=256, I=512, E=0, top_k=0, n_shared=1, T=5, act_bits=4,
+                   had_block_h=128, had_block_i=64),
+    synth.MoEShape("dense_small8", H=320, I=384, E=0, top_k=0, n_shared=1, T=16, act_bits=8,
+                   had_block_h=64, had_block_i=128),
+    synth.MoEShape("moe_small", H=256, I=192, E=8, top_k=2, n_shared=0, T=24, act_bits=4,
+                   had_block_h=256, had_block_i=64),
+    synth.MoEShape("moe_small_shared", H=192, I=128, E=6, top_k=3, n_shared=2, T=19,
+                   act_bits=8, had_block_h=64, had_block_i=128, bias_expert=0, bias=1.0),
+    synth.MoEShape("moe_norenorm", H=128, I=64, E=16, top_k=4, n_shared=0, T=9, act_bits=4,
+                   had_block_h=128, had_block_i=64, renormalize=0),
+    synth.MoEShape("moe_one_token", H=128, I=128, E=4, top_k=1, n_shared=1, T=1, act_bits=4,
+                   had_block_h=32, had_block_i=32),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL_MOE, ids=lambda s: s.name)
+def test_moe_small_full_parity(cq, shape):
+    inp = moe_inputs_cached(shape)
+    g = run_moe(inp)
+    st = check_moe(inp, g, e2e=True)
+    assert st["e2e_rel_l2"] < 5e-2, st
+
+
+# ---------------------------------------------------------------------------
+# the five workloads at full size, sampled rows / tokens
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("M,bits", synth.CFG1_VARIANTS)
+def test_config1_dense_ffn(cq, M, bits):
+    inp = moe_inputs_cached(synth.cfg1(M, bits))
+    g = run_moe(inp)
+    check_moe(inp, g, sample_rows=4, sample_tokens=4)
+
+
+@pytest.mark.slow
+def test_config2_qwen3_30b_moe(cq):
+    inp = moe_inputs_cached(synth.CFG2)
+    g = run_moe(inp)
+    check_moe(inp, g, sample_rows=12, sample_tokens=6)
+
+
+@pytest.mark.slow
+def test_config3_mixtral_moe(cq):
+    inp = moe_inputs_cached(synth.CFG3)
+    g = run_moe(inp)
+    check_moe(inp, g, sample_rows=4, sample_tokens=4)
+
+
+@pytest.mark.slow
+def test_config4_prefill_moe(cq):
+    inp = moe_inputs_cached(synth.CFG4)
+    g = run_moe(inp)
+    check_moe(inp, g, sample_rows=6, sample_tokens=4)
