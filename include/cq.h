@@ -126,6 +126,40 @@ CQ_API cq_status cq_lut_gemm(const void *q, const float *s_x, int64_t M, int64_t
                       cq_stream_t stream);
 
 /*
+ * cq_lut_gemm_noalloc -- cq_lut_gemm for callers that cannot allocate device
+ * memory.  The pages have no counterpart: this is a deployment variant.
+ *
+ * Some callers can pass a kernel only its inputs and outputs: plugins and
+ * custom-op hosts whose framework owns all device memory and exposes no
+ * allocator, and serving processes that forbid cudaMalloc after start-up
+ * because it synchronizes the device and fragments a pre-sized pool.  This
+ * entry point computes exactly what cq_lut_gemm computes (same kernels, same
+ * split of the contraction, so the same result) but keeps its split-K partial
+ * sums in a fixed array of CQ_NOALLOC_SCRATCH_BYTES bytes compiled into the
+ * library.  It calls no cudaMalloc / cudaFree and no allocating library
+ * routine.
+ *   - The array occupies CQ_NOALLOC_SCRATCH_BYTES of memory on every GPU that
+ *     loads the library, until the process exits.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, under a lock); make that first call before any stream
+ *     capture.
+ *   - All calls share the array and it keeps the last call's contents; each
+ *     call overwrites every partial sum it reads, so nothing needs clearing.
+ *     Calls whose work overlaps on the GPU (other streams, other threads)
+ *     race on the array and must be serialized by the caller.
+ *   - A problem whose partial sums need more than CQ_NOALLOC_SCRATCH_BYTES
+ *     (splits * M * N * 4 bytes, where the split count is chosen as for
+ *     cq_lut_gemm) returns CQ_ERR_UNSUPPORTED and enqueues nothing.
+ * Arguments, layouts and the other checks are those of cq_lut_gemm (without
+ * centroid_sums and workspace).
+ */
+#define CQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+CQ_API cq_status cq_lut_gemm_noalloc(const void *q, const float *s_x, int64_t M, int64_t K,
+                                     int32_t act_bits, const uint8_t *w_idx,
+                                     const void *codebook, int64_t N, float *y,
+                                     cq_stream_t stream);
+
+/*
  * MoE (or dense SwiGLU) FFN layer.
  *
  *   xq, s_x = rotate_quantize(x, had_block_h)              once per token

@@ -19,7 +19,7 @@ LIB_PATH = _PKG / "libcq_b200.so"
 # symbols declared in include/cq.h
 EXPORTS = ("cq_status_string", "cq_version", "cq_rotate_quantize", "cq_lut_gemm_workspace_size",
            "cq_lut_gemm", "cq_moe_ffn_workspace_size", "cq_moe_ffn", "cq_launch_count",
-           "cq_timing_enable", "cq_timing_read")
+           "cq_timing_enable", "cq_timing_read", "cq_lut_gemm_noalloc")
 
 CQ_OK, CQ_ERR_INVALID_ARGUMENT, CQ_ERR_UNSUPPORTED, CQ_ERR_WORKSPACE, CQ_ERR_CUDA = range(5)
 
@@ -74,6 +74,8 @@ lib.cq_moe_ffn_workspace_size.restype = _SZ
 lib.cq_moe_ffn.argtypes = [ctypes.POINTER(MoEDesc), _P, _P, _I64, ctypes.POINTER(MoEWeights), _P,
                            _SZ, _P, ctypes.POINTER(MoEDebug), _P]
 lib.cq_moe_ffn.restype = ctypes.c_int
+lib.cq_lut_gemm_noalloc.argtypes = [_P, _P, _I64, _I64, _I32, _P, _P, _I64, _P, _P]
+lib.cq_lut_gemm_noalloc.restype = ctypes.c_int
 lib.cq_launch_count.argtypes = []
 lib.cq_launch_count.restype = _I64
 lib.cq_timing_enable.argtypes = [_I32]
@@ -177,6 +179,25 @@ def cq_lut_gemm(q: torch.Tensor, s_x: torch.Tensor, K: int, act_bits: int, w_idx
                            _ptr(y), _ptr(centroid_sums if want_S else None), _ptr(workspace), wb,
                            _stream(stream)), "cq_lut_gemm")
     return (y, centroid_sums) if want_S else y
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def cq_lut_gemm_noalloc(q: torch.Tensor, s_x: torch.Tensor, K: int, act_bits: int,
+                        w_idx: torch.Tensor, codebook: torch.Tensor, y=None, stream=None):
+    """cq_lut_gemm without a workspace argument, for callers that cannot
+    allocate device memory: the split-K partial sums live in a fixed 4 MiB
+    array inside the library (shared by all calls; overlapping calls race).
+    Raises CQError(CQ_ERR_UNSUPPORTED) for problems whose partials exceed it."""
+    M = s_x.shape[0]
+    N = w_idx.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=w_idx.device)
+    _check(lib.cq_lut_gemm_noalloc(_ptr(q), _ptr(s_x), M, K, act_bits, _ptr(w_idx),
+                                   _ptr(codebook), N, _ptr(y), _stream(stream)),
+           "cq_lut_gemm_noalloc")
+    return y
 
 
 @dataclass

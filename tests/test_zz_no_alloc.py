@@ -1,0 +1,69 @@
+"""cq_lut_gemm_noalloc: the LUT GEMM for callers that cannot allocate device
+memory (framework plugins that are handed only inputs and outputs, serving
+processes that forbid cudaMalloc after start-up).  Its split-K scratch is a
+fixed array inside the library, so these checks call it through the C ABI
+with caller-owned inputs/outputs only and compare it with cq_lut_gemm, twice
+in a row (the second call reuses the array the first one left behind).
+
+This file is named to be collected last."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # (M, K, N, bits): all need split-K partials (several CTAs per row tile)
+    (4, 9728, 128, 4),
+    (16, 9728, 256, 8),
+    (1, 14336, 64, 4),
+]
+
+
+def _inputs(M, K, N, bits, seed):
+    g = np.random.default_rng(seed)
+    qmax = 2 ** (bits - 1) - 1
+    q = g.integers(-qmax, qmax + 1, (M, K)).astype(np.int8)
+    s = (g.random(M) * 0.05 + 1e-3).astype(np.float32)
+    w_idx, cb = synth.lut_weights(N, K, seed=seed, name=f"noalloc{M}.{K}.{N}")
+    return q, s, w_idx, cb
+
+
+@pytest.mark.parametrize("M,K,N,bits", CASES)
+def test_noalloc_matches_workspace_entry_point(M, K, N, bits):
+    import lut_clustered_weight_b200 as cq
+    assert torch.cuda.is_available()
+    dev = "cuda"
+    q, s, w_idx, cb = _inputs(M, K, N, bits, seed=M + K + N)
+    ws_bytes = cq.cq_lut_gemm_workspace_size(M, N, K, bits)
+    assert 0 < ws_bytes <= cq.NOALLOC_SCRATCH_BYTES   # the scratch path is exercised
+    qd = torch.from_numpy(oracle.pack_codes(q, bits)).to(dev)
+    sd = torch.from_numpy(s).to(dev)
+    wd = torch.from_numpy(w_idx).to(dev)
+    cd = torch.from_numpy(cb).to(dev)
+    y_ref = cq.cq_lut_gemm(qd, sd, K, bits, wd, cd)
+    _, mag, _ = oracle.lut_gemm(q, s, w_idx, cb)
+    tol = oracle.lut_tolerance(mag)
+    stream = torch.cuda.current_stream().cuda_stream
+    for _ in range(2):
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+        rc = cq.lib.cq_lut_gemm_noalloc(qd.data_ptr(), sd.data_ptr(), M, K, bits,
+                                        wd.data_ptr(), cd.data_ptr(), N, y.data_ptr(), stream)
+        assert rc == cq.CQ_OK, cq.status_string(rc)
+        torch.cuda.synchronize()
+        err = np.abs(y.cpu().numpy().astype(np.float64) - y_ref.cpu().numpy())
+        assert np.all(err <= tol)
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    import lut_clustered_weight_b200 as cq
+    M, K, N = 16, 9728, 32768        # partials need more than the fixed array
+    assert cq.cq_lut_gemm_workspace_size(M, N, K, 4) > cq.NOALLOC_SCRATCH_BYTES
+    fake = 1 << 20                   # never dereferenced: the check runs first
+    rc = cq.lib.cq_lut_gemm_noalloc(fake, fake, M, K, 4, fake, fake, N, fake, None)
+    assert rc == cq.CQ_ERR_UNSUPPORTED
