@@ -34,8 +34,8 @@ LutGemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
     LutGemmPlan g;
     const int nt = M <= 8 ? 1 : 2;
     g.tiles = (int)((M + 8 * nt - 1) / (8 * nt));
-    g.p = plan_lut((int)N, (int)K, false, (int)std::min<int64_t>(M, 16), g.tiles);
-    g.ws = g.p.splits > 1 ? align256((size_t)g.p.splits * M * N * sizeof(float)) : 0;
+    g.p = plan_lut((int)N, (int)K, false, (int)std::min<int64_t>(M, 16), g.tiles, (int)M, 1);
+    g.ws = align256((size_t)g.p.splits * M * N * sizeof(float));
     return g;
 }
 
@@ -73,8 +73,10 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
         m.dn_r = plan_lut((int)m.H, (int)m.I, false, rows_per_group, m.max_tiles_r);
     }
     if (m.ns > 0) {
-        m.gu_s = plan_lut((int)m.Is, (int)m.H, true, rows_per_group, m.tiles_s);
-        m.dn_s = plan_lut((int)m.H, (int)m.Is, false, rows_per_group, m.tiles_s);
+        m.gu_s = plan_lut((int)m.Is, (int)m.H, true, rows_per_group, m.tiles_s, (int)T,
+                          (int)m.ns);
+        m.dn_s = plan_lut((int)m.H, (int)m.Is, false, rows_per_group, m.tiles_s, (int)T,
+                          (int)m.ns);
     }
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -200,18 +202,11 @@ cq_status cq_lut_gemm(const void *q, const float *s_x, int64_t M, int64_t K, int
     L.N = (int)N;
     L.dual = false;
     L.out_row_stride = N;
-    if (g.p.splits == 1) {
-        L.direct = true;
-        L.out = y;
-        L.out_split_stride = 0;
-    } else {
-        L.direct = false;
-        L.out = reinterpret_cast<float *>(workspace);
-        L.out_split_stride = M * N;
-    }
+    L.direct = false;
+    L.out = reinterpret_cast<float *>(workspace);
+    L.out_split_stride = M * N;
     cudaError_t e = launch_lut(L, g.p, st);
-    if (e == cudaSuccess && g.p.splits > 1)
-        e = launch_reduce_plain(L.out, g.p.splits, M, N, s_x, y, st);
+    if (e == cudaSuccess) e = launch_reduce_plain(L.out, g.p, M, N, s_x, y, st);
     if (e == cudaSuccess && centroid_sums)
         e = launch_centroid_sums(q, M, K, act_bits, w_idx, N, centroid_sums, st);
     return cuda_status(e);
@@ -301,7 +296,7 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
     if (e == cudaSuccess) {
         SwigluArgs a{};
         a.part_r = pgu_r; a.part_s = pgu_s;
-        a.splits_r = m.E > 0 ? m.gu_r.splits : 0; a.splits_s = m.ns > 0 ? m.gu_s.splits : 0;
+        a.plan_r = m.gu_r; a.plan_s = m.gu_s;
         a.R_routed = m.Rr; a.R_shared = m.Rs;
         a.I = (int)m.I; a.I_shared = (int)m.Is; a.Imax = m.Imax;
         a.log2b_i = m.E > 0 ? ilog2(d->had_block_i) : 0;
@@ -335,7 +330,7 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
     if (e == cudaSuccess) {
         CombineArgs c{};
         c.part_r = pdn_r; c.part_s = pdn_s;
-        c.splits_r = m.E > 0 ? m.dn_r.splits : 0; c.splits_s = m.ns > 0 ? m.dn_s.splits : 0;
+        c.plan_r = m.dn_r; c.plan_s = m.dn_s;
         c.R_routed = m.Rr; c.R_shared = m.Rs;
         c.T = (int)T; c.H = (int)m.H; c.topk = (int)m.k; c.n_shared = (int)m.ns;
         c.inv_perm = inv; c.w = tw; c.h_scales = sh; c.out = out;

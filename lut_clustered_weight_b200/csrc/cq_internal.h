@@ -51,20 +51,67 @@ struct LutLaunch {
     bool direct;            // plain, splits == 1: out[r*N+n] = scale * acc
 };
 
+// How one LUT GEMM launch is cut into work.  A work item is (token tile,
+// row tile); its contraction is cut into 128-k chunks, and the units
+// (work item, chunk) are shared out in one of two ways:
+//   fixed    every work item is split into `splits` equal chunk ranges; the
+//            grid is (row tiles * splits) x (token tiles).  Used when the
+//            token tiles are only known on the device (routed experts).
+//   stream-K the W*C units of all work items are dealt out in equal
+//            contiguous ranges to `grid` CTAs (one wave), so no SM waits on
+//            a tail.  A work item is then covered by a variable number of
+//            CTAs; its partial sums occupy slots 0..n-1.
 struct LutPlan {
-    int nt;             // n8 token tiles per CTA (1 or 2)
-    int n_row_tiles;    // CTA row tiles
-    int chunks_total;   // ceil(K / 128)
+    int nt;             // n8 token tiles per CTA (1 or 2): a token tile has 8*nt rows
+    int warps;          // warps per CTA (4 or 8)
+    int rows_per_rt;    // plain: weight rows per row tile; dual: output columns
+    int n_row_tiles;
+    int chunks_total;   // C = ceil(K / 128)
+    int cps_max;        // most chunks one CTA stages at a time (shared memory)
+    int streamk;
+    int grid;           // CTAs (stream-K) / row_tiles * splits (fixed)
+    int splits;         // fixed: chunk ranges per work item; partial slots allocated
     int chunks_per_split;
-    int splits;
+    int64_t units;      // stream-K: total units (work items * C)
+    int uniform_rows;   // stream-K: rows per group (token tiles of a group are consecutive)
     size_t smem;
 };
 
-LutPlan plan_lut(int N, int K, bool dual, int max_rows_per_group, int64_t est_tiles);
+// Number of CTAs (partial slots) that cover work item w.
+__host__ __device__ inline int lut_item_splits(const LutPlan &P, int64_t w) {
+    if (!P.streamk) return P.splits;
+    const int64_t C = P.chunks_total, G = P.grid, U = P.units;
+    const int64_t cf = ((w * C + 1) * G - 1) / U;
+    const int64_t cl = (((w + 1) * C) * G - 1) / U;
+    return (int)(cl - cf + 1);
+}
+// CTA whose unit range contains unit u (stream-K).
+__host__ __device__ inline int64_t lut_cta_of_unit(const LutPlan &P, int64_t u) {
+    return ((u + 1) * (int64_t)P.grid - 1) / P.units;
+}
+// Work item holding output row p (relative to the launch) and column n
+// (stream-K launches, whose groups are uniform).
+__host__ __device__ inline int64_t lut_item_of(const LutPlan &P, int64_t p, int n) {
+    const int tt = 8 * P.nt;
+    const int64_t tpg = (P.uniform_rows + tt - 1) / tt;
+    const int64_t g = p / P.uniform_rows;
+    const int64_t tile = g * tpg + (p - g * P.uniform_rows) / tt;
+    return tile * P.n_row_tiles + n / P.rows_per_rt;
+}
+// Partial-slot count for output (row p, column n) of a launch.
+__host__ __device__ inline int lut_splits_at(const LutPlan &P, int64_t p, int n) {
+    return P.streamk ? lut_item_splits(P, lut_item_of(P, p, n)) : P.splits;
+}
+
+// uniform_rows > 0: the launch has n_groups groups of uniform_rows rows each
+// (dense / shared experts) and may use stream-K; otherwise the groups come
+// from device arrays and est_tiles estimates the token tiles.
+LutPlan plan_lut(int N, int K, bool dual, int max_rows_per_group, int64_t est_tiles,
+                 int uniform_rows = 0, int n_groups = 1);
 cudaError_t launch_lut(const LutLaunch &L, const LutPlan &P, cudaStream_t st);
 
-// y[m, n] = s[m] * sum_s part[s][m][n]
-cudaError_t launch_reduce_plain(const float *part, int splits, int64_t M, int64_t N,
+// y[m, n] = s[m] * sum_{s < n(m, n)} part[s][m][n]
+cudaError_t launch_reduce_plain(const float *part, const LutPlan &P, int64_t M, int64_t N,
                                 const float *s, float *y, cudaStream_t st);
 
 cudaError_t launch_centroid_sums(const void *q, int64_t M, int64_t K, int bits,

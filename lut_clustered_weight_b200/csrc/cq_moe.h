@@ -4,15 +4,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "cq_internal.h"
+
 namespace cq {
 
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 16;
 
 struct SwigluArgs {
-    const float *part_r;   // [splits_r][R_routed][I][2]
-    const float *part_s;   // [splits_s][R_shared][I_shared][2]
-    int splits_r, splits_s;
+    const float *part_r;   // [slots][R_routed][I][2]
+    const float *part_s;   // [slots][R_shared][I_shared][2]
+    LutPlan plan_r, plan_s;  // partial-slot counts of the gate/up launches
     int64_t R_routed, R_shared;
     int I, I_shared, Imax;
     int log2b_i, log2b_i_shared;
@@ -27,9 +29,9 @@ struct SwigluArgs {
 };
 
 struct CombineArgs {
-    const float *part_r;   // [splits_r][R_routed][H]
-    const float *part_s;   // [splits_s][R_shared][H]
-    int splits_r, splits_s;
+    const float *part_r;   // [slots][R_routed][H]
+    const float *part_s;   // [slots][R_shared][H]
+    LutPlan plan_r, plan_s;  // partial-slot counts of the down launches
     int64_t R_routed, R_shared;
     int T, H, topk, n_shared;
     const int32_t *inv_perm;  // slot -> routed row

@@ -25,12 +25,11 @@
 #include "cq_common.cuh"
 #include "cq_internal.h"
 
+#include <algorithm>
+
 namespace cq {
 
-constexpr int kLutThreads = 128;
 constexpr int kTokTile = 16;  // largest token tile (two n8 MMA tiles)
-constexpr int kPrefetch = 4;  // 128-k chunks in flight per lane
-constexpr size_t kLutSmemCap = 96 * 1024;
 
 // Byte-plane tables of one codebook row: lo[j] holds the low bytes of
 // C[4j..4j+3], hi[j] the high bytes.
@@ -73,194 +72,264 @@ CQ_DEV void dequant8(uint32_t w, const uint32_t (&lo)[4], const uint32_t (&hi)[4
 
 CQ_DEV __half code_to_half(int v) { return __short2half_rn((short)v); }
 
-template <int NT>
-__global__ void __launch_bounds__(kLutThreads) k_lut_mma(LutLaunch L, LutPlan P) {
+CQ_DEV void cp_async16(void *smem_dst, const void *gsrc) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+CQ_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+CQ_DEV void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+constexpr int kStages = 6;  // per-lane cp.async ring: kStages-1 chunks in flight
+
+// One CTA = W warps.  Shared memory: the activation fragments of the chunk
+// range being processed ([cps_max][8 mma][NT][32 lanes] x 4 fp16), then the
+// weight ring ([kStages][W warps][row A/B][32 lanes] x 16 bytes).  Every lane
+// copies exactly the 16 bytes it will consume, so a lane only waits for its
+// own copies (cp.async.wait_group) and reads are conflict-free.
+template <int NT, int W>
+__global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLaunch L,
+                                                                    const LutPlan P) {
+    constexpr int TT = 8 * NT;  // token rows per tile
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint2 *bfrag = reinterpret_cast<uint2 *>(smem_raw);
+    uint4 *ring = reinterpret_cast<uint4 *>(smem_raw + (size_t)P.cps_max * NT * 2048);
     __shared__ int s_code_row[kTokTile];
     __shared__ float s_scale[kTokTile];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int row_tile = blockIdx.x % P.n_row_tiles;
-    const int split = blockIdx.x / P.n_row_tiles;
-    const int tile = blockIdx.y;
-
-    // ---- which group / token tile
-    int g, row0, nrows;
-    constexpr int TT = 8 * NT;  // token rows per tile
-    if (L.uniform_rows > 0) {
-        const int tpg = (L.uniform_rows + TT - 1) / TT;
-        g = tile / tpg;
-        if (g >= L.G) return;
-        row0 = g * L.uniform_rows + (tile - g * tpg) * TT;
-        nrows = min(TT, (g + 1) * L.uniform_rows - row0);
-    } else {
-        if (tile >= L.grp_tiles[L.G]) return;
-        int lo = 0, hi = L.G;  // largest g with grp_tiles[g] <= tile
-        while (hi - lo > 1) {
-            int mid = (lo + hi) >> 1;
-            if (L.grp_tiles[mid] <= tile) lo = mid; else hi = mid;
-        }
-        g = lo;
-        row0 = L.grp_rows[g] + (tile - L.grp_tiles[g]) * TT;
-        nrows = min(TT, L.grp_rows[g + 1] - row0);
-    }
-    const int ch0 = split * P.chunks_per_split;
-    const int ch1 = min(ch0 + P.chunks_per_split, P.chunks_total);
-    const int nch = ch1 - ch0;
-    if (nch <= 0 || nrows <= 0) return;
+    const int gq = lane >> 2, cl = lane & 3;
     const int K = L.K;
+    const int C = P.chunks_total;
+    const int64_t rowbytes = K / 2;
+    const int tailc = (K & 127) >> 5;  // valid 32-k slices of a ragged last chunk
 
-    if (tid < TT) {
-        int cr = -1;
-        if (tid < nrows) {
-            const int p = row0 + tid;
-            cr = L.map_mode == kMapPerm ? L.perm[p] / L.topk
-               : L.map_mode == kMapModT ? p % L.T : p;
-        }
-        s_code_row[tid] = cr;
-        s_scale[tid] = (cr >= 0 && L.direct) ? L.scales[cr] : 0.0f;
+    // ---- this CTA's range of units (work item * C + chunk)
+    int64_t u, u_end;
+    int fixed_split = 0;
+    if (P.streamk) {
+        u = (int64_t)blockIdx.x * P.units / P.grid;
+        u_end = ((int64_t)blockIdx.x + 1) * P.units / P.grid;
+    } else {
+        const int rt = blockIdx.x % P.n_row_tiles;
+        fixed_split = blockIdx.x / P.n_row_tiles;
+        const int64_t w = (int64_t)blockIdx.y * P.n_row_tiles + rt;
+        u = w * C + (int64_t)fixed_split * P.chunks_per_split;
+        u_end = min(u + P.chunks_per_split, w * C + C);
     }
-    __syncthreads();
 
-    // ---- activation fragments for chunks [ch0, ch1): 8 consecutive k per item
-    const int items = NT * 8 * nch * 16;
-    for (int it = tid; it < items; it += kLutThreads) {
-        const int j = it / (nch * 16);
-        const int rem = it - j * (nch * 16);
-        const int ch = rem >> 4, o8 = rem & 15;
-        const int k = (ch0 + ch) * 128 + o8 * 8;
-        const int cr = s_code_row[j];
-        __align__(8) __half v[8];
+    float acc[NT][4];
+    int64_t cur_w = -1;
+    int cur_s = 0, row0 = 0, nrows = 0, nA = 0, nB = 0;
+    const uint8_t *pA = nullptr, *pB = nullptr;
+    uint32_t loA[4], hiA[4], loB[4], hiB[4];
+
+    auto flush = [&]() {
+        float *out = L.out + (int64_t)cur_s * L.out_split_stride;
 #pragma unroll
-        for (int e = 0; e < 8; e++) v[e] = __ushort_as_half(0);
-        if (cr >= 0 && k < K) {
-            if (L.act_bits == 4) {
-                const uint32_t w = *reinterpret_cast<const uint32_t *>(
-                    L.codes + (int64_t)cr * L.ld_codes + k / 2);
+        for (int t = 0; t < NT; t++) {
 #pragma unroll
-                for (int e = 0; e < 8; e++) v[e] = code_to_half(((int)(w << (28 - 4 * e))) >> 28);
-            } else {
-                const uint2 w = *reinterpret_cast<const uint2 *>(
-                    L.codes + (int64_t)cr * L.ld_codes + k);
-#pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    v[e] = code_to_half(((int)(w.x << (24 - 8 * e))) >> 24);
-                    v[4 + e] = code_to_half(((int)(w.y << (24 - 8 * e))) >> 24);
+            for (int e = 0; e < 2; e++) {
+                const int tok = 8 * t + 2 * cl + e;
+                if (tok < nrows) {
+                    const int64_t p = row0 + tok;
+                    if (L.dual) {
+                        *reinterpret_cast<float2 *>(out + p * L.out_row_stride + 2 * nA) =
+                            make_float2(acc[t][e], acc[t][2 + e]);
+                    } else if (L.direct) {
+                        const float sc = s_scale[tok];
+                        out[p * L.out_row_stride + nA] = sc * acc[t][e];
+                        out[p * L.out_row_stride + nB] = sc * acc[t][2 + e];
+                    } else {
+                        out[p * L.out_row_stride + nA] = acc[t][e];
+                        out[p * L.out_row_stride + nB] = acc[t][2 + e];
+                    }
                 }
             }
         }
-        const int c = o8 >> 2, i = 2 * (o8 & 3);
-        const int ln = 4 * (j & 7) + c, nt = j >> 3;
-        const uint2 *vv = reinterpret_cast<const uint2 *>(v);
-        bfrag[((ch * 8 + i) * NT + nt) * 32 + ln] = vv[0];
-        bfrag[((ch * 8 + i + 1) * NT + nt) * 32 + ln] = vv[1];
-    }
-    __syncthreads();
+    };
 
-    // ---- this lane's two weight rows
-    const int gq = lane >> 2, cl = lane & 3;
-    const int64_t rowbytes = K / 2;
-    const uint8_t *pA, *pB;
-    const __half *cA, *cB;
-    int nA, nB;
-    if (L.dual) {
-        nA = nB = row_tile * 32 + warp * 8 + gq;
-        pA = L.idx0 + (int64_t)g * L.w_stride + (int64_t)nA * rowbytes;
-        pB = L.idx1 + (int64_t)g * L.w_stride + (int64_t)nB * rowbytes;
-        cA = reinterpret_cast<const __half *>(L.cb0) + (int64_t)g * L.cb_stride + nA * 16;
-        cB = reinterpret_cast<const __half *>(L.cb1) + (int64_t)g * L.cb_stride + nB * 16;
-    } else {
-        nA = row_tile * 64 + warp * 16 + gq;
-        nB = nA + 8;
-        pA = L.idx0 + (int64_t)g * L.w_stride + (int64_t)nA * rowbytes;
-        pB = pA + 8 * rowbytes;
-        cA = reinterpret_cast<const __half *>(L.cb0) + (int64_t)g * L.cb_stride + nA * 16;
-        cB = cA + 8 * 16;
-    }
-    uint32_t loA[4], hiA[4], loB[4], hiB[4];
-    build_tables(cA, loA, hiA);
-    build_tables(cB, loB, hiB);
-
-    float acc[NT][4];
-#pragma unroll
-    for (int t = 0; t < NT; t++)
-#pragma unroll
-        for (int e = 0; e < 4; e++) acc[t][e] = 0.0f;
-
-    // lanes whose 32-k slice lies beyond K (ragged last chunk) read nothing;
-    // their activations are zero so index 0 contributes nothing
-    const int tailc = (K & 127) >> 5;  // valid 32-k slices in a ragged last chunk
-    auto load = [&](int ch, uint4 &a, uint4 &b) {
-        const int gch = ch0 + ch;
-        const bool ok = !(gch == P.chunks_total - 1 && tailc != 0 && cl >= tailc);
+    uint4 *my_slots = ring + (size_t)warp * 64 + lane;  // + (slot * W * 64) + r * 32
+    auto issue = [&](int gch, int slot) {
+        const bool ok = !(gch == C - 1 && tailc != 0 && cl >= tailc);
         if (ok) {
-            a = ldg_stream(pA + (int64_t)gch * 64 + cl * 16);
-            b = ldg_stream(pB + (int64_t)gch * 64 + cl * 16);
-        } else {
-            a = make_uint4(0, 0, 0, 0);
-            b = make_uint4(0, 0, 0, 0);
+            uint4 *dst = my_slots + (size_t)slot * W * 64;
+            cp_async16(dst, pA + (int64_t)gch * 64 + cl * 16);
+            cp_async16(dst + 32, pB + (int64_t)gch * 64 + cl * 16);
         }
     };
 
-    uint4 ra[kPrefetch], rb[kPrefetch];
+    while (u < u_end) {
+        const int64_t w = u / C;
+        const int ch_lo = (int)(u - w * C);
+        const int ch_hi = (int)min((int64_t)C, ch_lo + min(u_end - u, (int64_t)P.cps_max));
+        const int nch = ch_hi - ch_lo;
+        const bool new_item = (w != cur_w);
+        if (new_item) {
+            if (cur_w >= 0) flush();
+            const int64_t tile = w / P.n_row_tiles;
+            const int rt = (int)(w - tile * P.n_row_tiles);
+            int g;
+            if (L.uniform_rows > 0) {
+                const int tpg = (L.uniform_rows + TT - 1) / TT;
+                g = (int)(tile / tpg);
+                row0 = g * L.uniform_rows + (int)(tile - (int64_t)g * tpg) * TT;
+                nrows = min(TT, (g + 1) * L.uniform_rows - row0);
+            } else {
+                if (tile >= L.grp_tiles[L.G]) return;  // beyond the routed tiles (fixed mode)
+                int lo = 0, hi = L.G;  // largest g with grp_tiles[g] <= tile
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (L.grp_tiles[mid] <= tile) lo = mid; else hi = mid;
+                }
+                g = lo;
+                row0 = L.grp_rows[g] + (int)(tile - L.grp_tiles[g]) * TT;
+                nrows = min(TT, L.grp_rows[g + 1] - row0);
+            }
+            cur_w = w;
+            cur_s = P.streamk ? (int)(blockIdx.x - lut_cta_of_unit(P, w * C)) : fixed_split;
+            const __half *cA, *cB;
+            if (L.dual) {
+                nA = nB = rt * P.rows_per_rt + warp * 8 + gq;
+                pA = L.idx0 + (int64_t)g * L.w_stride + (int64_t)nA * rowbytes;
+                pB = L.idx1 + (int64_t)g * L.w_stride + (int64_t)nB * rowbytes;
+                cA = reinterpret_cast<const __half *>(L.cb0) + (int64_t)g * L.cb_stride + nA * 16;
+                cB = reinterpret_cast<const __half *>(L.cb1) + (int64_t)g * L.cb_stride + nB * 16;
+            } else {
+                nA = rt * P.rows_per_rt + warp * 16 + gq;
+                nB = nA + 8;
+                pA = L.idx0 + (int64_t)g * L.w_stride + (int64_t)nA * rowbytes;
+                pB = pA + 8 * rowbytes;
+                cA = reinterpret_cast<const __half *>(L.cb0) + (int64_t)g * L.cb_stride + nA * 16;
+                cB = cA + 8 * 16;
+            }
+            // weight stream first, so HBM latency overlaps the set-up below
 #pragma unroll
-    for (int p = 0; p < kPrefetch; p++)
-        if (p < nch) load(p, ra[p], rb[p]);
+            for (int sl = 0; sl < kStages - 1; sl++) {
+                if (sl < nch) issue(ch_lo + sl, sl);
+                cp_async_commit();
+            }
+            build_tables(cA, loA, hiA);
+            build_tables(cB, loB, hiB);
+#pragma unroll
+            for (int t = 0; t < NT; t++)
+#pragma unroll
+                for (int e = 0; e < 4; e++) acc[t][e] = 0.0f;
+            __syncthreads();  // previous piece is done with s_code_row / bfrag
+            if (tid < TT) {
+                int cr = -1;
+                if (tid < nrows) {
+                    const int p = row0 + tid;
+                    cr = L.map_mode == kMapPerm ? L.perm[p] / L.topk
+                       : L.map_mode == kMapModT ? p % L.T : p;
+                }
+                s_code_row[tid] = cr;
+                s_scale[tid] = (cr >= 0 && L.direct) ? L.scales[cr] : 0.0f;
+            }
+        } else {
+#pragma unroll
+            for (int sl = 0; sl < kStages - 1; sl++) {
+                if (sl < nch) issue(ch_lo + sl, sl);
+                cp_async_commit();
+            }
+        }
+        __syncthreads();  // s_code_row visible; bfrag free
 
-    for (int base = 0; base < nch; base += kPrefetch) {
+        // ---- activation fragments for chunks [ch_lo, ch_hi).  An item is the
+        // 32 consecutive k of one token that one lane consumes (lane = 4*(token
+        // % 8) + k-slice); consecutive threads write consecutive lanes, and each
+        // thread issues the wide loads of up to 4 items before converting.
+        {
+            const int items = nch * NT * 32;  // (chunk, n8 tile, lane)
+            constexpr int FB = 4;
+            for (int it0 = tid; it0 < items; it0 += FB * W * 32) {
+                uint4 raw[FB][2];
 #pragma unroll
-        for (int p = 0; p < kPrefetch; p++) {
-            const int ch = base + p;
-            if (ch < nch) {
-                const uint32_t wa[4] = {ra[p].x, ra[p].y, ra[p].z, ra[p].w};
-                const uint32_t wb[4] = {rb[p].x, rb[p].y, rb[p].z, rb[p].w};
-                if (ch + kPrefetch < nch) load(ch + kPrefetch, ra[p], rb[p]);
-                const uint2 *bf = bfrag + (size_t)ch * 8 * NT * 32 + lane;
+                for (int f = 0; f < FB; f++) {
+                    raw[f][0] = raw[f][1] = make_uint4(0, 0, 0, 0);
+                    const int it = it0 + f * W * 32;
+                    if (it < items) {
+                        const int ln = it & 31, nt = (it >> 5) % NT, ch = (it >> 5) / NT;
+                        const int cr = s_code_row[8 * nt + (ln >> 2)];
+                        const int k0 = (ch_lo + ch) * 128 + 32 * (ln & 3);
+                        if (cr >= 0 && k0 < K) {
+                            const uint8_t *src = L.codes + (int64_t)cr * L.ld_codes;
+                            if (L.act_bits == 4) {
+                                raw[f][0] = *reinterpret_cast<const uint4 *>(src + k0 / 2);
+                            } else {
+                                raw[f][0] = *reinterpret_cast<const uint4 *>(src + k0);
+                                raw[f][1] = *reinterpret_cast<const uint4 *>(src + k0 + 16);
+                            }
+                        }
+                    }
+                }
 #pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    uint32_t hA[4], hB[4];
-                    dequant8(wa[j], loA, hiA, hA);
-                    dequant8(wb[j], loB, hiB, hB);
+                for (int f = 0; f < FB; f++) {
+                    const int it = it0 + f * W * 32;
+                    if (it < items) {
+                        const int ln = it & 31, nt = (it >> 5) % NT, ch = (it >> 5) / NT;
+                        const uint32_t wd[8] = {raw[f][0].x, raw[f][0].y, raw[f][0].z,
+                                                raw[f][0].w, raw[f][1].x, raw[f][1].y,
+                                                raw[f][1].z, raw[f][1].w};
 #pragma unroll
-                    for (int hh = 0; hh < 2; hh++) {
-                        const int i = 2 * j + hh;
-                        const uint32_t af[4] = {hA[2 * hh], hB[2 * hh], hA[2 * hh + 1],
-                                                hB[2 * hh + 1]};
+                        for (int i = 0; i < 8; i++) {
+                            // codes of k0 + 4i .. k0 + 4i + 3
+                            __align__(8) __half v[4];
+                            if (L.act_bits == 4) {
+                                const uint32_t x = wd[i >> 1] >> (16 * (i & 1));
 #pragma unroll
-                        for (int t = 0; t < NT; t++) {
-                            const uint2 bv = bf[(i * NT + t) * 32];
-                            mma_16816(acc[t], af, bv.x, bv.y);
+                                for (int e = 0; e < 4; e++)
+                                    v[e] = code_to_half(((int)(x << (28 - 4 * e))) >> 28);
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 4; e++)
+                                    v[e] = code_to_half(((int)(wd[i] << (24 - 8 * e))) >> 24);
+                            }
+                            bfrag[((ch * 8 + i) * NT + nt) * 32 + ln] =
+                                *reinterpret_cast<const uint2 *>(v);
                         }
                     }
                 }
             }
         }
-    }
+        __syncthreads();
 
-    // ---- epilogue: acc[t][0..1] row A, tokens 8t + 2cl + {0,1}; acc[t][2..3] row B
-    float *out = L.out + (int64_t)split * L.out_split_stride;
+        // ---- the chunk pipeline
+        for (int ch = 0; ch < nch; ch++) {
+            cp_async_wait<kStages - 2>();
+            const int gch = ch_lo + ch;
+            const bool ok = !(gch == C - 1 && tailc != 0 && cl >= tailc);
+            const uint4 *src = my_slots + (size_t)(ch % kStages) * W * 64;
+            uint4 ra = ok ? src[0] : make_uint4(0, 0, 0, 0);
+            uint4 rb = ok ? src[32] : make_uint4(0, 0, 0, 0);
+            if (ch + kStages - 1 < nch) issue(gch + kStages - 1, (ch + kStages - 1) % kStages);
+            cp_async_commit();
+            const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+            const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+            const uint2 *bf = bfrag + (size_t)ch * 8 * NT * 32 + lane;
 #pragma unroll
-    for (int t = 0; t < NT; t++) {
+            for (int j = 0; j < 4; j++) {
+                uint32_t hA[4], hB[4];
+                dequant8(wa[j], loA, hiA, hA);
+                dequant8(wb[j], loB, hiB, hB);
 #pragma unroll
-        for (int e = 0; e < 2; e++) {
-            const int tok = 8 * t + 2 * cl + e;
-            if (tok < nrows) {
-                const int64_t p = row0 + tok;
-                if (L.dual) {
-                    *reinterpret_cast<float2 *>(out + p * L.out_row_stride + 2 * nA) =
-                        make_float2(acc[t][e], acc[t][2 + e]);
-                } else if (L.direct) {
-                    const float s = s_scale[tok];
-                    out[p * L.out_row_stride + nA] = s * acc[t][e];
-                    out[p * L.out_row_stride + nB] = s * acc[t][2 + e];
-                } else {
-                    out[p * L.out_row_stride + nA] = acc[t][e];
-                    out[p * L.out_row_stride + nB] = acc[t][2 + e];
+                for (int hh = 0; hh < 2; hh++) {
+                    const int i = 2 * j + hh;
+                    const uint32_t af[4] = {hA[2 * hh], hB[2 * hh], hA[2 * hh + 1],
+                                            hB[2 * hh + 1]};
+#pragma unroll
+                    for (int t = 0; t < NT; t++) {
+                        const uint2 bv = bf[(i * NT + t) * 32];
+                        mma_16816(acc[t], af, bv.x, bv.y);
+                    }
                 }
             }
         }
+        u += nch;
     }
+    if (cur_w >= 0) flush();
 }
 
 int sm_count() {
@@ -270,62 +339,91 @@ int sm_count() {
     return n;
 }
 
-LutPlan plan_lut(int N, int K, bool dual, int max_rows_per_group, int64_t est_tiles) {
-    LutPlan P;
+LutPlan plan_lut(int N, int K, bool dual, int max_rows_per_group, int64_t est_tiles,
+                 int uniform_rows, int n_groups) {
+    LutPlan P{};
     P.nt = max_rows_per_group <= 8 ? 1 : 2;
-    P.n_row_tiles = dual ? N / 32 : N / 64;
+    const int tt = 8 * P.nt;
+    // 8 warps when the row tile divides N, else 4
+    P.warps = (dual ? N % 64 == 0 : N % 128 == 0) ? 8 : 4;
+    P.rows_per_rt = dual ? 8 * P.warps : 16 * P.warps;
+    P.n_row_tiles = N / P.rows_per_rt;
     P.chunks_total = (K + 127) / 128;
-    const size_t per_chunk = (size_t)P.nt * 8 * 128 * 2;  // fp16 fragments
-    const int max_cps = (int)(kLutSmemCap / per_chunk);
-    // aim for ~3 resident CTAs per SM worth of independent CTAs
-    const int64_t target = (int64_t)sm_count() * 3;
-    const int64_t base = (int64_t)P.n_row_tiles * (est_tiles > 0 ? est_tiles : 1);
-    int splits = (int)((target + base - 1) / base);
-    if (splits < 1) splits = 1;
-    const int min_splits = (P.chunks_total + max_cps - 1) / max_cps;
-    if (splits < min_splits) splits = min_splits;
-    if (splits > P.chunks_total) splits = P.chunks_total;
-    P.chunks_per_split = (P.chunks_total + splits - 1) / splits;
-    P.splits = (P.chunks_total + P.chunks_per_split - 1) / P.chunks_per_split;
-    P.smem = per_chunk * P.chunks_per_split;
+    const int ctas_per_sm = P.warps == 8 ? 2 : 4;  // what __launch_bounds__ and smem allow
+    const size_t smem_cap = (size_t)(227 * 1024) / ctas_per_sm - 1024;
+    const size_t ring = (size_t)kStages * P.warps * 1024;
+    const size_t per_chunk = (size_t)P.nt * 2048;
+    P.cps_max = (int)std::min<size_t>(32, (smem_cap - ring) / per_chunk);
+    const int capacity = sm_count() * ctas_per_sm;
+    const int C = P.chunks_total;
+    if (uniform_rows > 0) {
+        const int64_t tiles = (int64_t)n_groups * ((uniform_rows + tt - 1) / tt);
+        P.streamk = 1;
+        P.uniform_rows = uniform_rows;
+        P.units = tiles * P.n_row_tiles * C;
+        P.grid = (int)std::min<int64_t>(capacity, P.units);
+        // partial slots: the most CTAs that share one work item
+        int smax = 1;
+        const int64_t items = tiles * P.n_row_tiles;
+        for (int64_t w = 0; w < items; w++) smax = std::max(smax, lut_item_splits(P, w));
+        P.splits = smax;
+        P.chunks_per_split = P.cps_max;
+    } else {
+        P.streamk = 0;
+        const int64_t base = (int64_t)P.n_row_tiles * std::max<int64_t>(est_tiles, 1);
+        int splits = base < capacity ? (int)(capacity / base) : 1;
+        const int min_splits = (C + P.cps_max - 1) / P.cps_max;
+        splits = std::max(std::min(splits, C), min_splits);
+        P.chunks_per_split = (C + splits - 1) / splits;
+        P.splits = (C + P.chunks_per_split - 1) / P.chunks_per_split;
+        P.grid = P.n_row_tiles * P.splits;
+        P.cps_max = P.chunks_per_split;  // the activation region holds one split
+    }
+    P.smem = ring + per_chunk * P.cps_max;
     return P;
 }
 
+template <int NT, int W>
+static cudaError_t launch_lut_t(const LutLaunch &L, const LutPlan &P, cudaStream_t st) {
+    cudaFuncSetAttribute(k_lut_mma<NT, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)P.smem);
+    dim3 grid(P.grid, P.streamk ? 1 : L.max_tiles);
+    k_lut_mma<NT, W><<<grid, W * 32, P.smem, st>>>(L, P);
+    return cudaSuccess;
+}
+
 cudaError_t launch_lut(const LutLaunch &L, const LutPlan &P, cudaStream_t st) {
-    dim3 grid(P.n_row_tiles * P.splits, L.max_tiles);
-    if (grid.y == 0 || grid.x == 0) return cudaSuccess;
+    if (P.grid == 0 || (!P.streamk && L.max_tiles == 0)) return cudaSuccess;
     const bool timed = timing_on();
     if (timed) timing_begin(st);
     count_launch();
-    if (P.nt == 1) {
-        cudaFuncSetAttribute(k_lut_mma<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kLutSmemCap);
-        k_lut_mma<1><<<grid, kLutThreads, P.smem, st>>>(L, P);
-    } else {
-        cudaFuncSetAttribute(k_lut_mma<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kLutSmemCap);
-        k_lut_mma<2><<<grid, kLutThreads, P.smem, st>>>(L, P);
-    }
+    if (P.nt == 1)
+        P.warps == 8 ? launch_lut_t<1, 8>(L, P, st) : launch_lut_t<1, 4>(L, P, st);
+    else
+        P.warps == 8 ? launch_lut_t<2, 8>(L, P, st) : launch_lut_t<2, 4>(L, P, st);
     if (timed) timing_end(st);
     return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- split-K reduce
-__global__ void k_reduce_plain(const float *__restrict__ part, int splits, int64_t M, int64_t N,
-                               const float *__restrict__ s, float *__restrict__ y) {
+__global__ void k_reduce_plain(const float *__restrict__ part, const LutPlan P, int64_t M,
+                               int64_t N, const float *__restrict__ s, float *__restrict__ y) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= M * N) return;
+    const int64_t m = i / N;
+    const int n = (int)(i - m * N);
+    const int ns = lut_splits_at(P, m, n);
     float acc = 0.0f;
-    for (int k = 0; k < splits; k++) acc += part[(int64_t)k * M * N + i];
-    y[i] = s[i / N] * acc;
+    for (int k = 0; k < ns; k++) acc += part[(int64_t)k * M * N + i];
+    y[i] = s[m] * acc;
 }
 
-cudaError_t launch_reduce_plain(const float *part, int splits, int64_t M, int64_t N,
+cudaError_t launch_reduce_plain(const float *part, const LutPlan &P, int64_t M, int64_t N,
                                 const float *s, float *y, cudaStream_t st) {
     const int64_t n = M * N;
     if (n == 0) return cudaSuccess;
     count_launch();
-    k_reduce_plain<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, splits, M, N, s, y);
+    k_reduce_plain<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, P, M, N, s, y);
     return cudaGetLastError();
 }
 

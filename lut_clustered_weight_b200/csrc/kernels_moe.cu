@@ -1,52 +1,10 @@
-// kernels_moe.cu -- rotate+quantize, routing / expert grouping, SwiGLU and
-// combine kernels of the CodeQuant MoE linear layer (sm_100a).
+// kernels_moe.cu -- routing / expert grouping and combine kernels of the
+// CodeQuant MoE linear layer (sm_100a).
 #include "cq_common.cuh"
 #include "cq_internal.h"
 #include "cq_moe.h"
-#include "rotate_quantize.cuh"
 
 namespace cq {
-
-constexpr int kRqThreads = 256;
-
-// ------------------------------------------------------------------ rotate + quantize
-// One CTA per token row: load fp16 -> fp64 in shared memory, exact block
-// Walsh-Hadamard, exact absmax, exact round-half-even codes.
-__global__ void __launch_bounds__(kRqThreads)
-k_rotate_quantize(const __half *__restrict__ x, int64_t ldx, int K, int log2b, int bits,
-                  uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s) {
-    extern __shared__ __align__(16) double buf[];
-    __shared__ double red[33];
-    const int64_t m = blockIdx.x;
-    const __half *xr = x + m * ldx;
-    for (int i = threadIdx.x; i < K / 8; i += kRqThreads) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(xr + 8 * i);
-        const __half2 *h = reinterpret_cast<const __half2 *>(&v);
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const float2 f = __half22float2(h[j]);
-            buf[8 * i + 2 * j] = (double)f.x;
-            buf[8 * i + 2 * j + 1] = (double)f.y;
-        }
-    }
-    __syncthreads();
-    block_fwht<kRqThreads>(buf, K, log2b);
-    const double A = block_absmax<kRqThreads>(buf, K, red);
-    block_quantize_store<kRqThreads>(buf, K, log2b, bits, A, q + m * ldq, s + m);
-}
-
-cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K, int log2b,
-                                   int bits, void *q, int64_t ldq, float *s, cudaStream_t st) {
-    if (M == 0) return cudaSuccess;
-    const size_t smem = (size_t)K * sizeof(double);
-    cudaFuncSetAttribute(k_rotate_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)(kMaxK * sizeof(double)));
-    count_launch();
-    k_rotate_quantize<<<(unsigned)M, kRqThreads, smem, st>>>(
-        reinterpret_cast<const __half *>(x), ldx, K, log2b, bits,
-        reinterpret_cast<uint8_t *>(q), ldq, s);
-    return cudaGetLastError();
-}
 
 // ------------------------------------------------------------------ routing
 // One CTA (1024 threads).  Top-k per token (one warp per token, descending,
@@ -184,55 +142,6 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
     return cudaGetLastError();
 }
 
-// ------------------------------------------------------------------ SwiGLU + rotate + quantize
-// One CTA per row of the intermediate: sum the split-K partials of g and u,
-// scale by the token's s_x, h = fp16(silu(g) * u), then the exact rotation
-// over I and per-row quantization of h.
-__global__ void __launch_bounds__(kRqThreads)
-k_swiglu_rq(SwigluArgs a) {
-    extern __shared__ __align__(16) double buf[];
-    __shared__ double red[33];
-    const int64_t p = blockIdx.x;
-    const bool routed = p < a.R_routed;
-    const int I = routed ? a.I : a.I_shared;
-    const int log2b = routed ? a.log2b_i : a.log2b_i_shared;
-    const float *part = routed ? a.part_r : a.part_s;
-    const int splits = routed ? a.splits_r : a.splits_s;
-    const int64_t rows = routed ? a.R_routed : a.R_shared;
-    const int64_t lp = routed ? p : p - a.R_routed;
-    const int tok = routed ? a.perm[p] / a.topk : (int)(lp % a.T);
-    const float sx = a.x_scales[tok];
-    for (int n = threadIdx.x; n < I; n += kRqThreads) {
-        float g = 0.0f, u = 0.0f;
-        for (int sp = 0; sp < splits; sp++) {
-            const float2 v = *reinterpret_cast<const float2 *>(
-                part + ((int64_t)sp * rows + lp) * (2 * (int64_t)I) + 2 * n);
-            g += v.x;
-            u += v.y;
-        }
-        g *= sx;
-        u *= sx;
-        const __half h = __float2half_rn(silu_mul(g, u));
-        if (a.h_dbg) reinterpret_cast<__half *>(a.h_dbg)[p * a.Imax + n] = h;
-        buf[n] = (double)__half2float(h);
-    }
-    __syncthreads();
-    block_fwht<kRqThreads>(buf, I, log2b);
-    const double A = block_absmax<kRqThreads>(buf, I, red);
-    block_quantize_store<kRqThreads>(buf, I, log2b, a.bits, A, a.hq + p * a.ldhq,
-                                     a.h_scales + p);
-}
-
-cudaError_t launch_swiglu_rq(const SwigluArgs &a, int64_t rows, cudaStream_t st) {
-    if (rows == 0) return cudaSuccess;
-    const int Imax = a.Imax;
-    cudaFuncSetAttribute(k_swiglu_rq, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)(kMaxK * sizeof(double)));
-    count_launch();
-    k_swiglu_rq<<<(unsigned)rows, kRqThreads, (size_t)Imax * sizeof(double), st>>>(a);
-    return cudaGetLastError();
-}
-
 // ------------------------------------------------------------------ combine
 // out[t, n] = sum_j w[t,j] * s_h[p] * sum_split part[split][p][n]  (j in order)
 //           + sum_s s_h[ps] * sum_split part_s[split][ps][n]
@@ -244,7 +153,7 @@ __global__ void k_combine(CombineArgs a) {
     for (int j = 0; j < a.topk; j++) {
         const int p = a.inv_perm[t * a.topk + j];
         float y = 0.0f;
-        for (int sp = 0; sp < a.splits_r; sp++)
+        for (int sp = 0; sp < a.plan_r.splits; sp++)
             y += a.part_r[((int64_t)sp * a.R_routed + p) * a.H + n];
         y *= a.h_scales[p];
         if (a.y_dbg) a.y_dbg[(int64_t)p * a.H + n] = y;
@@ -253,7 +162,8 @@ __global__ void k_combine(CombineArgs a) {
     for (int s = 0; s < a.n_shared; s++) {
         const int64_t lp = (int64_t)s * a.T + t;
         float y = 0.0f;
-        for (int sp = 0; sp < a.splits_s; sp++)
+        const int ns = lut_splits_at(a.plan_s, lp, n);
+        for (int sp = 0; sp < ns; sp++)
             y += a.part_s[((int64_t)sp * a.R_shared + lp) * a.H + n];
         y *= a.h_scales[a.R_routed + lp];
         if (a.y_dbg) a.y_dbg[(a.R_routed + lp) * a.H + n] = y;

@@ -75,16 +75,14 @@ extern "C" CQ_API cq_status cq_lut_gemm_noalloc(const void *q, const float *s_x,
     // same plan as cq_lut_gemm, so the two give the same result
     const int nt = M <= 8 ? 1 : 2;
     const int tiles = (int)((M + 8 * nt - 1) / (8 * nt));
-    const LutPlan P = plan_lut((int)N, (int)K, false, (int)std::min<int64_t>(M, 16), tiles);
-    const size_t need = P.splits > 1 ? (size_t)P.splits * M * N * sizeof(float) : 0;
+    const LutPlan P = plan_lut((int)N, (int)K, false, (int)std::min<int64_t>(M, 16), tiles,
+                               (int)M, 1);
+    const size_t need = (size_t)P.splits * M * N * sizeof(float);
     if (need > kNoAllocScratchBytes) return CQ_ERR_UNSUPPORTED;  // beyond the fixed scratch
 
-    float *scratch = nullptr;
-    if (need > 0) {
-        void *p = nullptr;
-        if (scratch_on_current_device(&p) != cudaSuccess) return CQ_ERR_CUDA;
-        scratch = reinterpret_cast<float *>(p);
-    }
+    void *p = nullptr;
+    if (scratch_on_current_device(&p) != cudaSuccess) return CQ_ERR_CUDA;
+    float *scratch = reinterpret_cast<float *>(p);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     LutLaunch L{};
     L.codes = reinterpret_cast<const uint8_t *>(q);
@@ -101,15 +99,10 @@ extern "C" CQ_API cq_status cq_lut_gemm_noalloc(const void *q, const float *s_x,
     L.N = (int)N;
     L.dual = false;
     L.out_row_stride = N;
-    if (P.splits == 1) {
-        L.direct = true;
-        L.out = y;
-    } else {
-        L.direct = false;
-        L.out = scratch;
-        L.out_split_stride = M * N;
-    }
+    L.direct = false;
+    L.out = scratch;
+    L.out_split_stride = M * N;
     cudaError_t e = launch_lut(L, P, st);
-    if (e == cudaSuccess && P.splits > 1) e = launch_reduce_plain(scratch, P.splits, M, N, s_x, y, st);
+    if (e == cudaSuccess) e = launch_reduce_plain(scratch, P, M, N, s_x, y, st);
     return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }

@@ -131,31 +131,49 @@ CQ_DEV float quant_scale(double A, int log2b, int qmax) {
                                        (double)qmax));
 }
 
-// Quantize the rotated row and store its codes: bits 4 -> K/2 packed bytes
-// (low nibble = even k), bits 8 -> K int8.  Writes the scale through s_out.
+// Code of one rotated value: round_half_even(qmax * |v| / A) with the sign
+// of v.  t = |v| * (qmax / A) in fp64 is within 3e-14 of the exact quotient
+// (which is at most 127), so unless t lies within 1e-9 of a half-integer
+// rint(t) is already the exact decision; near a half-integer the exact int64
+// rational decision is taken instead.
+CQ_DEV int quantize_fast(double v, double R, long long Ai, int qmax) {
+    const double t = fabs(v) * R;
+    const double fr = t - floor(t);
+    int q;
+    if (fabs(fr - 0.5) < 1e-9) {
+        q = quantize_exact(fabs(v), Ai, qmax);
+    } else {
+        q = (int)rint(t);
+    }
+    return v < 0 ? -q : q;
+}
+
+// Quantize buf[0, n) (rotated values of row positions [e0, e0 + n)) and
+// store the codes: bits 4 -> packed bytes (low nibble = even position),
+// bits 8 -> int8.  e0 and n are even.  A is the absmax of the whole row.
 template <int THREADS>
-__device__ void block_quantize_store(const double *buf, int K, int log2b, int bits, double A,
-                                     uint8_t *qrow, float *s_out) {
+__device__ void block_quantize_range(const double *buf, int n, int e0, int bits, double A,
+                                     uint8_t *qrow) {
     const int qmax = (1 << (bits - 1)) - 1;
     const long long Ai = __double2ll_rn(A * 16777216.0);
+    const double R = Ai > 0 ? __ddiv_rn((double)qmax, A) : 0.0;
     const double2 *b2 = reinterpret_cast<const double2 *>(buf);
-    for (int p = threadIdx.x; p < K / 2; p += THREADS) {
-        double2 v = b2[p];
+    for (int p = threadIdx.x; p < n / 2; p += THREADS) {
+        const double2 v = b2[p];
         int q0 = 0, q1 = 0;
         if (Ai > 0) {
-            q0 = quantize_exact(v.x, Ai, qmax);
-            q1 = quantize_exact(v.y, Ai, qmax);
+            q0 = quantize_fast(v.x, R, Ai, qmax);
+            q1 = quantize_fast(v.y, R, Ai, qmax);
         }
         if (bits == 4) {
-            qrow[p] = (uint8_t)((q0 & 15) | ((q1 & 15) << 4));
+            qrow[e0 / 2 + p] = (uint8_t)((q0 & 15) | ((q1 & 15) << 4));
         } else {
             char2 c;
             c.x = (char)q0;
             c.y = (char)q1;
-            reinterpret_cast<char2 *>(qrow)[p] = c;
+            reinterpret_cast<char2 *>(qrow + e0)[p] = c;
         }
     }
-    if (threadIdx.x == 0) *s_out = Ai > 0 ? quant_scale(A, log2b, qmax) : 0.0f;
 }
 
 }  // namespace cq
