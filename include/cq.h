@@ -133,8 +133,10 @@ CQ_API cq_status cq_lut_gemm(const void *q, const float *s_x, int64_t M, int64_t
  * custom-op hosts whose framework owns all device memory and exposes no
  * allocator, and serving processes that forbid cudaMalloc after start-up
  * because it synchronizes the device and fragments a pre-sized pool.  This
- * entry point computes exactly what cq_lut_gemm computes (same kernels, same
- * split of the contraction, so the same result) but keeps its split-K partial
+ * entry point computes the same product as cq_lut_gemm with the mma.sync LUT
+ * kernel (the one cq_lut_gemm uses for M <= 16, with the same split of the
+ * contraction, so for M <= 16 the results are identical; for larger M the
+ * two agree within the stated error bound), but keeps its split-K partial
  * sums in a fixed array of CQ_NOALLOC_SCRATCH_BYTES bytes compiled into the
  * library.  It calls no cudaMalloc / cudaFree and no allocating library
  * routine.
@@ -236,7 +238,7 @@ CQ_API size_t cq_moe_ffn_workspace_size(const cq_moe_desc *d, int64_t T);
  * out     fp32 [T, H]
  * dbg     NULL or a cq_moe_debug with device pointers to fill
  * Requires H % 64 == 0, I % 64 == 0, I_shared % 64 == 0 (when used),
- * H, I <= 16384, 1 <= top_k <= min(E, 16) when E > 0, E <= 1024,
+ * H, I <= 16384, 1 <= top_k <= min(E, 16) when E > 0, E <= 256, n_shared <= 4,
  * had blocks powers of two dividing their dimension, act_bits in {4, 8}.
  */
 CQ_API cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_logits, int64_t T,
@@ -257,6 +259,15 @@ CQ_API cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *ro
  * it is guarded by a mutex.  Enable it only around single-threaded use.
  */
 CQ_API int64_t cq_launch_count(void);
+
+/*
+ * cq_device_error -- the device error word: 0 if no kernel of this library
+ * stopped early since the last call, else a nonzero code (1 = a bounded wait
+ * inside a tensor-core kernel gave up; its outputs are then unspecified).
+ * Synchronizes the current device and clears the word; -1 if it could not be
+ * read.
+ */
+CQ_API int32_t cq_device_error(void);
 CQ_API cq_status cq_timing_enable(int32_t on);
 CQ_API cq_status cq_timing_read(int64_t *launches, double *total_ms);
 

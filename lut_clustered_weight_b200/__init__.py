@@ -19,7 +19,7 @@ LIB_PATH = _PKG / "libcq_b200.so"
 # symbols declared in include/cq.h
 EXPORTS = ("cq_status_string", "cq_version", "cq_rotate_quantize", "cq_lut_gemm_workspace_size",
            "cq_lut_gemm", "cq_moe_ffn_workspace_size", "cq_moe_ffn", "cq_launch_count",
-           "cq_timing_enable", "cq_timing_read", "cq_lut_gemm_noalloc")
+           "cq_timing_enable", "cq_timing_read", "cq_lut_gemm_noalloc", "cq_device_error")
 
 CQ_OK, CQ_ERR_INVALID_ARGUMENT, CQ_ERR_UNSUPPORTED, CQ_ERR_WORKSPACE, CQ_ERR_CUDA = range(5)
 
@@ -76,6 +76,8 @@ lib.cq_moe_ffn.argtypes = [ctypes.POINTER(MoEDesc), _P, _P, _I64, ctypes.POINTER
 lib.cq_moe_ffn.restype = ctypes.c_int
 lib.cq_lut_gemm_noalloc.argtypes = [_P, _P, _I64, _I64, _I32, _P, _P, _I64, _P, _P]
 lib.cq_lut_gemm_noalloc.restype = ctypes.c_int
+lib.cq_device_error.argtypes = []
+lib.cq_device_error.restype = _I32
 lib.cq_launch_count.argtypes = []
 lib.cq_launch_count.restype = _I64
 lib.cq_timing_enable.argtypes = [_I32]
@@ -87,6 +89,11 @@ lib.cq_timing_read.restype = ctypes.c_int
 def cq_launch_count() -> int:
     """Kernels launched by the library since it was loaded."""
     return int(lib.cq_launch_count())
+
+
+def cq_device_error() -> int:
+    """Device error word (0 = none); synchronizes and clears it."""
+    return int(lib.cq_device_error())
 
 
 def cq_timing_enable(on: bool = True) -> None:

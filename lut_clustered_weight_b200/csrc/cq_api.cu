@@ -28,24 +28,47 @@ struct LutGemmPlan {
     LutPlan p;
     int tiles;
     size_t ws;
+    size_t b_off;  // tensor-core path: fp16 activations at workspace + b_off
 };
+
+// Tensor-core (tcgen05) kernel for groups of more than 16 rows, mma.sync
+// with register tables for decode-sized groups.  rows = typical rows per group.
+bool use_tc(int64_t rows, int64_t N, bool dual) {
+    if (dual ? N % 64 : N % 128) return false;  // 128 weight rows per tile
+    const LutPath p = lut_path();
+    if (p != kPathAuto) return p == kPathTc;
+    return rows > 16;
+}
 
 LutGemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
     LutGemmPlan g;
+    if (use_tc(M, N, false)) {
+        const int mr = (int)std::min<int64_t>(M, 256);
+        const int ntok = tc_ntok_for(mr);
+        g.tiles = (int)((M + ntok - 1) / ntok);
+        g.p = plan_lut_tc((int)N, (int)K, false, mr, g.tiles, (int)M, 1);
+        g.b_off = align256((size_t)g.p.splits * M * N * sizeof(float));
+        g.ws = g.b_off + align256((size_t)M * K * 2);
+        return g;
+    }
     const int nt = M <= 8 ? 1 : 2;
     g.tiles = (int)((M + 8 * nt - 1) / (8 * nt));
     g.p = plan_lut((int)N, (int)K, false, (int)std::min<int64_t>(M, 16), g.tiles, (int)M, 1);
     g.ws = align256((size_t)g.p.splits * M * N * sizeof(float));
+    g.b_off = 0;
     return g;
 }
 
 // ------------------------------------------------------------------ MoE plan
 struct MoePlan {
     int64_t T, H, I, E, k, ns, Is, Rr, Rs, R;
-    int bits, Imax, nt, tile_rows, max_tiles_r, tiles_s;
+    int bits, Imax, nt, tile_rows, max_tiles_r, tiles_s, tile_rows_s;
+    bool tc_r, tc_s, tc_dn_r, tc_dn_s;  // tensor-core kernel per launch
     LutPlan gu_r, gu_s, dn_r, dn_s;
     size_t o_xq, o_sx, o_ids, o_w, o_counts, o_offsets, o_perm, o_inv, o_tiles;
-    size_t o_pgu_r, o_pgu_s, o_hq, o_sh, o_pdn_r, o_pdn_s, total;
+    size_t o_pgu_r, o_pgu_s, o_hq, o_sh, o_pdn_r, o_pdn_s;
+    size_t o_bx_r, o_bx_s, o_bh_r, o_bh_s;  // fp16 B operands of tensor-core launches
+    size_t total;
 };
 
 MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
@@ -63,20 +86,43 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
     m.bits = d->act_bits;
     m.Imax = (int)std::max<int64_t>(m.E > 0 ? m.I : 0, m.Is);
     m.nt = T <= 8 ? 1 : 2;
-    m.tile_rows = 8 * m.nt;
+    // routed experts: typical rows per expert decide the kernel and tile size
+    const int64_t avg_r = m.E > 0 ? (m.Rr + m.E - 1) / m.E : 0;
+    m.tc_r = m.E > 0 && use_tc(avg_r, m.I, true);
+    m.tc_dn_r = m.tc_r && use_tc(avg_r, m.H, false);
+    if (m.tc_r != m.tc_dn_r) m.tc_r = m.tc_dn_r = false;  // one token tiling per group
+    const int rows_r = (int)std::min<int64_t>(T, std::max<int64_t>(2 * avg_r, 1));
+    m.tile_rows = m.tc_r ? tc_ntok_for(rows_r) : 8 * m.nt;
     const int64_t nonempty = std::min<int64_t>(m.E, m.Rr);
     m.max_tiles_r = (int)(m.Rr / m.tile_rows + nonempty);
-    m.tiles_s = (int)(m.ns * ((T + m.tile_rows - 1) / m.tile_rows));
+    // shared experts: every token
+    m.tc_s = m.ns > 0 && use_tc(T, m.Is, true);
+    m.tc_dn_s = m.ns > 0 && use_tc(T, m.H, false);
+    if (m.tc_s != m.tc_dn_s) m.tc_s = m.tc_dn_s = false;
+    m.tile_rows_s = m.tc_s ? tc_ntok_for((int)std::min<int64_t>(T, 256)) : 8 * m.nt;
+    m.tiles_s = (int)(m.ns * ((T + m.tile_rows_s - 1) / m.tile_rows_s));
     const int rows_per_group = (int)std::min<int64_t>(T, 16);
     if (m.E > 0) {
-        m.gu_r = plan_lut((int)m.I, (int)m.H, true, rows_per_group, m.max_tiles_r);
-        m.dn_r = plan_lut((int)m.H, (int)m.I, false, rows_per_group, m.max_tiles_r);
+        if (m.tc_r) {
+            m.gu_r = plan_lut_tc((int)m.I, (int)m.H, true, m.tile_rows, m.max_tiles_r);
+            m.dn_r = plan_lut_tc((int)m.H, (int)m.I, false, m.tile_rows, m.max_tiles_r);
+        } else {
+            m.gu_r = plan_lut((int)m.I, (int)m.H, true, rows_per_group, m.max_tiles_r);
+            m.dn_r = plan_lut((int)m.H, (int)m.I, false, rows_per_group, m.max_tiles_r);
+        }
     }
     if (m.ns > 0) {
-        m.gu_s = plan_lut((int)m.Is, (int)m.H, true, rows_per_group, m.tiles_s, (int)T,
-                          (int)m.ns);
-        m.dn_s = plan_lut((int)m.H, (int)m.Is, false, rows_per_group, m.tiles_s, (int)T,
-                          (int)m.ns);
+        if (m.tc_s) {
+            m.gu_s = plan_lut_tc((int)m.Is, (int)m.H, true, m.tile_rows_s, m.tiles_s, (int)T,
+                                 (int)m.ns);
+            m.dn_s = plan_lut_tc((int)m.H, (int)m.Is, false, m.tile_rows_s, m.tiles_s, (int)T,
+                                 (int)m.ns);
+        } else {
+            m.gu_s = plan_lut((int)m.Is, (int)m.H, true, rows_per_group, m.tiles_s, (int)T,
+                              (int)m.ns);
+            m.dn_s = plan_lut((int)m.H, (int)m.Is, false, rows_per_group, m.tiles_s, (int)T,
+                              (int)m.ns);
+        }
     }
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -99,6 +145,10 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
     m.o_sh = take((size_t)m.R * 4);
     m.o_pdn_r = take(m.E > 0 ? (size_t)m.dn_r.splits * m.Rr * m.H * 4 : 0);
     m.o_pdn_s = take(m.ns > 0 ? (size_t)m.dn_s.splits * m.Rs * m.H * 4 : 0);
+    m.o_bx_r = take(m.tc_r ? (size_t)m.Rr * m.H * 2 : 0);
+    m.o_bx_s = take(m.tc_s ? (size_t)T * m.H * 2 : 0);
+    m.o_bh_r = take(m.tc_r ? (size_t)m.Rr * m.I * 2 : 0);
+    m.o_bh_s = take(m.tc_s ? (size_t)m.Rs * m.Is * 2 : 0);
     m.total = o;
     return m;
 }
@@ -116,6 +166,7 @@ cq_status check_moe_desc(const cq_moe_desc *d, int64_t T) {
     } else if (d->top_k != 0) {
         return CQ_ERR_INVALID_ARGUMENT;
     }
+    if (d->n_shared > 4) return CQ_ERR_UNSUPPORTED;
     if (d->n_shared > 0) {
         if (d->I_shared <= 0) return CQ_ERR_INVALID_ARGUMENT;
         if (!is_pow2(d->had_block_i_shared) || d->I_shared % d->had_block_i_shared)
@@ -205,7 +256,15 @@ cq_status cq_lut_gemm(const void *q, const float *s_x, int64_t M, int64_t K, int
     L.direct = false;
     L.out = reinterpret_cast<float *>(workspace);
     L.out_split_stride = M * N;
-    cudaError_t e = launch_lut(L, g.p, st);
+    cudaError_t e;
+    if (g.p.tc) {
+        void *b = reinterpret_cast<uint8_t *>(workspace) + g.b_off;
+        e = launch_codes_to_f16(q, code_bytes(K, act_bits), act_bits, (int)K, M, kMapIdentity,
+                                nullptr, 1, 1, b, st);
+        if (e == cudaSuccess) e = launch_lut_tc(L, g.p, b, M, 0, st);
+    } else {
+        e = launch_lut(L, g.p, st);
+    }
     if (e == cudaSuccess) e = launch_reduce_plain(L.out, g.p, M, N, s_x, y, st);
     if (e == cudaSuccess && centroid_sums)
         e = launch_centroid_sums(q, M, K, act_bits, w_idx, N, centroid_sums, st);
@@ -280,7 +339,14 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.idx0 = w->gate_idx; L.cb0 = w->gate_cb; L.idx1 = w->up_idx; L.cb1 = w->up_cb;
         L.w_stride = m.I * (m.H / 2); L.cb_stride = m.I * 16; L.N = (int)m.I; L.dual = true;
         L.out = pgu_r; L.out_split_stride = m.Rr * m.I * 2; L.out_row_stride = m.I * 2;
-        e = launch_lut(L, m.gu_r, st);
+        if (m.tc_r) {
+            void *b = ws + m.o_bx_r;
+            e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, m.Rr, kMapPerm, perm, (int)m.k,
+                                    (int)T, b, st);
+            if (e == cudaSuccess) e = launch_lut_tc(L, m.gu_r, b, m.Rr, 0, st);
+        } else {
+            e = launch_lut(L, m.gu_r, st);
+        }
     }
     if (e == cudaSuccess && m.ns > 0) {
         LutLaunch L{};
@@ -290,7 +356,14 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.idx0 = w->sh_gate_idx; L.cb0 = w->sh_gate_cb; L.idx1 = w->sh_up_idx; L.cb1 = w->sh_up_cb;
         L.w_stride = m.Is * (m.H / 2); L.cb_stride = m.Is * 16; L.N = (int)m.Is; L.dual = true;
         L.out = pgu_s; L.out_split_stride = m.Rs * m.Is * 2; L.out_row_stride = m.Is * 2;
-        e = launch_lut(L, m.gu_s, st);
+        if (m.tc_s) {
+            void *b = ws + m.o_bx_s;
+            e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, T, kMapIdentity, nullptr, 1,
+                                    (int)T, b, st);
+            if (e == cudaSuccess) e = launch_lut_tc(L, m.gu_s, b, T, (int)T, st);
+        } else {
+            e = launch_lut(L, m.gu_s, st);
+        }
     }
     // SwiGLU + rotate + quantize of h
     if (e == cudaSuccess) {
@@ -315,7 +388,14 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.idx0 = w->down_idx; L.cb0 = w->down_cb;
         L.w_stride = m.H * (m.I / 2); L.cb_stride = m.H * 16; L.N = (int)m.H; L.dual = false;
         L.out = pdn_r; L.out_split_stride = m.Rr * m.H; L.out_row_stride = m.H;
-        e = launch_lut(L, m.dn_r, st);
+        if (m.tc_dn_r) {
+            void *b = ws + m.o_bh_r;
+            e = launch_codes_to_f16(hq, ldh, m.bits, (int)m.I, m.Rr, kMapIdentity, nullptr, 1, 1,
+                                    b, st);
+            if (e == cudaSuccess) e = launch_lut_tc(L, m.dn_r, b, m.Rr, 0, st);
+        } else {
+            e = launch_lut(L, m.dn_r, st);
+        }
     }
     if (e == cudaSuccess && m.ns > 0) {
         LutLaunch L{};
@@ -325,7 +405,14 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.idx0 = w->sh_down_idx; L.cb0 = w->sh_down_cb;
         L.w_stride = m.H * (m.Is / 2); L.cb_stride = m.H * 16; L.N = (int)m.H; L.dual = false;
         L.out = pdn_s; L.out_split_stride = m.Rs * m.H; L.out_row_stride = m.H;
-        e = launch_lut(L, m.dn_s, st);
+        if (m.tc_dn_s) {
+            void *b = ws + m.o_bh_s;
+            e = launch_codes_to_f16(hq + m.Rr * ldh, ldh, m.bits, (int)m.Is, m.Rs, kMapIdentity,
+                                    nullptr, 1, 1, b, st);
+            if (e == cudaSuccess) e = launch_lut_tc(L, m.dn_s, b, m.Rs, 0, st);
+        } else {
+            e = launch_lut(L, m.dn_s, st);
+        }
     }
     if (e == cudaSuccess) {
         CombineArgs c{};

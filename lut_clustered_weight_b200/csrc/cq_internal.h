@@ -74,6 +74,7 @@ struct LutPlan {
     int chunks_per_split;
     int64_t units;      // stream-K: total units (work items * C)
     int uniform_rows;   // stream-K: rows per group (token tiles of a group are consecutive)
+    int tc;             // 1: tensor-memory kernel (64-k chunks, 128-row tiles)
     size_t smem;
 };
 
@@ -109,6 +110,25 @@ __host__ __device__ inline int lut_splits_at(const LutPlan &P, int64_t p, int n)
 LutPlan plan_lut(int N, int K, bool dual, int max_rows_per_group, int64_t est_tiles,
                  int uniform_rows = 0, int n_groups = 1);
 cudaError_t launch_lut(const LutLaunch &L, const LutPlan &P, cudaStream_t st);
+
+// Tensor-memory (tcgen05) LUT GEMM.  The activations are read as fp16 rows
+// b_f16 [b_rows][K]; the GEMM row p of a token tile maps to B row
+// (b_row_mod > 0 ? p % b_row_mod : p).
+int tc_ntok_for(int max_rows_per_group);
+LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est_tiles,
+                    int uniform_rows = 0, int n_groups = 1);
+cudaError_t launch_lut_tc(const LutLaunch &L, const LutPlan &P, const void *b_f16, int64_t b_rows,
+                          int b_row_mod, cudaStream_t st);
+// fp16 copies of activation codes (B operand), rows mapped like LutLaunch::map_mode.
+cudaError_t launch_codes_to_f16(const void *codes, int64_t ld_codes, int bits, int K,
+                                int64_t rows, int map_mode, const int32_t *perm, int topk, int T,
+                                void *out, cudaStream_t st);
+// Reads and clears the device error word (-1 if the read failed).
+int read_device_error();
+// Which LUT kernel a launch uses: "mma" (mma.sync, register tables), "tc"
+// (tcgen05 / tensor memory), or automatic (default).
+enum LutPath : int { kPathAuto = 0, kPathMma = 1, kPathTc = 2 };
+LutPath lut_path();
 
 // y[m, n] = s[m] * sum_{s < n(m, n)} part[s][m][n]
 cudaError_t launch_reduce_plain(const float *part, const LutPlan &P, int64_t M, int64_t N,

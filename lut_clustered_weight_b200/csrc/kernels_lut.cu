@@ -24,51 +24,13 @@
 //    Split-K partial sums go to a workspace and are reduced in a fixed order.
 #include "cq_common.cuh"
 #include "cq_internal.h"
+#include "lut_lookup.cuh"
 
 #include <algorithm>
 
 namespace cq {
 
 constexpr int kTokTile = 16;  // largest token tile (two n8 MMA tiles)
-
-// Byte-plane tables of one codebook row: lo[j] holds the low bytes of
-// C[4j..4j+3], hi[j] the high bytes.
-CQ_DEV void build_tables(const __half *cb, uint32_t (&lo)[4], uint32_t (&hi)[4]) {
-    const uint4 a = *reinterpret_cast<const uint4 *>(cb);
-    const uint4 b = *reinterpret_cast<const uint4 *>(cb + 8);
-    const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-        lo[j] = prmt(u[2 * j], u[2 * j + 1], 0x6420);
-        hi[j] = prmt(u[2 * j], u[2 * j + 1], 0x7531);
-    }
-}
-
-// Eight 4-bit indices (nibble i of w = index of element i) -> four half2:
-// h[0] = (C[i0], C[i1]), h[1] = (C[i2], C[i3]), h[2] = (C[i4], C[i5]),
-// h[3] = (C[i6], C[i7]).  Selector nibble bit 3 switches prmt to
-// sign-replicate mode, so entries 0-7 and 8-15 are fetched from the two
-// halves of each plane and merged with a per-byte mask built from bit 3.
-CQ_DEV void dequant8(uint32_t w, const uint32_t (&lo)[4], const uint32_t (&hi)[4],
-                     uint32_t (&h)[4]) {
-    const uint32_t s0 = w, s1 = w >> 16;
-    const uint32_t x0 = s0 ^ 0x8888u, x1 = s1 ^ 0x8888u;
-    const uint32_t w4 = w << 4;
-    const uint32_t m0 = prmt(w4, w, 0xD9C8);  // 0xFF in byte i iff nibble i >= 8
-    const uint32_t m1 = prmt(w4, w, 0xFBEA);
-    {
-        const uint32_t l = (prmt(lo[0], lo[1], s0) & ~m0) | (prmt(lo[2], lo[3], x0) & m0);
-        const uint32_t g = (prmt(hi[0], hi[1], s0) & ~m0) | (prmt(hi[2], hi[3], x0) & m0);
-        h[0] = prmt(l, g, 0x5140);
-        h[1] = prmt(l, g, 0x7362);
-    }
-    {
-        const uint32_t l = (prmt(lo[0], lo[1], s1) & ~m1) | (prmt(lo[2], lo[3], x1) & m1);
-        const uint32_t g = (prmt(hi[0], hi[1], s1) & ~m1) | (prmt(hi[2], hi[3], x1) & m1);
-        h[2] = prmt(l, g, 0x5140);
-        h[3] = prmt(l, g, 0x7362);
-    }
-}
 
 CQ_DEV __half code_to_half(int v) { return __short2half_rn((short)v); }
 
@@ -406,13 +368,21 @@ cudaError_t launch_lut(const LutLaunch &L, const LutPlan &P, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- split-K reduce
-__global__ void k_reduce_plain(const float *__restrict__ part, const LutPlan P, int64_t M,
-                               int64_t N, const float *__restrict__ s, float *__restrict__ y) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= M * N) return;
-    const int64_t m = i / N;
-    const int n = (int)(i - m * N);
-    const int ns = lut_splits_at(P, m, n);
+// grid: (column blocks of 256, M rows)
+__global__ void __launch_bounds__(256) k_reduce_plain(const float *__restrict__ part, const LutPlan P,
+                                                      int64_t M, int64_t N, const float *__restrict__ s,
+                                                      float *__restrict__ y) {
+    __shared__ int s_ns[8];
+    const int64_t m = blockIdx.y;
+    const int n0 = blockIdx.x * 256;
+    const int rt0 = n0 / P.rows_per_rt;
+    const int nrt = (min((int64_t)n0 + 255, N - 1)) / P.rows_per_rt - rt0 + 1;
+    if (threadIdx.x < nrt) s_ns[threadIdx.x] = lut_splits_at(P, m, (rt0 + threadIdx.x) * P.rows_per_rt);
+    __syncthreads();
+    const int n = n0 + threadIdx.x;
+    if (n >= N) return;
+    const int ns = s_ns[n / P.rows_per_rt - rt0];
+    const int64_t i = m * N + n;
     float acc = 0.0f;
     for (int k = 0; k < ns; k++) acc += part[(int64_t)k * M * N + i];
     y[i] = s[m] * acc;
@@ -423,7 +393,8 @@ cudaError_t launch_reduce_plain(const float *part, const LutPlan &P, int64_t M, 
     const int64_t n = M * N;
     if (n == 0) return cudaSuccess;
     count_launch();
-    k_reduce_plain<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, P, M, N, s, y);
+    dim3 grid((unsigned)((N + 255) / 256), (unsigned)M);
+    k_reduce_plain<<<grid, 256, 0, st>>>(part, P, M, N, s, y);
     return cudaGetLastError();
 }
 

@@ -1,0 +1,566 @@
+// kernels_lut_tc.cu -- LUT (codebook) GEMM on the sm_100a tensor cores
+// (tcgen05 / tensor memory).
+//
+//   y[m, n] = s_x[m] * sum_k C[n, I[n,k]] * q[m, k]
+//
+// CodeQuant2 Figure 4 describes the LUT kernel as a one-time LUT precompute
+// held in shared memory followed by table lookups.  Here:
+//  * One thread per weight row: thread t of the four "expand" warps owns row
+//    t of a 128-row tile, which is also lane t of tensor memory (TMEM).
+//  * PAIR mode (decode): the one-time precompute is a 256-entry pair table per
+//    row in shared memory -- entry b holds the two fp16 centroids selected by
+//    an index byte b (low nibble = even k).  Entry b of thread t sits at
+//    b * 512 + 4 t, so the 32 lanes of a warp always hit 32 different banks,
+//    whatever the indices.  One byte (two weights) costs one byte extract,
+//    one address multiply-add and one 4-byte shared load.
+//  * PRMT mode (prefill): the codebook is held as two byte-plane tables in
+//    registers and looked up with byte permutes; no shared memory is spent on
+//    tables, which leaves room for wide activation tiles.
+//  * The looked-up fp16 weights of a 64-k chunk are stored to TMEM
+//    (tcgen05.st, 32 columns per row) and used as the A operand of
+//    tcgen05.mma kind::f16; the activations (int codes converted to fp16,
+//    exact) are the B operand, a 128-byte-swizzled shared tile loaded by TMA.
+//    The fp32 accumulator lives in TMEM and is read back with tcgen05.ld.
+//  * Roles: warps 0-3 expand (and prefetch their rows' index bytes into
+//    registers); lane 0 of warp 4 issues the TMA loads and the MMAs.
+//    mbarriers connect them; every wait is bounded.
+//  * Work is cut into (128-row tile x token tile) items and 64-k chunks,
+//    shared out like the mma.sync kernel (stream-K for uniform launches).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "cq_common.cuh"
+#include "cq_internal.h"
+#include "lut_lookup.cuh"
+#include "sm100.cuh"
+
+namespace cq {
+
+constexpr int kTcThreads = 160;      // 4 expand warps + 1 MMA / TMA warp
+constexpr int kTcRows = 128;         // rows per tile (TMEM lanes)
+constexpr int kTcChunk = 64;         // k per chunk (32 TMEM columns of fp16 pairs)
+constexpr int kTcA = 8;              // A ring depth: TMEM, 32 columns per chunk
+// B ring depth (shared memory, NTOK x 128 B per chunk); a B slot is freed by
+// the commit of the chunk that used it.  B for chunk j + B - B/2 is loaded
+// while chunk j is issued.
+template <int NTOK> struct TcB { static constexpr int n = NTOK <= 128 ? 8 : 4; };
+constexpr int kTcWStages = 16;       // index-byte ring: 15 chunks in flight per thread
+constexpr size_t kPairTableBytes = 256 * kTcRows * 4;  // 128 KB
+
+struct TcSchedule {
+    const LutLaunch *L;
+    const LutPlan *P;
+    // work item -> (group, first row, rows, row tile)
+    CQ_DEV void item(int64_t w, int &g, int &row0, int &nrows, int &rt) const {
+        const int TT = 8 * P->nt;
+        const int64_t tile = w / P->n_row_tiles;
+        rt = (int)(w - tile * P->n_row_tiles);
+        if (L->uniform_rows > 0) {
+            const int tpg = (L->uniform_rows + TT - 1) / TT;
+            g = (int)(tile / tpg);
+            row0 = g * L->uniform_rows + (int)(tile - (int64_t)g * tpg) * TT;
+            nrows = min(TT, (g + 1) * L->uniform_rows - row0);
+        } else {
+            if (tile >= L->grp_tiles[L->G]) {
+                g = -1;
+                row0 = nrows = 0;
+                return;
+            }
+            int lo = 0, hi = L->G;
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (L->grp_tiles[mid] <= tile) lo = mid; else hi = mid;
+            }
+            g = lo;
+            row0 = L->grp_rows[g] + (int)(tile - L->grp_tiles[g]) * TT;
+            nrows = min(TT, L->grp_rows[g + 1] - row0);
+        }
+    }
+    // this thread's weight row: index bytes and codebook (t = 0..127)
+    CQ_DEV void row_ptrs(int g, int rt, int t, const uint8_t *&idx, const __half *&cb, int &col) const {
+        const int64_t rowbytes = L->K / 2;
+        if (L->dual) {
+            const int n = rt * 64 + (t & 63);
+            const bool up = t >= 64;
+            idx = (up ? L->idx1 : L->idx0) + (int64_t)g * L->w_stride + (int64_t)n * rowbytes;
+            cb = reinterpret_cast<const __half *>(up ? L->cb1 : L->cb0) + (int64_t)g * L->cb_stride + n * 16;
+            col = 2 * n + (up ? 1 : 0);
+        } else {
+            const int n = rt * kTcRows + t;
+            idx = L->idx0 + (int64_t)g * L->w_stride + (int64_t)n * rowbytes;
+            cb = reinterpret_cast<const __half *>(L->cb0) + (int64_t)g * L->cb_stride + n * 16;
+            col = n;
+        }
+    }
+};
+
+// Walks a CTA's units in order: (work item w, chunk ch), dividing only when
+// the walk enters a new item.
+struct TcCursor {
+    int64_t w;
+    int ch;
+    CQ_DEV void init(int64_t u, int C) {
+        w = u / C;
+        ch = (int)(u - w * C);
+    }
+    CQ_DEV void next(int C) {
+        if (++ch == C) {
+            ch = 0;
+            ++w;
+        }
+    }
+};
+
+template <int NTOK, bool PAIR>
+__global__ void __launch_bounds__(kTcThreads, 1)
+k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPlan P, int b_row_mod) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+    uint8_t *sm = smem_raw + pad;
+    constexpr uint32_t kBSlot = NTOK * 128;  // bytes of one B chunk tile
+    constexpr int kTcB = TcB<NTOK>::n;
+    constexpr int kTcBLag = kTcB / 2;
+    uint8_t *bslots = sm;                                     // [kTcB][NTOK][128 B]
+    uint8_t *tables = sm + kTcB * kBSlot;                     // PAIR: [256][128 threads] x 4 B
+    uint8_t *wring_raw = tables + (PAIR ? kPairTableBytes : 0);  // [stages][2][128] x 16 B
+    uint64_t *bars = reinterpret_cast<uint64_t *>(wring_raw + kTcWStages * 2 * kTcRows * 16);
+    uint64_t *a_full = bars, *a_empty = bars + kTcA;
+    uint64_t *b_full = bars + 2 * kTcA;
+    uint64_t *d_full = b_full + kTcB, *d_empty = d_full + 1, *fin = d_full + 2;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(fin + 1);
+    int *s_stop = reinterpret_cast<int *>(s_tmem + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr uint32_t kTmemCols = 512;  // A ring 256 + accumulator NTOK (<= 256)
+    const TcSchedule S{&L, &P};
+    const int C = P.chunks_total;
+
+    if (warp == 4) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+        if (lane == 0) {
+            for (int s = 0; s < kTcA; s++) {
+                mbar_init(&a_full[s], 4);  // one arrival per expand warp
+                mbar_init(&a_empty[s], 1);
+            }
+            for (int s = 0; s < kTcB; s++) mbar_init(&b_full[s], 1);
+            mbar_init(d_full, 1);
+            mbar_init(d_empty, 4);
+            mbar_init(fin, 1);
+            *s_stop = 0;
+            fence_barrier_init();
+            prefetch_tmap(&tmB);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tmem_a = tmem;                // columns [0, 256): A ring (8 x 32)
+    const uint32_t tmem_d = tmem + kTcA * 32;    // columns [256, 256 + NTOK): accumulator
+
+    // ---- this CTA's units
+    int64_t u0, u1;
+    if (P.streamk) {
+        u0 = (int64_t)blockIdx.x * P.units / P.grid;
+        u1 = ((int64_t)blockIdx.x + 1) * P.units / P.grid;
+    } else {
+        const int rt = blockIdx.x % P.n_row_tiles;
+        const int split = blockIdx.x / P.n_row_tiles;
+        const int64_t w = (int64_t)blockIdx.y * P.n_row_tiles + rt;
+        u0 = w * C + (int64_t)split * P.chunks_per_split;
+        u1 = min(u0 + P.chunks_per_split, w * C + C);
+        int g, r0, nr, rtt;
+        S.item(w, g, r0, nr, rtt);
+        if (g < 0) u1 = u0;  // beyond the routed tiles: nothing to do
+    }
+    const int nchunks = (int)(u1 - u0);
+
+    if (warp == 4) {
+        // ====================== TMA + MMA issuer (one thread) ======================
+        if (lane == 0 && nchunks > 0) {
+            constexpr uint32_t idesc = idesc_f16(kTcRows, NTOK);
+            TcCursor bc;  // chunk of the next B load
+            bc.init(u0, C);
+            int64_t b_item = -1;
+            int b_y = 0;
+            auto issue_b = [&](int j) {
+                const int s = j % kTcB;
+                if (bc.w != b_item) {
+                    int g, row0, nrows, rt;
+                    S.item(bc.w, g, row0, nrows, rt);
+                    b_item = bc.w;
+                    b_y = b_row_mod > 0 ? row0 % b_row_mod : row0;
+                }
+                mbar_arrive_expect_tx(&b_full[s], kBSlot);
+                tma_load_2d(bslots + s * kBSlot, &tmB, bc.ch * kTcChunk, b_y, &b_full[s]);
+                bc.next(C);
+            };
+            TcCursor mc;  // chunk of the next MMA
+            mc.init(u0, C);
+            int issued = 0, consumed = 0;
+            for (int j = 0; j < kTcB - kTcBLag && j < nchunks; j++) {
+                issue_b(j);
+                issued++;
+            }
+            int items = 0;
+            bool ok = true;
+            for (int j = 0; j < nchunks && ok; j++) {
+                const int s = j % kTcA, sb = j % kTcB;
+                const int ch = mc.ch;
+                mc.next(C);
+                const bool first = (j == 0) || ch == 0;
+                const bool last = (j == nchunks - 1) || ch == C - 1;
+                if (first && items > 0) ok = mbar_wait(d_empty, (uint32_t)(items - 1) & 1u);
+                ok = ok && mbar_wait(&a_full[s], (uint32_t)(j / kTcA) & 1u) &&
+                     mbar_wait(&b_full[sb], (uint32_t)(j / kTcB) & 1u);
+                if (!ok) break;
+                consumed++;
+                tc_fence_after();
+                const uint64_t bd = smem_desc_sw128(smem_u32(bslots + sb * kBSlot));
+#pragma unroll
+                for (int kk = 0; kk < kTcChunk / 16; kk++)
+                    tc_mma_ts(tmem_d, tmem_a + s * 32 + kk * 8, bd + (uint64_t)(2 * kk), idesc,
+                              (first && kk == 0) ? 0u : 1u);
+                tc_commit(&a_empty[s]);  // frees A slot s and B slot sb (= s)
+                if (last) {
+                    tc_commit(d_full);
+                    items++;
+                }
+                // load B of chunk j + kTcB - kTcBLag into the slot of chunk
+                // j - kTcBLag, whose MMAs were issued kTcBLag chunks ago
+                const int jn = j + kTcB - kTcBLag;
+                if (jn < nchunks) {
+                    if (jn >= kTcB) {  // the slot was used by chunk jn - kTcB
+                        const int jo = jn - kTcB;
+                        ok = mbar_wait(&a_empty[jo % kTcA], (uint32_t)(jo / kTcA) & 1u);
+                        static_assert(kTcA % TcB<NTOK>::n == 0, "B slots must divide A slots");
+                    }
+                    if (ok) {
+                        issue_b(jn);
+                        issued++;
+                    }
+                }
+            }
+            if (!ok) atomicExch(s_stop, 1);
+            // nothing may still be writing shared or tensor memory when the CTA
+            // leaves: wait for every issued TMA load and for all issued MMAs
+            for (int j = consumed; j < issued; j++)
+                mbar_wait(&b_full[j % kTcB], (uint32_t)(j / kTcB) & 1u);
+            tc_commit(fin);
+            mbar_wait(fin, 0);
+        }
+    } else {
+        // ====================== expand warps: one thread per row ======================
+        const int t = tid;  // 0..127 = TMEM lane
+        const uint32_t lane_base = ((uint32_t)(warp * 32)) << 16;
+        uint32_t *tab = reinterpret_cast<uint32_t *>(tables) + t;  // entry b at tab[b * 128]
+        uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};      // PRMT mode tables
+        // per-thread ring of index bytes: stage st holds 2 x 16 B at
+        // wring[(st * 2 + r) * 128 + t] (consecutive threads -> consecutive 16 B)
+        uint4 *wring = reinterpret_cast<uint4 *>(wring_raw);
+        TcCursor pc;  // chunk of the next index-byte copy
+        pc.init(u0, C);
+        int64_t p_item = -1;
+        const uint8_t *p_row = nullptr;
+        auto issue_w = [&](int j) {
+            if (pc.w != p_item) {
+                int gg, r0, nr, rtt, cc;
+                S.item(pc.w, gg, r0, nr, rtt);
+                const __half *cbx;
+                S.row_ptrs(max(gg, 0), rtt, t, p_row, cbx, cc);
+                p_item = pc.w;
+            }
+            const uint8_t *p = p_row;
+            const int k0 = pc.ch * kTcChunk;
+            pc.next(C);
+            uint4 *dst = wring + (size_t)((j % kTcWStages) * 2) * kTcRows + t;
+            const bool h0 = k0 < L.K, h1 = k0 + 32 < L.K;  // ragged last chunk: zeros
+            cp_async16_zfill(dst, h0 ? p + k0 / 2 : p, h0 ? 16 : 0);
+            cp_async16_zfill(dst + kTcRows, h1 ? p + k0 / 2 + 16 : p, h1 ? 16 : 0);
+        };
+        for (int j = 0; j < kTcWStages - 1; j++) {
+            if (j < nchunks) issue_w(j);
+            cp_async_commit_group();
+        }
+        int64_t cur_w = -1;
+        int g = 0, row0 = 0, nrows = 0, rt = 0, col = 0, items = 0;
+        bool ok = true;
+        TcCursor wc;  // chunk being expanded
+        wc.init(u0, C);
+        for (int j = 0; j < nchunks; j++) {
+            const int64_t w = wc.w;
+            const int ch = wc.ch;
+            wc.next(C);
+            if (w != cur_w) {
+                cur_w = w;
+                const uint8_t *idxp;
+                const __half *cbp;
+                S.item(w, g, row0, nrows, rt);
+                S.row_ptrs(max(g, 0), rt, t, idxp, cbp, col);
+                // the one-time LUT precompute for this row
+                const uint4 c0v = *reinterpret_cast<const uint4 *>(cbp);
+                const uint4 c1v = *reinterpret_cast<const uint4 *>(cbp + 8);
+                const uint32_t cu[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
+                if (PAIR) {
+#pragma unroll 1
+                    for (int h = 0; h < 16; h++) {
+                        const uint32_t hv = (uint32_t)__half_as_ushort(cbp[h]);
+#pragma unroll
+                        for (int l = 0; l < 16; l++)
+                            tab[(h * 16 + l) * kTcRows] =
+                                prmt(cu[l >> 1], hv, (l & 1) ? 0x5432u : 0x5410u);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; q++) {
+                        lo[q] = prmt(cu[2 * q], cu[2 * q + 1], 0x6420);
+                        hi[q] = prmt(cu[2 * q], cu[2 * q + 1], 0x7531);
+                    }
+                }
+            }
+            cp_async_wait_group<kTcWStages - 2>();
+            const uint4 *src = wring + (size_t)((j % kTcWStages) * 2) * kTcRows + t;
+            const uint4 wa = src[0], wb = src[kTcRows];
+            if (j + kTcWStages - 1 < nchunks) issue_w(j + kTcWStages - 1);
+            cp_async_commit_group();
+            const uint32_t wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            // 64 weights -> 32 fp16 pairs (k = 2b, 2b + 1 in column b)
+            uint32_t v[32];
+            if (PAIR) {
+#pragma unroll
+                for (int b = 0; b < 32; b++) {
+                    const uint32_t byte = prmt(wd[b >> 2], 0u, 0x4440u | (uint32_t)(b & 3));
+                    v[b] = tab[byte * kTcRows];
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; q++) {
+                    uint32_t h4[4];
+                    dequant8(wd[q], lo, hi, h4);
+                    v[4 * q] = h4[0];
+                    v[4 * q + 1] = h4[1];
+                    v[4 * q + 2] = h4[2];
+                    v[4 * q + 3] = h4[3];
+                }
+            }
+            const int s = j % kTcA;
+            if (j >= kTcA) {
+                ok = mbar_wait(&a_empty[s], (uint32_t)(j / kTcA - 1) & 1u);
+                if (!ok) break;
+                tc_fence_after();
+            }
+            tmem_st32(tmem_a + lane_base + s * 32, v);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[s]);
+            if (ch == C - 1 || j == nchunks - 1) {
+                // item done: D (NTOK fp32 columns of this row) -> partial sums
+                ok = mbar_wait(d_full, (uint32_t)items & 1u);
+                if (!ok) break;
+                tc_fence_after();
+                const int slot = P.streamk ? (int)(blockIdx.x - lut_cta_of_unit(P, cur_w * C))
+                                           : (int)(blockIdx.x / P.n_row_tiles);
+                float *out = L.out + (int64_t)slot * L.out_split_stride;
+#pragma unroll 1
+                for (int c0 = 0; c0 < NTOK; c0 += 16) {
+                    uint32_t d[16];
+                    tmem_ld16(tmem_d + lane_base + c0, d);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 16; q++)
+                        if (c0 + q < nrows)
+                            out[(int64_t)(row0 + c0 + q) * L.out_row_stride + col] =
+                                __uint_as_float(d[q]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(d_empty);
+                items++;
+                cur_w = -1;
+            }
+        }
+        cp_async_wait_group<0>();
+        if (!ok) atomicExch(s_stop, 1);
+    }
+    // ---- teardown: all MMAs and TMEM reads are complete before TMEM is freed
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 4) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map over fp16 [rows][K] (row stride K), box [ntok rows][64 k], 128-byte swizzle.
+static bool make_b_map(CUtensorMap *m, const void *base, int64_t rows, int K, int ntok) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kTcChunk, (cuuint32_t)ntok};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int tc_ntok_for(int max_rows_per_group) {
+    return max_rows_per_group <= 16 ? 16 : max_rows_per_group <= 64 ? 64
+         : max_rows_per_group <= 128 ? 128 : 256;
+}
+
+LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est_tiles,
+                    int uniform_rows, int n_groups) {
+    LutPlan P{};
+    const int ntok = tc_ntok_for(max_rows_per_group);
+    P.nt = ntok / 8;
+    P.warps = 4;
+    P.rows_per_rt = dual ? 64 : kTcRows;
+    P.n_row_tiles = N / P.rows_per_rt;
+    P.chunks_total = (K + kTcChunk - 1) / kTcChunk;
+    P.cps_max = P.chunks_total;
+    const int capacity = sm_count();  // one CTA per SM
+    const int C = P.chunks_total;
+    if (uniform_rows > 0) {
+        const int64_t tiles = (int64_t)n_groups * ((uniform_rows + ntok - 1) / ntok);
+        P.streamk = 1;
+        P.uniform_rows = uniform_rows;
+        P.units = tiles * P.n_row_tiles * C;
+        P.grid = (int)std::min<int64_t>(capacity, P.units);
+        int smax = 1;
+        const int64_t items = tiles * P.n_row_tiles;
+        for (int64_t w = 0; w < items; w++) smax = std::max(smax, lut_item_splits(P, w));
+        P.splits = smax;
+        P.chunks_per_split = C;
+    } else {
+        P.streamk = 0;
+        const int64_t base = (int64_t)P.n_row_tiles * std::max<int64_t>(est_tiles, 1);
+        int splits = base < capacity ? (int)(capacity / base) : 1;
+        splits = std::max(1, std::min(splits, C));
+        P.chunks_per_split = (C + splits - 1) / splits;
+        P.splits = (C + P.chunks_per_split - 1) / P.chunks_per_split;
+        P.grid = P.n_row_tiles * P.splits;
+    }
+    const bool pair = ntok <= 16;
+    const int nb = ntok <= 128 ? 8 : 4;
+    P.smem = 1024 + (size_t)nb * ntok * 128 + (pair ? kPairTableBytes : 0) +
+             (size_t)kTcWStages * 2 * kTcRows * 16 + 512;
+    P.tc = 1;
+    return P;
+}
+
+template <int NTOK, bool PAIR>
+static cudaError_t launch_tc_t(const CUtensorMap &m, const LutLaunch &L, const LutPlan &P,
+                               int b_row_mod, cudaStream_t st) {
+    cudaFuncSetAttribute(k_lut_tc<NTOK, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)P.smem);
+    dim3 grid(P.grid, P.streamk ? 1 : L.max_tiles);
+    k_lut_tc<NTOK, PAIR><<<grid, kTcThreads, P.smem, st>>>(m, L, P, b_row_mod);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lut_tc(const LutLaunch &L, const LutPlan &P, const void *b_f16,
+                          int64_t b_rows, int b_row_mod, cudaStream_t st) {
+    if (P.grid == 0 || (!P.streamk && L.max_tiles == 0)) return cudaSuccess;
+    const int ntok = 8 * P.nt;
+    CUtensorMap m;
+    std::memset(&m, 0, sizeof(m));
+    if (!make_b_map(&m, b_f16, b_rows, L.K, ntok)) return cudaErrorInvalidValue;
+    const bool timed = timing_on();
+    if (timed) timing_begin(st);
+    count_launch();
+    cudaError_t e;
+    switch (ntok) {
+    case 16: e = launch_tc_t<16, true>(m, L, P, b_row_mod, st); break;
+    case 64: e = launch_tc_t<64, false>(m, L, P, b_row_mod, st); break;
+    case 128: e = launch_tc_t<128, false>(m, L, P, b_row_mod, st); break;
+    default: e = launch_tc_t<256, false>(m, L, P, b_row_mod, st); break;
+    }
+    if (timed) timing_end(st);
+    return e;
+}
+
+// ---------------------------------------------------------------- codes -> fp16 rows
+// out[p, k] = fp16(code of row map(p), position k): the B operand of the
+// tensor-core kernel.  One thread per 8 codes.
+__global__ void k_codes_to_f16(const uint8_t *__restrict__ codes, int64_t ld_codes, int bits,
+                               int K, int64_t rows, int map_mode, const int32_t *__restrict__ perm,
+                               int topk, int T, __half *__restrict__ out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int per_row = K / 8;
+    if (i >= rows * per_row) return;
+    const int64_t p = i / per_row;
+    const int k = (int)(i - p * per_row) * 8;
+    const int64_t cr = map_mode == kMapPerm ? perm[p] / topk : map_mode == kMapModT ? p % T : p;
+    const uint8_t *src = codes + cr * ld_codes;
+    __align__(16) __half v[8];
+    if (bits == 4) {
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(src + k / 2);
+#pragma unroll
+        for (int e = 0; e < 8; e++) v[e] = __short2half_rn((short)(((int)(w << (28 - 4 * e))) >> 28));
+    } else {
+        const uint2 w = *reinterpret_cast<const uint2 *>(src + k);
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            v[e] = __short2half_rn((short)(((int)(w.x << (24 - 8 * e))) >> 24));
+            v[4 + e] = __short2half_rn((short)(((int)(w.y << (24 - 8 * e))) >> 24));
+        }
+    }
+    *reinterpret_cast<uint4 *>(out + p * K + k) = *reinterpret_cast<const uint4 *>(v);
+}
+
+cudaError_t launch_codes_to_f16(const void *codes, int64_t ld_codes, int bits, int K,
+                                int64_t rows, int map_mode, const int32_t *perm, int topk, int T,
+                                void *out, cudaStream_t st) {
+    const int64_t n = rows * (K / 8);
+    if (n == 0) return cudaSuccess;
+    count_launch();
+    k_codes_to_f16<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        reinterpret_cast<const uint8_t *>(codes), ld_codes, bits, K, rows, map_mode, perm, topk, T,
+        reinterpret_cast<__half *>(out));
+    return cudaGetLastError();
+}
+
+LutPath lut_path() {
+    static LutPath p = [] {
+        const char *e = getenv("CQ_LUT_PATH");
+        if (e && !strcmp(e, "mma")) return kPathMma;
+        if (e && !strcmp(e, "tc")) return kPathTc;
+        return kPathAuto;
+    }();
+    return p;
+}
+
+int read_device_error() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return -1;
+    if (v) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    }
+    return v;
+}
+
+}  // namespace cq

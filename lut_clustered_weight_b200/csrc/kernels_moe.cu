@@ -145,38 +145,46 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
 // ------------------------------------------------------------------ combine
 // out[t, n] = sum_j w[t,j] * s_h[p] * sum_split part[split][p][n]  (j in order)
 //           + sum_s s_h[ps] * sum_split part_s[split][ps][n]
-__global__ void k_combine(CombineArgs a) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (int64_t)a.T * a.H) return;
-    const int t = (int)(i / a.H), n = (int)(i % a.H);
-    float acc = 0.0f;
-    for (int j = 0; j < a.topk; j++) {
-        const int p = a.inv_perm[t * a.topk + j];
-        float y = 0.0f;
-        for (int sp = 0; sp < a.plan_r.splits; sp++)
-            y += a.part_r[((int64_t)sp * a.R_routed + p) * a.H + n];
-        y *= a.h_scales[p];
-        if (a.y_dbg) a.y_dbg[(int64_t)p * a.H + n] = y;
-        acc += a.w[t * a.topk + j] * y;
-    }
-    for (int s = 0; s < a.n_shared; s++) {
+__global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
+    // slot counts of the shared-expert down launch, per (shared expert, row tile)
+    __shared__ int s_ns[4][256];
+    const int t = blockIdx.x;
+    const int nrt = a.n_shared ? a.plan_s.n_row_tiles : 0;
+    for (int i = threadIdx.x; i < a.n_shared * nrt; i += blockDim.x) {
+        const int s = i / nrt, rt = i - s * nrt;
         const int64_t lp = (int64_t)s * a.T + t;
-        float y = 0.0f;
-        const int ns = lut_splits_at(a.plan_s, lp, n);
-        for (int sp = 0; sp < ns; sp++)
-            y += a.part_s[((int64_t)sp * a.R_shared + lp) * a.H + n];
-        y *= a.h_scales[a.R_routed + lp];
-        if (a.y_dbg) a.y_dbg[(a.R_routed + lp) * a.H + n] = y;
-        acc += y;
+        s_ns[s][rt] = lut_splits_at(a.plan_s, lp, rt * a.plan_s.rows_per_rt);
     }
-    a.out[i] = acc;
+    __syncthreads();
+    for (int n = threadIdx.x; n < a.H; n += blockDim.x) {
+        float acc = 0.0f;
+        for (int j = 0; j < a.topk; j++) {
+            const int p = a.inv_perm[t * a.topk + j];
+            float y = 0.0f;
+            for (int sp = 0; sp < a.plan_r.splits; sp++)
+                y += a.part_r[((int64_t)sp * a.R_routed + p) * a.H + n];
+            y *= a.h_scales[p];
+            if (a.y_dbg) a.y_dbg[(int64_t)p * a.H + n] = y;
+            acc += a.w[t * a.topk + j] * y;
+        }
+        for (int s = 0; s < a.n_shared; s++) {
+            const int64_t lp = (int64_t)s * a.T + t;
+            float y = 0.0f;
+            const int ns = s_ns[s][n / a.plan_s.rows_per_rt];
+            for (int sp = 0; sp < ns; sp++)
+                y += a.part_s[((int64_t)sp * a.R_shared + lp) * a.H + n];
+            y *= a.h_scales[a.R_routed + lp];
+            if (a.y_dbg) a.y_dbg[(a.R_routed + lp) * a.H + n] = y;
+            acc += y;
+        }
+        a.out[(int64_t)t * a.H + n] = acc;
+    }
 }
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
-    const int64_t n = (int64_t)a.T * a.H;
-    if (n == 0) return cudaSuccess;
+    if ((int64_t)a.T * a.H == 0) return cudaSuccess;
     count_launch();
-    k_combine<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a);
+    k_combine<<<(unsigned)a.T, 256, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -99,10 +99,17 @@ __global__ void __launch_bounds__(kRqThreads) k_rq_swiglu(const SwigluArgs a) {
     const int tok = routed ? a.perm[p] / a.topk : (int)(lp % a.T);
     const float sx = a.x_scales[tok];
     const RowPart rp = row_part(I, log2b, rank, cs);
+    // slot counts of the gate/up launch for the row tiles of this CTA's columns
+    __shared__ int s_ns[kMaxK / 64];
+    const int rt0 = rp.e0 / P.rows_per_rt;
+    const int nrt = rp.n > 0 ? (rp.e0 + rp.n - 1) / P.rows_per_rt - rt0 + 1 : 0;
+    for (int i = threadIdx.x; i < nrt; i += kRqThreads)
+        s_ns[i] = lut_splits_at(P, lp, (rt0 + i) * P.rows_per_rt);
+    __syncthreads();
     for (int i = threadIdx.x; i < rp.n; i += kRqThreads) {
         const int n = rp.e0 + i;
         float g = 0.0f, u = 0.0f;
-        const int splits = lut_splits_at(P, lp, n);
+        const int splits = s_ns[n / P.rows_per_rt - rt0];
         for (int sp = 0; sp < splits; sp++) {
             const float2 v = *reinterpret_cast<const float2 *>(
                 part + ((int64_t)sp * rows + lp) * (2 * (int64_t)I) + 2 * n);

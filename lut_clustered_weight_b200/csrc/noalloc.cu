@@ -72,7 +72,7 @@ extern "C" CQ_API cq_status cq_lut_gemm_noalloc(const void *q, const float *s_x,
         return CQ_ERR_UNSUPPORTED;
     if (M == 0) return CQ_OK;
 
-    // same plan as cq_lut_gemm, so the two give the same result
+    // the mma.sync kernel with the plan cq_lut_gemm uses for it (M <= 16)
     const int nt = M <= 8 ? 1 : 2;
     const int tiles = (int)((M + 8 * nt - 1) / (8 * nt));
     const LutPlan P = plan_lut((int)N, (int)K, false, (int)std::min<int64_t>(M, 16), tiles,

@@ -53,6 +53,8 @@ extern "C" {
 
 CQ_API int64_t cq_launch_count(void) { return cq::g_launches.load(); }
 
+CQ_API int32_t cq_device_error(void) { return cq::read_device_error(); }
+
 CQ_API cq_status cq_timing_enable(int32_t on) {
     cq::g_timing.store(on ? 1 : 0);
     return CQ_OK;

@@ -91,6 +91,11 @@ LUT_CASES = [
     (40, 768, 128, 8),
     (5, 9728, 128, 4),
     (2, 14336, 64, 8),
+    # more than 16 rows and N % 128 == 0: the tcgen05 tensor-memory kernel
+    (64, 2048, 256, 4),
+    (130, 1408, 384, 8),
+    (300, 2560, 128, 4),
+    (257, 96, 256, 4),
 ]
 
 
@@ -163,6 +168,11 @@ SMALL_MOE = [
                    had_block_h=128, had_block_i=64, renormalize=0),
     synth.MoEShape("moe_one_token", H=128, I=128, E=4, top_k=1, n_shared=1, T=1, act_bits=4,
                    had_block_h=32, had_block_i=32),
+    # > 16 rows per expert: routed and shared experts on the tcgen05 kernel
+    synth.MoEShape("moe_tc_small", H=256, I=256, E=4, top_k=2, n_shared=1, T=80, act_bits=4,
+                   had_block_h=256, had_block_i=128, bias_expert=1, bias=1.0),
+    synth.MoEShape("moe_tc_small8", H=384, I=192, E=2, top_k=1, n_shared=0, T=40, act_bits=8,
+                   had_block_h=128, had_block_i=64),
 ]
 
 
