@@ -5,8 +5,10 @@
 //
 // CodeQuant2 Figure 4 describes the LUT kernel as a one-time LUT precompute
 // held in shared memory followed by table lookups.  Here:
-//  * One thread per weight row: thread t of the four "expand" warps owns row
-//    t of a 128-row tile, which is also lane t of tensor memory (TMEM).
+//  * Two threads per weight row: row t of a 128-row tile is lane t of tensor
+//    memory (TMEM); of the eight "expand" warps, warps w and w + 4 both serve
+//    TMEM lane quarter w, one taking the low and one the high 32 k of every
+//    64-k chunk.
 //  * PAIR mode (decode): the one-time precompute is a 256-entry pair table per
 //    row in shared memory -- entry b holds the two fp16 centroids selected by
 //    an index byte b (low nibble = even k).  Entry b of thread t sits at
@@ -17,13 +19,14 @@
 //    registers and looked up with byte permutes; no shared memory is spent on
 //    tables, which leaves room for wide activation tiles.
 //  * The looked-up fp16 weights of a 64-k chunk are stored to TMEM
-//    (tcgen05.st, 32 columns per row) and used as the A operand of
+//    (tcgen05.st, 32 columns per row and chunk) and used as the A operand of
 //    tcgen05.mma kind::f16; the activations (int codes converted to fp16,
 //    exact) are the B operand, a 128-byte-swizzled shared tile loaded by TMA.
 //    The fp32 accumulator lives in TMEM and is read back with tcgen05.ld.
-//  * Roles: warps 0-3 expand (and prefetch their rows' index bytes into
-//    registers); lane 0 of warp 4 issues the TMA loads and the MMAs.
-//    mbarriers connect them; every wait is bounded.
+//  * Roles: warps 0-7 expand (each thread streams its row's index bytes
+//    through a private cp.async ring) and write the accumulator back; lane 0
+//    of warp 8 issues the MMAs; lane 0 of warp 9 issues the TMA loads of the
+//    activation tiles.  mbarriers connect them; every wait is bounded.
 //  * Work is cut into (128-row tile x token tile) items and 64-k chunks,
 //    shared out like the mma.sync kernel (stream-K for uniform launches).
 #include <cuda.h>
@@ -41,7 +44,10 @@
 
 namespace cq {
 
-constexpr int kTcThreads = 160;      // 4 expand warps + 1 MMA / TMA warp
+constexpr int kTcExpand = 256;       // 8 expand warps: 2 per TMEM lane quarter
+constexpr int kWarpMma = 8;          // warp 8: TMEM allocation + MMA issue (lane 0)
+constexpr int kWarpTma = 9;          // warp 9: B tile loads (lane 0)
+constexpr int kTcThreads = 320;
 constexpr int kTcRows = 128;         // rows per tile (TMEM lanes)
 constexpr int kTcChunk = 64;         // k per chunk (32 TMEM columns of fp16 pairs)
 constexpr int kTcA = 8;              // A ring depth: TMEM, 32 columns per chunk
@@ -125,35 +131,32 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     uint8_t *sm = smem_raw + pad;
     constexpr uint32_t kBSlot = NTOK * 128;  // bytes of one B chunk tile
     constexpr int kTcB = TcB<NTOK>::n;
-    constexpr int kTcBLag = kTcB / 2;
     uint8_t *bslots = sm;                                     // [kTcB][NTOK][128 B]
-    uint8_t *tables = sm + kTcB * kBSlot;                     // PAIR: [256][128 threads] x 4 B
-    uint8_t *wring_raw = tables + (PAIR ? kPairTableBytes : 0);  // [stages][2][128] x 16 B
-    uint64_t *bars = reinterpret_cast<uint64_t *>(wring_raw + kTcWStages * 2 * kTcRows * 16);
+    uint8_t *tables = sm + kTcB * kBSlot;                     // PAIR: [256][128 rows] x 4 B
+    uint8_t *wring_raw = tables + (PAIR ? kPairTableBytes : 0);  // [stages][256 thr] x 16 B
+    uint64_t *bars = reinterpret_cast<uint64_t *>(wring_raw + kTcWStages * kTcExpand * 16);
     uint64_t *a_full = bars, *a_empty = bars + kTcA;
     uint64_t *b_full = bars + 2 * kTcA;
     uint64_t *d_full = b_full + kTcB, *d_empty = d_full + 1, *fin = d_full + 2;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(fin + 1);
-    int *s_stop = reinterpret_cast<int *>(s_tmem + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr uint32_t kTmemCols = 512;  // A ring 256 + accumulator NTOK (<= 256)
     const TcSchedule S{&L, &P};
     const int C = P.chunks_total;
 
-    if (warp == 4) {
+    if (warp == kWarpMma) {
         tmem_alloc(s_tmem, kTmemCols);
         tmem_relinquish();
         if (lane == 0) {
             for (int s = 0; s < kTcA; s++) {
-                mbar_init(&a_full[s], 4);  // one arrival per expand warp
+                mbar_init(&a_full[s], kTcExpand / 32);  // one arrival per expand warp
                 mbar_init(&a_empty[s], 1);
             }
             for (int s = 0; s < kTcB; s++) mbar_init(&b_full[s], 1);
             mbar_init(d_full, 1);
-            mbar_init(d_empty, 4);
+            mbar_init(d_empty, kTcExpand / 32);
             mbar_init(fin, 1);
-            *s_stop = 0;
             fence_barrier_init();
             prefetch_tmap(&tmB);
         }
@@ -182,16 +185,19 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     }
     const int nchunks = (int)(u1 - u0);
 
-    if (warp == 4) {
-        // ====================== TMA + MMA issuer (one thread) ======================
+    if (warp == kWarpTma) {
+        // ====================== B loads (one thread) ======================
         if (lane == 0 && nchunks > 0) {
-            constexpr uint32_t idesc = idesc_f16(kTcRows, NTOK);
-            TcCursor bc;  // chunk of the next B load
+            TcCursor bc;
             bc.init(u0, C);
             int64_t b_item = -1;
             int b_y = 0;
-            auto issue_b = [&](int j) {
+            for (int j = 0; j < nchunks; j++) {
                 const int s = j % kTcB;
+                if (j >= kTcB) {  // slot s was used by chunk j - kTcB
+                    const int jo = j - kTcB;
+                    if (!mbar_wait(&a_empty[jo % kTcA], (uint32_t)(jo / kTcA) & 1u)) break;
+                }
                 if (bc.w != b_item) {
                     int g, row0, nrows, rt;
                     S.item(bc.w, g, row0, nrows, rt);
@@ -201,15 +207,15 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 mbar_arrive_expect_tx(&b_full[s], kBSlot);
                 tma_load_2d(bslots + s * kBSlot, &tmB, bc.ch * kTcChunk, b_y, &b_full[s]);
                 bc.next(C);
-            };
-            TcCursor mc;  // chunk of the next MMA
-            mc.init(u0, C);
-            int issued = 0, consumed = 0;
-            for (int j = 0; j < kTcB - kTcBLag && j < nchunks; j++) {
-                issue_b(j);
-                issued++;
             }
-            int items = 0;
+        }
+    } else if (warp == kWarpMma) {
+        // ====================== MMA issuer (one thread) ======================
+        if (lane == 0 && nchunks > 0) {
+            constexpr uint32_t idesc = idesc_f16(kTcRows, NTOK);
+            TcCursor mc;
+            mc.init(u0, C);
+            int items = 0, consumed = 0;
             bool ok = true;
             for (int j = 0; j < nchunks && ok; j++) {
                 const int s = j % kTcA, sb = j % kTcB;
@@ -228,44 +234,31 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 for (int kk = 0; kk < kTcChunk / 16; kk++)
                     tc_mma_ts(tmem_d, tmem_a + s * 32 + kk * 8, bd + (uint64_t)(2 * kk), idesc,
                               (first && kk == 0) ? 0u : 1u);
-                tc_commit(&a_empty[s]);  // frees A slot s and B slot sb (= s)
+                tc_commit(&a_empty[s]);  // frees A slot s and B slot sb
                 if (last) {
                     tc_commit(d_full);
                     items++;
                 }
-                // load B of chunk j + kTcB - kTcBLag into the slot of chunk
-                // j - kTcBLag, whose MMAs were issued kTcBLag chunks ago
-                const int jn = j + kTcB - kTcBLag;
-                if (jn < nchunks) {
-                    if (jn >= kTcB) {  // the slot was used by chunk jn - kTcB
-                        const int jo = jn - kTcB;
-                        ok = mbar_wait(&a_empty[jo % kTcA], (uint32_t)(jo / kTcA) & 1u);
-                        static_assert(kTcA % TcB<NTOK>::n == 0, "B slots must divide A slots");
-                    }
-                    if (ok) {
-                        issue_b(jn);
-                        issued++;
-                    }
-                }
             }
-            if (!ok) atomicExch(s_stop, 1);
             // nothing may still be writing shared or tensor memory when the CTA
-            // leaves: wait for every issued TMA load and for all issued MMAs
-            for (int j = consumed; j < issued; j++)
+            // leaves: the B loads of chunks not consumed, and all MMAs
+            const int issued_max = nchunks;
+            for (int j = consumed; j < issued_max && j < consumed + kTcB; j++)
                 mbar_wait(&b_full[j % kTcB], (uint32_t)(j / kTcB) & 1u);
             tc_commit(fin);
             mbar_wait(fin, 0);
         }
     } else {
-        // ====================== expand warps: one thread per row ======================
-        const int t = tid;  // 0..127 = TMEM lane
-        const uint32_t lane_base = ((uint32_t)(warp * 32)) << 16;
+        // ====================== expand warps ======================
+        // warp w: TMEM lane quarter w % 4 (row t), half h = w / 4 of every
+        // 64-k chunk (16 index bytes -> 16 TMEM columns)
+        const int t = (warp & 3) * 32 + lane;  // row within the tile = TMEM lane
+        const int hf = warp >> 2;
+        const uint32_t lane_base = ((uint32_t)((warp & 3) * 32)) << 16;
         uint32_t *tab = reinterpret_cast<uint32_t *>(tables) + t;  // entry b at tab[b * 128]
         uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};      // PRMT mode tables
-        // per-thread ring of index bytes: stage st holds 2 x 16 B at
-        // wring[(st * 2 + r) * 128 + t] (consecutive threads -> consecutive 16 B)
         uint4 *wring = reinterpret_cast<uint4 *>(wring_raw);
-        TcCursor pc;  // chunk of the next index-byte copy
+        TcCursor pc;
         pc.init(u0, C);
         int64_t p_item = -1;
         const uint8_t *p_row = nullptr;
@@ -277,13 +270,11 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 S.row_ptrs(max(gg, 0), rtt, t, p_row, cbx, cc);
                 p_item = pc.w;
             }
-            const uint8_t *p = p_row;
-            const int k0 = pc.ch * kTcChunk;
+            const int k0 = pc.ch * kTcChunk + hf * 32;
             pc.next(C);
-            uint4 *dst = wring + (size_t)((j % kTcWStages) * 2) * kTcRows + t;
-            const bool h0 = k0 < L.K, h1 = k0 + 32 < L.K;  // ragged last chunk: zeros
-            cp_async16_zfill(dst, h0 ? p + k0 / 2 : p, h0 ? 16 : 0);
-            cp_async16_zfill(dst + kTcRows, h1 ? p + k0 / 2 + 16 : p, h1 ? 16 : 0);
+            const bool h0 = k0 < L.K;  // ragged last chunk: zeros
+            cp_async16_zfill(wring + (size_t)(j % kTcWStages) * kTcExpand + tid,
+                             h0 ? p_row + k0 / 2 : p_row, h0 ? 16 : 0);
         };
         for (int j = 0; j < kTcWStages - 1; j++) {
             if (j < nchunks) issue_w(j);
@@ -292,7 +283,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
         int64_t cur_w = -1;
         int g = 0, row0 = 0, nrows = 0, rt = 0, col = 0, items = 0;
         bool ok = true;
-        TcCursor wc;  // chunk being expanded
+        TcCursor wc;
         wc.init(u0, C);
         for (int j = 0; j < nchunks; j++) {
             const int64_t w = wc.w;
@@ -304,7 +295,8 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 const __half *cbp;
                 S.item(w, g, row0, nrows, rt);
                 S.row_ptrs(max(g, 0), rt, t, idxp, cbp, col);
-                // the one-time LUT precompute for this row
+                // the one-time LUT precompute for this row (both halves write the
+                // same table entries; each only reads after its own writes)
                 const uint4 c0v = *reinterpret_cast<const uint4 *>(cbp);
                 const uint4 c1v = *reinterpret_cast<const uint4 *>(cbp + 8);
                 const uint32_t cu[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
@@ -326,22 +318,21 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 }
             }
             cp_async_wait_group<kTcWStages - 2>();
-            const uint4 *src = wring + (size_t)((j % kTcWStages) * 2) * kTcRows + t;
-            const uint4 wa = src[0], wb = src[kTcRows];
+            const uint4 wv = wring[(size_t)(j % kTcWStages) * kTcExpand + tid];
             if (j + kTcWStages - 1 < nchunks) issue_w(j + kTcWStages - 1);
             cp_async_commit_group();
-            const uint32_t wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-            // 64 weights -> 32 fp16 pairs (k = 2b, 2b + 1 in column b)
-            uint32_t v[32];
+            const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+            // 32 weights -> 16 fp16 pairs (k = 2b, 2b + 1 in column b)
+            uint32_t v[16];
             if (PAIR) {
 #pragma unroll
-                for (int b = 0; b < 32; b++) {
+                for (int b = 0; b < 16; b++) {
                     const uint32_t byte = prmt(wd[b >> 2], 0u, 0x4440u | (uint32_t)(b & 3));
                     v[b] = tab[byte * kTcRows];
                 }
             } else {
 #pragma unroll
-                for (int q = 0; q < 8; q++) {
+                for (int q = 0; q < 4; q++) {
                     uint32_t h4[4];
                     dequant8(wd[q], lo, hi, h4);
                     v[4 * q] = h4[0];
@@ -356,29 +347,33 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 if (!ok) break;
                 tc_fence_after();
             }
-            tmem_st32(tmem_a + lane_base + s * 32, v);
+            tmem_st16(tmem_a + lane_base + s * 32 + hf * 16, v);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[s]);
             if (ch == C - 1 || j == nchunks - 1) {
-                // item done: D (NTOK fp32 columns of this row) -> partial sums
+                // item done: this warp's half of the NTOK fp32 columns -> partials
                 ok = mbar_wait(d_full, (uint32_t)items & 1u);
                 if (!ok) break;
                 tc_fence_after();
                 const int slot = P.streamk ? (int)(blockIdx.x - lut_cta_of_unit(P, cur_w * C))
                                            : (int)(blockIdx.x / P.n_row_tiles);
                 float *out = L.out + (int64_t)slot * L.out_split_stride;
+                constexpr int kHalf = NTOK >= 32 ? NTOK / 2 : 16;
+                const int cbeg = NTOK >= 32 ? hf * kHalf : 0;
+                if (NTOK >= 32 || hf == 0) {
 #pragma unroll 1
-                for (int c0 = 0; c0 < NTOK; c0 += 16) {
-                    uint32_t d[16];
-                    tmem_ld16(tmem_d + lane_base + c0, d);
-                    tmem_wait_ld();
+                    for (int c0 = cbeg; c0 < cbeg + kHalf; c0 += 16) {
+                        uint32_t d[16];
+                        tmem_ld16(tmem_d + lane_base + c0, d);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int q = 0; q < 16; q++)
-                        if (c0 + q < nrows)
-                            out[(int64_t)(row0 + c0 + q) * L.out_row_stride + col] =
-                                __uint_as_float(d[q]);
+                        for (int q = 0; q < 16; q++)
+                            if (c0 + q < nrows)
+                                out[(int64_t)(row0 + c0 + q) * L.out_row_stride + col] =
+                                    __uint_as_float(d[q]);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -388,13 +383,12 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
             }
         }
         cp_async_wait_group<0>();
-        if (!ok) atomicExch(s_stop, 1);
     }
     // ---- teardown: all MMAs and TMEM reads are complete before TMEM is freed
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 4) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------- host side
@@ -466,7 +460,7 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
     const bool pair = ntok <= 16;
     const int nb = ntok <= 128 ? 8 : 4;
     P.smem = 1024 + (size_t)nb * ntok * 128 + (pair ? kPairTableBytes : 0) +
-             (size_t)kTcWStages * 2 * kTcRows * 16 + 512;
+             (size_t)kTcWStages * kTcExpand * 16 + 512;
     P.tc = 1;
     return P;
 }

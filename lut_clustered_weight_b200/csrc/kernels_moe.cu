@@ -7,102 +7,121 @@
 namespace cq {
 
 // ------------------------------------------------------------------ routing
-// One CTA (1024 threads).  Top-k per token (one warp per token, descending,
-// ties to the lower expert id), softmax weights, per-expert counts and
-// offsets, a stable permutation of the slots t*k+j grouped by expert, its
-// inverse, and the per-expert prefix of token tiles used by the grouped GEMM.
-constexpr int kRouteThreads = 1024;
-constexpr int kRouteWarps = kRouteThreads / 32;
+// (1) k_topk: one warp per token, the token's logits held in registers:
+//     the k largest in descending order, ties to the lower expert id, and the
+//     softmax weights.
+// (2) k_group: one CTA: per-expert counts and offsets, a stable permutation
+//     of the slots t*k+j grouped by expert (each warp places a contiguous
+//     chunk of slots in slot order), its inverse, and the per-expert prefix of
+//     token tiles used by the grouped GEMM.
+constexpr int kTopkWarps = 8;
 
-__global__ void __launch_bounds__(kRouteThreads)
-k_route(const float *__restrict__ logits, int T, int E, int k, int renorm, int tile_rows,
-        int32_t *__restrict__ ids, float *__restrict__ w, int32_t *__restrict__ counts,
-        int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm,
-        int32_t *__restrict__ grp_tiles) {
-    __shared__ int32_t hist[kRouteWarps][kMaxExperts];
+__global__ void __launch_bounds__(kTopkWarps * 32)
+k_topk(const float *__restrict__ logits, int T, int E, int k, int renorm,
+       int32_t *__restrict__ ids, float *__restrict__ w) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * kTopkWarps + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float *l = logits + (int64_t)t * E;
+    constexpr int kPer = kMaxExperts / 32;
+    float v[kPer];
+    uint32_t taken = 0;  // bit i: expert i*32 + lane taken (or absent)
+#pragma unroll
+    for (int i = 0; i < kPer; i++) {
+        const int e = i * 32 + lane;
+        v[i] = e < E ? l[e] : -INFINITY;
+        if (e >= E) taken |= 1u << i;
+    }
+    float top0 = 0.0f, den_all = 0.0f;
+    float sel_l = 0.0f;  // lane j keeps the logit of choice j
+    int sel_e = 0;
+    for (int j = 0; j < k; j++) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < kPer; i++)
+            if (!((taken >> i) & 1u) && (be == 0x7fffffff || v[i] > bv)) {
+                bv = v[i];
+                be = i * 32 + lane;
+            }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (j == 0) top0 = bv;
+        if (lane == j) {
+            sel_l = bv;
+            sel_e = be;
+        }
+    }
+    if (!renorm) {
+        float part = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kPer; i++)
+            if (i * 32 + lane < E) part += expf(v[i] - top0);
+        den_all = warp_sum(part);
+    }
+    const float ex = lane < k ? expf(sel_l - top0) : 0.0f;
+    const float den = renorm ? warp_sum(ex) : den_all;
+    if (lane < k) {
+        ids[t * k + lane] = sel_e;
+        w[t * k + lane] = ex / den;
+    }
+}
+
+constexpr int kGroupThreads = 1024;
+constexpr int kGroupWarps = kGroupThreads / 32;
+
+__global__ void __launch_bounds__(kGroupThreads)
+k_group(const int32_t *__restrict__ ids, int T, int E, int k, int tile_rows,
+        int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+        int32_t *__restrict__ inv_perm, int32_t *__restrict__ grp_tiles) {
+    __shared__ int32_t hist[kGroupWarps][kMaxExperts];
     __shared__ int32_t s_off[kMaxExperts + 1];
     __shared__ int32_t s_tiles[kMaxExperts + 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int S = T * k;
-
-    // ---- top-k, one warp per token
-    for (int t = warp; t < T; t += kRouteWarps) {
-        const float *l = logits + (int64_t)t * E;
-        uint32_t taken[kMaxExperts / 32];
-#pragma unroll
-        for (int i = 0; i < kMaxExperts / 32; i++) taken[i] = 0;
-        float top0 = 0.0f;
-        float sel_l[16];
-        int sel_e[16];
-        for (int j = 0; j < k; j++) {
-            float bv = -INFINITY;
-            int be = 0x7fffffff;
-            for (int i = 0; i * 32 < E; i++) {
-                const int e = i * 32 + lane;
-                if (e < E && !((taken[i] >> lane) & 1u)) {
-                    const float v = l[e];
-                    if (be == 0x7fffffff || v > bv) { bv = v; be = e; }
-                }
-            }
-#pragma unroll
-            for (int o = 16; o; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                if (oe != 0x7fffffff &&
-                    (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
-                    bv = ov;
-                    be = oe;
-                }
-            }
-            if ((be & 31) == lane) taken[be >> 5] |= 1u << lane;
-            if (j == 0) top0 = bv;
-            sel_l[j] = bv;
-            sel_e[j] = be;
-        }
-        float den;
-        if (renorm) {
-            den = 0.0f;
-            for (int j = 0; j < k; j++) den += expf(sel_l[j] - top0);
-        } else {
-            float part = 0.0f;
-            for (int e = lane; e < E; e += 32) part += expf(l[e] - top0);
-            den = warp_sum(part);
-        }
-        if (lane == 0) {
-            for (int j = 0; j < k; j++) {
-                ids[t * k + j] = sel_e[j];
-                w[t * k + j] = expf(sel_l[j] - top0) / den;
-            }
-        }
-    }
-    // ---- per-warp histograms over contiguous slot chunks
-    for (int i = tid; i < kRouteWarps * kMaxExperts; i += kRouteThreads)
-        (&hist[0][0])[i] = 0;
-    __syncthreads();  // also orders the ids writes above (same block)
-    const int chunk = (S + kRouteWarps - 1) / kRouteWarps;
+    for (int i = tid; i < kGroupWarps * kMaxExperts; i += kGroupThreads) (&hist[0][0])[i] = 0;
+    __syncthreads();
+    const int chunk = (S + kGroupWarps - 1) / kGroupWarps;
     const int c0 = warp * chunk, c1 = min(S, c0 + chunk);
     for (int sl = c0 + lane; sl < c1; sl += 32) atomicAdd(&hist[warp][ids[sl]], 1);
     __syncthreads();
-    // ---- counts, offsets (exclusive scan), per-warp bases
     if (tid < E) {
         int c = 0;
-        for (int ww = 0; ww < kRouteWarps; ww++) c += hist[ww][tid];
+        for (int ww = 0; ww < kGroupWarps; ww++) c += hist[ww][tid];
         s_off[tid + 1] = c;
         s_tiles[tid + 1] = (c + tile_rows - 1) / tile_rows;
     }
     if (tid == 0) { s_off[0] = 0; s_tiles[0] = 0; }
     __syncthreads();
-    if (tid == 0) {
-        for (int e = 0; e < E; e++) {
-            s_off[e + 1] += s_off[e];
-            s_tiles[e + 1] += s_tiles[e];
+    if (warp == 0) {  // inclusive scans over E <= 256 entries, 8 per lane
+        int base_o = 0, base_t = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane + 1;
+            int vo = e <= E ? s_off[e] : 0, vt = e <= E ? s_tiles[e] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int uo = __shfl_up_sync(0xffffffffu, vo, o);
+                const int ut = __shfl_up_sync(0xffffffffu, vt, o);
+                if (lane >= o) { vo += uo; vt += ut; }
+            }
+            if (e <= E) { s_off[e] = vo + base_o; s_tiles[e] = vt + base_t; }
+            base_o += __shfl_sync(0xffffffffu, vo, 31);
+            base_t += __shfl_sync(0xffffffffu, vt, 31);
         }
     }
     __syncthreads();
     if (tid < E) {
         int base = s_off[tid];
         counts[tid] = s_off[tid + 1] - s_off[tid];
-        for (int ww = 0; ww < kRouteWarps; ww++) {
+        for (int ww = 0; ww < kGroupWarps; ww++) {
             const int h = hist[ww][tid];
             hist[ww][tid] = base;
             base += h;
@@ -113,7 +132,6 @@ k_route(const float *__restrict__ logits, int T, int E, int k, int renorm, int t
         grp_tiles[tid] = s_tiles[tid];
     }
     __syncthreads();
-    // ---- stable placement: each warp walks its chunk in slot order
     for (int sb = c0; sb < c1; sb += 32) {
         const int sl = sb + lane;
         const bool ok = sl < c1;
@@ -136,55 +154,77 @@ k_route(const float *__restrict__ logits, int T, int E, int k, int renorm, int t
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int tile_rows,
                          int32_t *ids, float *w, int32_t *counts, int32_t *offsets, int32_t *perm,
                          int32_t *inv_perm, int32_t *grp_tiles, cudaStream_t st) {
-    count_launch();
-    k_route<<<1, kRouteThreads, 0, st>>>(logits, T, E, k, renorm, tile_rows, ids, w, counts,
-                                          offsets, perm, inv_perm, grp_tiles);
+    count_launch(2);
+    k_topk<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, st>>>(logits, T, E, k,
+                                                                          renorm, ids, w);
+    k_group<<<1, kGroupThreads, 0, st>>>(ids, T, E, k, tile_rows, counts, offsets, perm, inv_perm,
+                                         grp_tiles);
     return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ combine
 // out[t, n] = sum_j w[t,j] * s_h[p] * sum_split part[split][p][n]  (j in order)
 //           + sum_s s_h[ps] * sum_split part_s[split][ps][n]
+// grid (T, ceil(H / 1024)); each thread 4 consecutive columns.
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
-    // slot counts of the shared-expert down launch, per (shared expert, row tile)
-    __shared__ int s_ns[4][256];
+    __shared__ int s_p[kMaxTopK];
+    __shared__ float s_c[kMaxTopK];   // w[t, j] (scale of row p applied separately)
+    __shared__ float s_sh[kMaxTopK];  // h scale of row p
+    __shared__ int s_ns[4][24];       // slot counts, shared expert x row tile of this block (<= 17)
     const int t = blockIdx.x;
-    const int nrt = a.n_shared ? a.plan_s.n_row_tiles : 0;
-    for (int i = threadIdx.x; i < a.n_shared * nrt; i += blockDim.x) {
-        const int s = i / nrt, rt = i - s * nrt;
-        const int64_t lp = (int64_t)s * a.T + t;
-        s_ns[s][rt] = lut_splits_at(a.plan_s, lp, rt * a.plan_s.rows_per_rt);
+    const int n0 = blockIdx.y * 1024;
+    if (threadIdx.x < a.topk) {
+        const int p = a.inv_perm[t * a.topk + threadIdx.x];
+        s_p[threadIdx.x] = p;
+        s_c[threadIdx.x] = a.w[t * a.topk + threadIdx.x];
+        s_sh[threadIdx.x] = a.h_scales[p];
+    }
+    const int rpt = a.n_shared ? a.plan_s.rows_per_rt : 1;
+    const int rt0 = n0 / rpt;
+    const int nrt = a.n_shared ? (min(n0 + 1023, a.H - 1)) / rpt - rt0 + 1 : 0;
+    if (threadIdx.x < a.n_shared * nrt) {
+        const int s = threadIdx.x / nrt, r = threadIdx.x - s * nrt;
+        s_ns[s][r] = lut_splits_at(a.plan_s, (int64_t)s * a.T + t, (rt0 + r) * rpt);
     }
     __syncthreads();
-    for (int n = threadIdx.x; n < a.H; n += blockDim.x) {
-        float acc = 0.0f;
-        for (int j = 0; j < a.topk; j++) {
-            const int p = a.inv_perm[t * a.topk + j];
-            float y = 0.0f;
-            for (int sp = 0; sp < a.plan_r.splits; sp++)
-                y += a.part_r[((int64_t)sp * a.R_routed + p) * a.H + n];
-            y *= a.h_scales[p];
-            if (a.y_dbg) a.y_dbg[(int64_t)p * a.H + n] = y;
-            acc += a.w[t * a.topk + j] * y;
+    const int n = n0 + 4 * threadIdx.x;
+    if (n >= a.H) return;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < a.topk; j++) {
+        const int p = s_p[j];
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < a.plan_r.splits; sp++) {
+            const float4 v = *reinterpret_cast<const float4 *>(
+                a.part_r + ((int64_t)sp * a.R_routed + p) * a.H + n);
+            y.x += v.x; y.y += v.y; y.z += v.z; y.w += v.w;
         }
-        for (int s = 0; s < a.n_shared; s++) {
-            const int64_t lp = (int64_t)s * a.T + t;
-            float y = 0.0f;
-            const int ns = s_ns[s][n / a.plan_s.rows_per_rt];
-            for (int sp = 0; sp < ns; sp++)
-                y += a.part_s[((int64_t)sp * a.R_shared + lp) * a.H + n];
-            y *= a.h_scales[a.R_routed + lp];
-            if (a.y_dbg) a.y_dbg[(a.R_routed + lp) * a.H + n] = y;
-            acc += y;
-        }
-        a.out[(int64_t)t * a.H + n] = acc;
+        const float sc = s_sh[j];
+        y.x *= sc; y.y *= sc; y.z *= sc; y.w *= sc;
+        if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + (int64_t)p * a.H + n) = y;
+        const float c = s_c[j];
+        acc.x += c * y.x; acc.y += c * y.y; acc.z += c * y.z; acc.w += c * y.w;
     }
+    for (int s = 0; s < a.n_shared; s++) {
+        const int64_t lp = (int64_t)s * a.T + t;
+        const int ns = s_ns[s][n / rpt - rt0];
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < ns; sp++) {
+            const float4 v = *reinterpret_cast<const float4 *>(
+                a.part_s + ((int64_t)sp * a.R_shared + lp) * a.H + n);
+            y.x += v.x; y.y += v.y; y.z += v.z; y.w += v.w;
+        }
+        const float sc = a.h_scales[a.R_routed + lp];
+        y.x *= sc; y.y *= sc; y.z *= sc; y.w *= sc;
+        if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + (a.R_routed + lp) * a.H + n) = y;
+        acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w;
+    }
+    *reinterpret_cast<float4 *>(a.out + (int64_t)t * a.H + n) = acc;
 }
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
     if ((int64_t)a.T * a.H == 0) return cudaSuccess;
     count_launch();
-    k_combine<<<(unsigned)a.T, 256, 0, st>>>(a);
+    k_combine<<<dim3((unsigned)a.T, (unsigned)((a.H + 1023) / 1024)), 256, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -34,36 +34,54 @@ CQ_DEV RowPart row_part(int K, int log2b, int rank, int csize) {
     return {u0 * ub, (u1 - u0) * ub};
 }
 
-// Rotate buf[0, n) (complete blocks), reduce the absmax over the cluster,
-// quantize and store this CTA's codes; rank 0 stores the scale.
-CQ_DEV void rq_finish(double *buf, RowPart part, int K, int log2b, int bits, uint8_t *qrow,
+// Rotate buf[0, n) (complete blocks), reduce the absmax over the row (across
+// the cluster when CLUSTER), quantize and store this CTA's codes; rank 0
+// stores the scale.
+template <bool CLUSTER>
+CQ_DEV void rq_finish(double *buf, RowPart part, int log2b, int bits, uint8_t *qrow,
                       float *s_out) {
     __shared__ double red[33];
     __shared__ double s_amax;
-    cg::cluster_group cluster = cg::this_cluster();
     block_fwht<kRqThreads>(buf, part.n, log2b);
-    const double a_loc = block_absmax<kRqThreads>(buf, part.n, red);
-    if (threadIdx.x == 0) s_amax = a_loc;
-    cluster.sync();
-    double A = 0.0;
-    const int cs = (int)cluster.num_blocks();
-    for (int r = 0; r < cs; r++) A = fmax(A, *cluster.map_shared_rank(&s_amax, r));
-    cluster.sync();  // every CTA has read every s_amax
+    double A = block_absmax<kRqThreads>(buf, part.n, red);
+    bool rank0 = true;
+    if (CLUSTER) {
+        cg::cluster_group cluster = cg::this_cluster();
+        if (threadIdx.x == 0) s_amax = A;
+        cluster.sync();
+        A = 0.0;
+        const int cs = (int)cluster.num_blocks();
+        for (int r = 0; r < cs; r++) A = fmax(A, *cluster.map_shared_rank(&s_amax, r));
+        cluster.sync();  // every CTA has read every s_amax
+        rank0 = cluster.block_rank() == 0;
+    }
     block_quantize_range<kRqThreads>(buf, part.n, part.e0, bits, A, qrow);
-    if (cluster.block_rank() == 0 && threadIdx.x == 0) {
+    if (rank0 && threadIdx.x == 0) {
         const int qmax = (1 << (bits - 1)) - 1;
         *s_out = A > 0.0 ? quant_scale(A, log2b, qmax) : 0.0f;
     }
-    (void)K;
+}
+
+template <bool CLUSTER>
+CQ_DEV void cluster_pos(int &cs, int &rank) {
+    if (CLUSTER) {
+        cg::cluster_group cluster = cg::this_cluster();
+        cs = (int)cluster.num_blocks();
+        rank = (int)cluster.block_rank();
+    } else {
+        cs = 1;
+        rank = 0;
+    }
 }
 
 // ------------------------------------------------------------------ x rows
+template <bool CLUSTER>
 __global__ void __launch_bounds__(kRqThreads)
 k_rq_x(const __half *__restrict__ x, int64_t ldx, int K, int log2b, int bits,
        uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s) {
     extern __shared__ __align__(16) double buf[];
-    cg::cluster_group cluster = cg::this_cluster();
-    const int cs = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
+    int cs, rank;
+    cluster_pos<CLUSTER>(cs, rank);
     const int64_t m = blockIdx.x / cs;
     const RowPart part = row_part(K, log2b, rank, cs);
     const __half *xr = x + m * ldx + part.e0;
@@ -78,16 +96,17 @@ k_rq_x(const __half *__restrict__ x, int64_t ldx, int K, int log2b, int bits,
         }
     }
     __syncthreads();
-    rq_finish(buf, part, K, log2b, bits, q + m * ldq, s + m);
+    rq_finish<CLUSTER>(buf, part, log2b, bits, q + m * ldq, s + m);
 }
 
 // ------------------------------------------------------------------ SwiGLU rows
 // Row p of the intermediate: g, u = sum of the split-K partials, scaled by the
 // token's s_x; h = fp16(silu(g) * u) (round to nearest even); then as above.
+template <bool CLUSTER>
 __global__ void __launch_bounds__(kRqThreads) k_rq_swiglu(const SwigluArgs a) {
     extern __shared__ __align__(16) double buf[];
-    cg::cluster_group cluster = cg::this_cluster();
-    const int cs = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
+    int cs, rank;
+    cluster_pos<CLUSTER>(cs, rank);
     const int64_t p = blockIdx.x / cs;
     const bool routed = p < a.R_routed;
     const int I = routed ? a.I : a.I_shared;
@@ -106,24 +125,123 @@ __global__ void __launch_bounds__(kRqThreads) k_rq_swiglu(const SwigluArgs a) {
     for (int i = threadIdx.x; i < nrt; i += kRqThreads)
         s_ns[i] = lut_splits_at(P, lp, (rt0 + i) * P.rows_per_rt);
     __syncthreads();
-    for (int i = threadIdx.x; i < rp.n; i += kRqThreads) {
-        const int n = rp.e0 + i;
-        float g = 0.0f, u = 0.0f;
-        const int splits = s_ns[n / P.rows_per_rt - rt0];
-        for (int sp = 0; sp < splits; sp++) {
-            const float2 v = *reinterpret_cast<const float2 *>(
-                part + ((int64_t)sp * rows + lp) * (2 * (int64_t)I) + 2 * n);
-            g += v.x;
-            u += v.y;
+    // batches of 4 elements per thread: all partial loads first, then the math
+    const int64_t slot_stride = rows * 2 * (int64_t)I;
+    const float *rowp = part + lp * (2 * (int64_t)I);
+    for (int i0 = 0; i0 < rp.n; i0 += 4 * kRqThreads) {
+        float2 acc[4];
+#pragma unroll
+        for (int f = 0; f < 4; f++) {
+            acc[f] = make_float2(0.f, 0.f);
+            const int i = i0 + f * kRqThreads + threadIdx.x;
+            if (i < rp.n) {
+                const int n = rp.e0 + i;
+                const int splits = s_ns[n / P.rows_per_rt - rt0];
+                for (int sp = 0; sp < splits; sp++) {
+                    const float2 v =
+                        *reinterpret_cast<const float2 *>(rowp + sp * slot_stride + 2 * n);
+                    acc[f].x += v.x;
+                    acc[f].y += v.y;
+                }
+            }
         }
-        g *= sx;
-        u *= sx;
-        const __half h = __float2half_rn(silu_mul(g, u));
-        if (a.h_dbg) reinterpret_cast<__half *>(a.h_dbg)[p * a.Imax + n] = h;
-        buf[i] = (double)__half2float(h);
+#pragma unroll
+        for (int f = 0; f < 4; f++) {
+            const int i = i0 + f * kRqThreads + threadIdx.x;
+            if (i < rp.n) {
+                const int n = rp.e0 + i;
+                const __half h = __float2half_rn(silu_mul(acc[f].x * sx, acc[f].y * sx));
+                if (a.h_dbg) reinterpret_cast<__half *>(a.h_dbg)[p * a.Imax + n] = h;
+                buf[i] = (double)__half2float(h);
+            }
+        }
     }
     __syncthreads();
-    rq_finish(buf, rp, I, log2b, a.bits, a.hq + p * a.ldhq, a.h_scales + p);
+    rq_finish<CLUSTER>(buf, rp, log2b, a.bits, a.hq + p * a.ldhq, a.h_scales + p);
+}
+
+// ------------------------------------------------------------------ one warp per row
+// For many short rows with rotation blocks of at most 256: no block barrier,
+// kWarpRows rows per CTA, each row in its warp's slice of shared memory.
+constexpr int kWarpRows = 4;
+
+__global__ void __launch_bounds__(kWarpRows * 32)
+k_rq_x_warp(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log2b, int bits,
+            uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s) {
+    extern __shared__ __align__(16) double wbuf[];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t m = (int64_t)blockIdx.x * kWarpRows + w;
+    if (m >= M) return;
+    double *buf = wbuf + (size_t)w * K;
+    const __half *xr = x + m * ldx;
+    for (int i = lane; i < K / 8; i += 32) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(xr + 8 * i);
+        const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float2 f = __half22float2(h[j]);
+            buf[8 * i + 2 * j] = (double)f.x;
+            buf[8 * i + 2 * j + 1] = (double)f.y;
+        }
+    }
+    __syncwarp();
+    const double A = warp_fwht_absmax(buf, K, log2b);
+    warp_quantize_row(buf, K, log2b, bits, A, q + m * ldq, s + m);
+}
+
+__global__ void __launch_bounds__(kWarpRows * 32) k_rq_swiglu_warp(const SwigluArgs a, int64_t R) {
+    extern __shared__ __align__(16) double wbuf[];
+    __shared__ int s_ns[kWarpRows][kMaxK / 64];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t p = (int64_t)blockIdx.x * kWarpRows + w;
+    if (p >= R) return;
+    const bool routed = p < a.R_routed;
+    const int I = routed ? a.I : a.I_shared;
+    const int log2b = routed ? a.log2b_i : a.log2b_i_shared;
+    const float *part = routed ? a.part_r : a.part_s;
+    const LutPlan &P = routed ? a.plan_r : a.plan_s;
+    const int64_t rows = routed ? a.R_routed : a.R_shared;
+    const int64_t lp = routed ? p : p - a.R_routed;
+    const int tok = routed ? a.perm[p] / a.topk : (int)(lp % a.T);
+    const float sx = a.x_scales[tok];
+    double *buf = wbuf + (size_t)w * a.Imax;
+    const int nrt = (I + P.rows_per_rt - 1) / P.rows_per_rt;
+    for (int i = lane; i < nrt; i += 32) s_ns[w][i] = lut_splits_at(P, lp, i * P.rows_per_rt);
+    __syncwarp();
+    const int64_t slot_stride = rows * 2 * (int64_t)I;
+    const float *rowp = part + lp * (2 * (int64_t)I);
+    for (int n0 = 0; n0 < I; n0 += 4 * 32) {
+        float2 acc[4];
+#pragma unroll
+        for (int f = 0; f < 4; f++) {
+            acc[f] = make_float2(0.f, 0.f);
+            const int n = n0 + f * 32 + lane;
+            if (n < I) {
+                const int ns = s_ns[w][n / P.rows_per_rt];
+                for (int sp = 0; sp < ns; sp++) {
+                    const float2 v = *reinterpret_cast<const float2 *>(rowp + sp * slot_stride + 2 * n);
+                    acc[f].x += v.x;
+                    acc[f].y += v.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int f = 0; f < 4; f++) {
+            const int n = n0 + f * 32 + lane;
+            if (n < I) {
+                const __half h = __float2half_rn(silu_mul(acc[f].x * sx, acc[f].y * sx));
+                if (a.h_dbg) reinterpret_cast<__half *>(a.h_dbg)[p * a.Imax + n] = h;
+                buf[n] = (double)__half2float(h);
+            }
+        }
+    }
+    __syncwarp();
+    const double A = warp_fwht_absmax(buf, I, log2b);
+    warp_quantize_row(buf, I, log2b, a.bits, A, a.hq + p * a.ldhq, a.h_scales + p);
+}
+
+static bool use_warp_rows(int64_t rows, int K, int log2b) {
+    return log2b <= 8 && K <= 4096 && rows >= 4LL * sm_count();
 }
 
 // ------------------------------------------------------------------ launchers
@@ -146,6 +264,11 @@ static cudaError_t launch_clustered(Kern kern, int64_t rows, int cs, size_t smem
                                     cudaStream_t st, Args... args) {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)(kMaxK * sizeof(double)));
+    if (cs == 1) {  // one CTA per row: a plain launch
+        count_launch();
+        kern<<<(unsigned)rows, kRqThreads, smem, st>>>(args...);
+        return cudaGetLastError();
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(rows * cs));
     cfg.blockDim = dim3(kRqThreads);
@@ -165,14 +288,36 @@ static cudaError_t launch_clustered(Kern kern, int64_t rows, int cs, size_t smem
 cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K, int log2b,
                                    int bits, void *q, int64_t ldq, float *s, cudaStream_t st) {
     if (M == 0) return cudaSuccess;
+    if (use_warp_rows(M, K, log2b)) {
+        const size_t smem = (size_t)kWarpRows * K * sizeof(double);
+        cudaFuncSetAttribute(k_rq_x_warp, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(kWarpRows * 4096 * sizeof(double)));
+        count_launch();
+        k_rq_x_warp<<<(unsigned)((M + kWarpRows - 1) / kWarpRows), kWarpRows * 32, smem, st>>>(
+            reinterpret_cast<const __half *>(x), ldx, M, K, log2b, bits,
+            reinterpret_cast<uint8_t *>(q), ldq, s);
+        return cudaGetLastError();
+    }
     const int cs = cluster_size(M, K, log2b);
-    return launch_clustered(k_rq_x, M, cs, part_smem(K, log2b, cs), st,
+    auto kern = cs == 1 ? k_rq_x<false> : k_rq_x<true>;
+    return launch_clustered(kern, M, cs, part_smem(K, log2b, cs), st,
                             reinterpret_cast<const __half *>(x), ldx, K, log2b, bits,
                             reinterpret_cast<uint8_t *>(q), ldq, s);
 }
 
 cudaError_t launch_swiglu_rq(const SwigluArgs &a, int64_t rows, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
+    const bool warp_r = a.R_routed == 0 || use_warp_rows(rows, a.I, a.log2b_i);
+    const bool warp_s = a.R_shared == 0 || use_warp_rows(rows, a.I_shared, a.log2b_i_shared);
+    if (warp_r && warp_s) {
+        const size_t smem = (size_t)kWarpRows * a.Imax * sizeof(double);
+        cudaFuncSetAttribute(k_rq_swiglu_warp, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(kWarpRows * 4096 * sizeof(double)));
+        count_launch();
+        k_rq_swiglu_warp<<<(unsigned)((rows + kWarpRows - 1) / kWarpRows), kWarpRows * 32, smem,
+                           st>>>(a, rows);
+        return cudaGetLastError();
+    }
     // one cluster size for the launch: the coarser of the two row kinds
     int cs = kMaxCluster;
     size_t smem = 0;
@@ -180,7 +325,8 @@ cudaError_t launch_swiglu_rq(const SwigluArgs &a, int64_t rows, cudaStream_t st)
     if (a.R_shared > 0) cs = std::min(cs, cluster_size(rows, a.I_shared, a.log2b_i_shared));
     if (a.R_routed > 0) smem = std::max(smem, part_smem(a.I, a.log2b_i, cs));
     if (a.R_shared > 0) smem = std::max(smem, part_smem(a.I_shared, a.log2b_i_shared, cs));
-    return launch_clustered(k_rq_swiglu, rows, cs, smem, st, a);
+    auto kern = cs == 1 ? k_rq_swiglu<false> : k_rq_swiglu<true>;
+    return launch_clustered(kern, rows, cs, smem, st, a);
 }
 
 }  // namespace cq

@@ -27,9 +27,12 @@ CQ_DEV void build_tables(const __half *cb, uint32_t (&lo)[4], uint32_t (&hi)[4])
 // halves of each plane and merged with a per-byte mask built from bit 3.
 CQ_DEV void dequant8(uint32_t w, const uint32_t (&lo)[4], const uint32_t (&hi)[4],
                      uint32_t (&h)[4]) {
-    const uint32_t s0 = w, s1 = w >> 16;
-    const uint32_t x0 = s0 ^ 0x8888u, x1 = s1 ^ 0x8888u;
-    const uint32_t w4 = w << 4;
+    // (the integer/logic pipe runs at half rate: the two right shifts and the
+    // left shift are multiplies, which issue to the FMA pipe)
+    const uint32_t wx = w ^ 0x88888888u;
+    const uint32_t s0 = w, s1 = __umulhi(w, 0x10000u);
+    const uint32_t x0 = wx, x1 = __umulhi(wx, 0x10000u);
+    const uint32_t w4 = w * 16u;
     const uint32_t m0 = prmt(w4, w, 0xD9C8);  // 0xFF in byte i iff nibble i >= 8
     const uint32_t m1 = prmt(w4, w, 0xFBEA);
     {

@@ -12,6 +12,34 @@
 
 namespace cq {
 
+// Index bits 8.. of the transform: one thread per column of R = b / 256
+// elements at stride 256 (R known at compile time so the column stays in
+// registers).
+template <int THREADS, int R>
+__device__ void fwht_columns(double *buf, int K, int log2b) {
+    const int ncols = K >> (log2b - 8);
+    for (int col = threadIdx.x; col < ncols; col += THREADS) {
+        const int blk = col >> 8, c = col & 255;
+        double *p = buf + ((size_t)blk << log2b) + c;
+        double v[R];
+#pragma unroll
+        for (int r = 0; r < R; r++) v[r] = p[256 * r];
+#pragma unroll
+        for (int h = 1; h < R; h <<= 1) {
+#pragma unroll
+            for (int r = 0; r < R; r++) {
+                if ((r & h) == 0) {
+                    const double a = v[r], d = v[r + h];
+                    v[r] = a + d;
+                    v[r + h] = a - d;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; r++) p[256 * r] = v[r];
+    }
+}
+
 // In-place Walsh-Hadamard transform (Sylvester order) of every contiguous
 // block of b = 2^log2b elements of buf[0, K).  K % 8 == 0, K % b == 0.
 //   levels 0..4 (index bits 0-4): lanes of a warp, via shuffles
@@ -61,31 +89,12 @@ __device__ void block_fwht(double *buf, int K, int log2b) {
         __syncthreads();
     }
     if (log2b > 8) {
-        const int R = 1 << (log2b - 8);  // 2..32 elements per column
-        const int ncols = K >> (log2b - 8);
-        for (int col = threadIdx.x; col < ncols; col += THREADS) {
-            const int blk = col >> 8, c = col & 255;
-            double *p = buf + ((size_t)blk << log2b) + c;
-            double v[32];
-#pragma unroll
-            for (int r = 0; r < 32; r++)
-                if (r < R) v[r] = p[256 * r];
-#pragma unroll
-            for (int h = 1; h < 32; h <<= 1) {
-                if (h < R) {
-#pragma unroll
-                    for (int r = 0; r < 32; r++) {
-                        if (r < R && (r & h) == 0) {
-                            double a = v[r], d = v[r + h];
-                            v[r] = a + d;
-                            v[r + h] = a - d;
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < 32; r++)
-                if (r < R) p[256 * r] = v[r];
+        switch (log2b - 8) {
+        case 1: fwht_columns<THREADS, 2>(buf, K, log2b); break;
+        case 2: fwht_columns<THREADS, 4>(buf, K, log2b); break;
+        case 3: fwht_columns<THREADS, 8>(buf, K, log2b); break;
+        case 4: fwht_columns<THREADS, 16>(buf, K, log2b); break;
+        default: fwht_columns<THREADS, 32>(buf, K, log2b); break;
         }
         __syncthreads();
     }
@@ -174,6 +183,80 @@ __device__ void block_quantize_range(const double *buf, int n, int e0, int bits,
             reinterpret_cast<char2 *>(qrow + e0)[p] = c;
         }
     }
+}
+
+// ---------------------------------------------------------------- one warp per row
+// Rotation blocks of b <= 256: the whole transform of a 256-aligned chunk is
+// inside one warp (index bits 0-4 across lanes, 5-7 in registers).  buf holds
+// the row (K doubles, K % 256 == 0 or a ragged last chunk); returns max |.|.
+CQ_DEV double warp_fwht_absmax(double *buf, int K, int log2b) {
+    const int lane = threadIdx.x & 31;
+    double amax = 0.0;
+    for (int base = 0; base < K; base += 256) {
+        double v[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const int k = base + lane + 32 * j;
+            v[j] = k < K ? buf[k] : 0.0;
+        }
+        for (int L = 0; L < (log2b < 5 ? log2b : 5); L++) {
+            const int bit = 1 << L;
+            const bool upper = lane & bit;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const double p = __shfl_xor_sync(0xffffffffu, v[j], bit);
+                v[j] = upper ? (p - v[j]) : (v[j] + p);
+            }
+        }
+        for (int L = 5; L < log2b; L++) {
+            const int h = 1 << (L - 5);
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if ((j & h) == 0) {
+                    const double a = v[j], c = v[j + h];
+                    v[j] = a + c;
+                    v[j + h] = a - c;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const int k = base + lane + 32 * j;
+            if (k < K) {
+                buf[k] = v[j];
+                amax = fmax(amax, fabs(v[j]));
+            }
+        }
+    }
+    __syncwarp();
+    return warp_max_d(amax);
+}
+
+// Quantize a rotated row held by one warp and store codes and scale.
+CQ_DEV void warp_quantize_row(const double *buf, int K, int log2b, int bits, double A,
+                              uint8_t *qrow, float *s_out) {
+    const int lane = threadIdx.x & 31;
+    const int qmax = (1 << (bits - 1)) - 1;
+    const long long Ai = __double2ll_rn(A * 16777216.0);
+    const double R = Ai > 0 ? __ddiv_rn((double)qmax, A) : 0.0;
+    const double2 *b2 = reinterpret_cast<const double2 *>(buf);
+    for (int p = lane; p < K / 2; p += 32) {
+        const double2 v = b2[p];
+        int q0 = 0, q1 = 0;
+        if (Ai > 0) {
+            q0 = quantize_fast(v.x, R, Ai, qmax);
+            q1 = quantize_fast(v.y, R, Ai, qmax);
+        }
+        if (bits == 4) {
+            qrow[p] = (uint8_t)((q0 & 15) | ((q1 & 15) << 4));
+        } else {
+            char2 c;
+            c.x = (char)q0;
+            c.y = (char)q1;
+            reinterpret_cast<char2 *>(qrow)[p] = c;
+        }
+    }
+    if (lane == 0) *s_out = Ai > 0 ? quant_scale(A, log2b, qmax) : 0.0f;
 }
 
 }  // namespace cq

@@ -46,6 +46,10 @@ RQ_CASES = [
     (5, 24, 1, 8, 1),
     (33, 64, 4, 4, 0),
     (0, 256, 256, 4, 0),
+    # many short rows with blocks of at most 256: one warp per row
+    (600, 1408, 128, 4, 8),
+    (700, 4096, 256, 8, 4),
+    (593, 64, 8, 4, 0),
 ]
 
 
@@ -173,6 +177,11 @@ SMALL_MOE = [
                    had_block_h=256, had_block_i=128, bias_expert=1, bias=1.0),
     synth.MoEShape("moe_tc_small8", H=384, I=192, E=2, top_k=1, n_shared=0, T=40, act_bits=8,
                    had_block_h=128, had_block_i=64),
+    # hundreds of rows: 256-token tiles and the warp-per-row SwiGLU kernel
+    synth.MoEShape("dense_many_rows", H=128, I=256, E=0, top_k=0, n_shared=1, T=600,
+                   act_bits=4, had_block_h=128, had_block_i=64),
+    synth.MoEShape("moe_many_rows", H=192, I=128, E=4, top_k=2, n_shared=1, T=320, act_bits=8,
+                   had_block_h=64, had_block_i=128, I_shared=256),
 ]
 
 
