@@ -16,8 +16,10 @@ Reported (one JSON line from rank 0):
   e2e         the same metric through the C-ABI calls with host buffers: the
               step's activations copied from pinned host memory and the
               outputs copied back inside the timed region
-  roofline    the dominant kernel (the LUT GEMM): algorithmic bytes over its
-              CUDA-event-timed launches, against the measured HBM copy peak
+  roofline    the dominant LUT GEMM kernel, from its CUDA-event-timed launches:
+              the mma.sync decode kernel as algorithmic bytes against the
+              measured HBM copy peak, the tensor-memory kernel (groups of more
+              than 16 rows) as flops against the measured dense bf16 peak
   cpu_baseline  the CPU oracle on the host cores, on a bounded token sample
 Multi-GPU: replicas only (each rank runs the whole workload on its own GPU);
 the timing is the max over ranks.
@@ -57,13 +59,11 @@ def workload_shapes(name):
         return [synth.CFG3]
     if name == "prefill_moe_e64_s2":
         return [synth.CFG4]
-    if name == "linear_m1_k2048":
-        return None
     raise SystemExit(f"unknown workload {name}")
 
 
 WORKLOADS = ["qwen3_4b_ffn_decode", "qwen3_30b_a3b_moe_decode", "mixtral_8x7b_moe",
-             "prefill_moe_e64_s2", "linear_m1_k2048"]
+             "prefill_moe_e64_s2"]
 
 
 def load_peaks():
@@ -101,26 +101,60 @@ def layer_alg(shape, counts=None):
     return nbytes, flops
 
 
-def lut_launch_bytes(shape, counts=None):
-    """Algorithmic bytes of every LUT GEMM launch in one layer call, in
-    launch order (gate/up routed, gate/up shared, down routed, down shared)."""
+def lut_launches(shape, counts=None):
+    """(algorithmic bytes, flops) of every LUT GEMM launch in one layer call,
+    in launch order: gate/up routed, gate/up shared, down routed, down shared."""
     s = shape
     T, H, I, bits = s.T, s.H, s.I, s.act_bits
-    out = []
     gu, dn = [], []
     if s.E:
-        b_gu = b_dn = 0
+        b_gu = b_dn = f_gu = f_dn = 0
         for c in counts:
             if c > 0:
                 b_gu += lut_alg_bytes(int(c), 2 * I, H, bits)
                 b_dn += lut_alg_bytes(int(c), H, I, bits)
-        gu.append(b_gu)
-        dn.append(b_dn)
+                f_gu += 2 * int(c) * 2 * I * H
+                f_dn += 2 * int(c) * H * I
+        gu.append((b_gu, f_gu))
+        dn.append((b_dn, f_dn))
     if s.n_shared:
-        gu.append(s.n_shared * lut_alg_bytes(T, 2 * s.I_shared, H, bits))
-        dn.append(s.n_shared * lut_alg_bytes(T, H, s.I_shared, bits))
-    out = gu + dn
-    return out
+        Is = s.I_shared
+        gu.append((s.n_shared * lut_alg_bytes(T, 2 * Is, H, bits), s.n_shared * 2 * T * 2 * Is * H))
+        dn.append((s.n_shared * lut_alg_bytes(T, H, Is, bits), s.n_shared * 2 * T * H * Is))
+    return gu + dn
+
+
+def lut_roofline(launch_alg, timed, steps, ms_step, peak_gbs, peak_tf, peak_kind):
+    """Roofline entry of the dominant LUT GEMM kernel.  launch_alg: (bytes,
+    flops) of each launch of one step, in launch order; timed: (kernel, ms) of
+    every timed launch over `steps` steps.  The mma.sync kernel (decode) is
+    bound by HBM: its algorithmic bytes over its time, against the copy peak.
+    The tensor-memory kernel (prefill) is bound by the tensor pipe: its flops
+    over its time, against the measured dense bf16 peak (fp16 runs at the
+    same tensor-core rate)."""
+    per = {}
+    for i, (kern, ms) in enumerate(timed):
+        b, f = launch_alg[i % len(launch_alg)]
+        e = per.setdefault(kern, [0, 0.0, 0.0, 0])
+        e[0] += b
+        e[1] += f
+        e[2] += ms
+        e[3] += 1
+    kern = max(per, key=lambda k: per[k][2])
+    b, f, ms, n = per[kern]
+    src = {"k_lut_mma": "kernels_lut.cu", "k_lut_tc": "kernels_lut_tc.cu"}[kern]
+    common = {"kernel": kern, "avg_launch_us": 1e3 * ms / n, "launches_timed": n,
+              "share_of_step": (ms / steps) / ms_step,
+              "kernels_timed": {k: {"launches": v[3], "ms": v[2]} for k, v in per.items()}}
+    if kern == "k_lut_mma":
+        a = b / (ms / 1e3) / 1e9
+        return {"bound": "hbm", "achieved": a, "peak": peak_gbs, "unit": "GB/s",
+                "frac": a / peak_gbs, "peak_source": f"{peak_kind} hbm_gbs",
+                "alg_bytes_per_launch": b / n, **common}, src
+    a = f / (ms / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": a, "peak": peak_tf, "unit": "TFLOP/s",
+            "frac": a / peak_tf, "peak_source": f"{peak_kind} bf16_tflops (burst; fp16 = bf16 rate)",
+            "alg_flops_per_launch": f / n, **common}, src
 
 
 # ---------------------------------------------------------------------------
@@ -272,8 +306,6 @@ def cpu_oracle_sample(shapes, inputs, budget_s):
 def run_reference(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
-    if args.workload == "linear_m1_k2048":
-        raise SystemExit("the reference arm runs the FFN / MoE workloads")
     shapes, inputs = workload_inputs(args.workload)
     for _ in range(args.warmup):
         cpu_oracle_sample(shapes, inputs, 0.0)
@@ -417,8 +449,7 @@ def main():
 
     # byte / flop accounting (routing counts of the synthetic inputs)
     counts = [L.counts(dev) for L in layers]
-    lut_bytes_step = sum(sum(lut_launch_bytes(L.s, c)) for L, c in zip(layers, counts))
-    lut_launches_step = sum(len(lut_launch_bytes(L.s, c)) for L, c in zip(layers, counts))
+    launch_alg = [a for L, c in zip(layers, counts) for a in lut_launches(L.s, c)]
     alg_bytes_step = sum(layer_alg(L.s, c)[0] for L, c in zip(layers, counts))
     alg_flops_step = sum(layer_alg(L.s, c)[1] for L, c in zip(layers, counts))
 
@@ -454,17 +485,12 @@ def main():
         step()
     torch.cuda.synchronize()
     cq.cq_timing_enable(False)
-    n_lut, lut_ms = cq.cq_timing_read()
-    assert n_lut == args.steps * lut_launches_step, (n_lut, lut_launches_step)
-    lut_gbs = args.steps * lut_bytes_step / (lut_ms / 1e3) / 1e9
-    traffic = profile_traffic(ROOT / "lut_clustered_weight_b200" / "csrc" / "kernels_lut.cu",
-                              ROOT / "profiles" / f"lut_gemm_{args.workload}.md")
-    roofline = {"bound": "hbm", "achieved": lut_gbs, "peak": peak_gbs, "unit": "GB/s",
-                "frac": lut_gbs / peak_gbs, "peak_source": f"{peak_kind} hbm_gbs",
-                "traffic": traffic, "kernel": "k_lut_mma",
-                "alg_bytes_per_launch": lut_bytes_step / lut_launches_step,
-                "avg_launch_us": 1e3 * lut_ms / n_lut, "launches_timed": n_lut,
-                "lut_share_of_step": (lut_ms / args.steps) / ms_step}
+    timed_launches = cq.cq_timing_read_launches()
+    assert len(timed_launches) == args.steps * len(launch_alg), (len(timed_launches), len(launch_alg))
+    roofline, kern_src = lut_roofline(launch_alg, timed_launches, args.steps, ms_step,
+                                      peak_gbs, peak_tf, peak_kind)
+    roofline["traffic"] = profile_traffic(ROOT / "lut_clustered_weight_b200" / "csrc" / kern_src,
+                                          ROOT / "profiles" / f"{roofline['kernel']}_{args.workload}.md")
 
     # ---- e2e: host buffers through the C-ABI, copies inside the timed region
     def step_e2e():
@@ -503,8 +529,9 @@ def main():
             "alg_bytes_per_step": alg_bytes_step, "alg_flops_per_step": alg_flops_step,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
-            "dtype_note": "int4/int8 codes and 4-bit indices; LUT weights as fp16 into "
-                          "mma.sync with fp32 accumulation; rotation exact in fp64",
+            "dtype_note": "int4/int8 codes and 4-bit indices; looked-up weights as fp16 "
+                          "into mma.sync (decode) or tcgen05 kind::f16 (more than 16 "
+                          "rows per group) with fp32 accumulation; rotation exact in fp64",
         }
         print(json.dumps(line), flush=True)
     if world > 1:

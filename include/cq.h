@@ -255,9 +255,21 @@ CQ_API cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *ro
  * cq_timing_read    waits for the recorded events, returns the number of timed
  *                   launches and their summed device time in ms, and clears
  *                   the record.  Returns CQ_ERR_CUDA if an event failed.
+ * cq_timing_read_launches
+ *                   the same record launch by launch, in launch order: for the
+ *                   first min(*n, cap) launches, kinds[i] (CQ_KERNEL_*: which
+ *                   LUT GEMM kernel ran) and ms[i] (device time; -1 if its
+ *                   events failed, and the call then returns CQ_ERR_CUDA).
+ *                   *n = number of recorded launches.  Host arrays of cap
+ *                   entries, owned by the caller (NULL allowed when cap = 0).
+ *                   Clears the record.
  * The timing record is the one piece of process-wide state in the library;
  * it is guarded by a mutex.  Enable it only around single-threaded use.
  */
+enum cq_kernel_kind {
+    CQ_KERNEL_LUT_MMA = 0, /* mma.sync kernel, register / shared lookup tables */
+    CQ_KERNEL_LUT_TC = 1   /* tcgen05 kernel, looked-up weights in tensor memory */
+};
 CQ_API int64_t cq_launch_count(void);
 
 /*
@@ -270,6 +282,7 @@ CQ_API int64_t cq_launch_count(void);
 CQ_API int32_t cq_device_error(void);
 CQ_API cq_status cq_timing_enable(int32_t on);
 CQ_API cq_status cq_timing_read(int64_t *launches, double *total_ms);
+CQ_API cq_status cq_timing_read_launches(int32_t *kinds, float *ms, int64_t cap, int64_t *n);
 
 #ifdef __cplusplus
 }

@@ -19,7 +19,8 @@ LIB_PATH = _PKG / "libcq_b200.so"
 # symbols declared in include/cq.h
 EXPORTS = ("cq_status_string", "cq_version", "cq_rotate_quantize", "cq_lut_gemm_workspace_size",
            "cq_lut_gemm", "cq_moe_ffn_workspace_size", "cq_moe_ffn", "cq_launch_count",
-           "cq_timing_enable", "cq_timing_read", "cq_lut_gemm_noalloc", "cq_device_error")
+           "cq_timing_enable", "cq_timing_read", "cq_lut_gemm_noalloc", "cq_device_error",
+           "cq_timing_read_launches")
 
 CQ_OK, CQ_ERR_INVALID_ARGUMENT, CQ_ERR_UNSUPPORTED, CQ_ERR_WORKSPACE, CQ_ERR_CUDA = range(5)
 
@@ -84,6 +85,8 @@ lib.cq_timing_enable.argtypes = [_I32]
 lib.cq_timing_enable.restype = ctypes.c_int
 lib.cq_timing_read.argtypes = [ctypes.POINTER(_I64), ctypes.POINTER(ctypes.c_double)]
 lib.cq_timing_read.restype = ctypes.c_int
+lib.cq_timing_read_launches.argtypes = [_P, _P, _I64, ctypes.POINTER(_I64)]
+lib.cq_timing_read_launches.restype = ctypes.c_int
 
 
 def cq_launch_count() -> int:
@@ -106,6 +109,21 @@ def cq_timing_read() -> tuple[int, float]:
     ms = ctypes.c_double(0.0)
     _check(lib.cq_timing_read(ctypes.byref(n), ctypes.byref(ms)), "cq_timing_read")
     return int(n.value), float(ms.value)
+
+
+KERNEL_KINDS = {0: "k_lut_mma", 1: "k_lut_tc"}   # cq_kernel_kind
+
+
+def cq_timing_read_launches(cap: int = 1 << 16) -> list[tuple[str, float]]:
+    """[(kernel, device ms)] of every timed LUT GEMM launch, in launch order;
+    clears the record."""
+    kinds = (ctypes.c_int32 * cap)()
+    ms = (ctypes.c_float * cap)()
+    n = _I64(0)
+    _check(lib.cq_timing_read_launches(kinds, ms, cap, ctypes.byref(n)), "cq_timing_read_launches")
+    if n.value > cap:
+        raise CQError(CQ_ERR_INVALID_ARGUMENT, f"cq_timing_read_launches: {n.value} > cap {cap}")
+    return [(KERNEL_KINDS[int(kinds[i])], float(ms[i])) for i in range(int(n.value))]
 
 
 def status_string(s: int) -> str:

@@ -53,4 +53,41 @@ CQ_DEV void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32
 // fp32 silu(g) * u
 CQ_DEV float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
+// ---------------------------------------------------------------- split-K slot sums
+CQ_DEV void vadd(float &a, float b) { a += b; }
+CQ_DEV void vadd(float2 &a, float2 b) {
+    a.x += b.x;
+    a.y += b.y;
+}
+CQ_DEV void vadd(float4 &a, float4 b) {
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+}
+
+// acc[f] += p[f][0] + p[f][stride] + ... (ns[f] slots, added in slot order),
+// for F independent sums at once: every round issues the loads of two slots
+// of all F sums before the first add, so 2F loads are in flight instead of a
+// chain of dependent round trips.
+template <int F, typename T>
+CQ_DEV void sum_slots(const T *const (&p)[F], const int (&ns)[F], int64_t stride, T (&acc)[F]) {
+    int nsmax = 0;
+#pragma unroll
+    for (int f = 0; f < F; f++) nsmax = max(nsmax, ns[f]);
+    for (int s0 = 0; s0 < nsmax; s0 += 2) {
+        T v[F][2];
+#pragma unroll
+        for (int f = 0; f < F; f++)
+#pragma unroll
+            for (int u = 0; u < 2; u++)
+                v[f][u] = s0 + u < ns[f] ? p[f][(int64_t)(s0 + u) * stride] : T{};
+#pragma unroll
+        for (int f = 0; f < F; f++)
+#pragma unroll
+            for (int u = 0; u < 2; u++)
+                if (s0 + u < ns[f]) vadd(acc[f], v[f][u]);
+    }
+}
+
 }  // namespace cq

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/cq.h"
+
 namespace cq {
 
 // ---------------------------------------------------------------- rotate + quantize
@@ -143,7 +145,7 @@ int sm_count();
 // ---------------------------------------------------------------- measurement aids
 void count_launch(int n = 1);
 bool timing_on();
-void timing_begin(cudaStream_t st);
+void timing_begin(cudaStream_t st, int kind);  // kind: CQ_KERNEL_*
 void timing_end(cudaStream_t st);
 
 }  // namespace cq

@@ -357,7 +357,7 @@ static cudaError_t launch_lut_t(const LutLaunch &L, const LutPlan &P, cudaStream
 cudaError_t launch_lut(const LutLaunch &L, const LutPlan &P, cudaStream_t st) {
     if (P.grid == 0 || (!P.streamk && L.max_tiles == 0)) return cudaSuccess;
     const bool timed = timing_on();
-    if (timed) timing_begin(st);
+    if (timed) timing_begin(st, CQ_KERNEL_LUT_MMA);
     count_launch();
     if (P.nt == 1)
         P.warps == 8 ? launch_lut_t<1, 8>(L, P, st) : launch_lut_t<1, 4>(L, P, st);
@@ -381,11 +381,12 @@ __global__ void __launch_bounds__(256) k_reduce_plain(const float *__restrict__ 
     __syncthreads();
     const int n = n0 + threadIdx.x;
     if (n >= N) return;
-    const int ns = s_ns[n / P.rows_per_rt - rt0];
     const int64_t i = m * N + n;
-    float acc = 0.0f;
-    for (int k = 0; k < ns; k++) acc += part[(int64_t)k * M * N + i];
-    y[i] = s[m] * acc;
+    const float *pp[1] = {part + i};
+    const int ns[1] = {s_ns[n / P.rows_per_rt - rt0]};
+    float acc[1] = {0.0f};
+    sum_slots<1>(pp, ns, M * N, acc);
+    y[i] = s[m] * acc[0];
 }
 
 cudaError_t launch_reduce_plain(const float *part, const LutPlan &P, int64_t M, int64_t N,

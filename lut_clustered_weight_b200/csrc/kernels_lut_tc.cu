@@ -44,18 +44,23 @@
 
 namespace cq {
 
-constexpr int kTcExpand = 256;       // 8 expand warps: 2 per TMEM lane quarter
-constexpr int kWarpMma = 8;          // warp 8: TMEM allocation + MMA issue (lane 0)
-constexpr int kWarpTma = 9;          // warp 9: B tile loads (lane 0)
+constexpr int kTcExpandWarps = 8;    // 2 per TMEM lane quarter: low / high half of a group
+constexpr int kTcExpand = kTcExpandWarps * 32;
+constexpr int kWarpMma = 8;          // TMEM allocation + MMA issue (lane 0)
+constexpr int kWarpTma = 9;          // B tile loads (lane 0)
 constexpr int kTcThreads = 320;
 constexpr int kTcRows = 128;         // rows per tile (TMEM lanes)
-constexpr int kTcChunk = 64;         // k per chunk (32 TMEM columns of fp16 pairs)
-constexpr int kTcA = 8;              // A ring depth: TMEM, 32 columns per chunk
-// B ring depth (shared memory, NTOK x 128 B per chunk); a B slot is freed by
-// the commit of the chunk that used it.  B for chunk j + B - B/2 is loaded
-// while chunk j is issued.
+constexpr int kTcChunk = 64;         // k per chunk: one B tile, 4 MMAs, 32 TMEM columns
+constexpr int kTcG = 4;              // chunks per group: the expand / A-ring unit (256 k)
+constexpr int kTcA = 2;              // A ring depth in groups (TMEM columns [0, 256))
+// B ring depth in chunks (shared memory, NTOK x 128 B per chunk); a B slot is
+// freed by the commit of the chunk that used it.
 template <int NTOK> struct TcB { static constexpr int n = NTOK <= 128 ? 8 : 4; };
-constexpr int kTcWStages = 16;       // index-byte ring: 15 chunks in flight per thread
+// Independent accumulators: a chain of small MMAs into one accumulator is
+// bound by the MMA latency, so tiles of few tokens spread the four K steps
+// of a chunk over four accumulators (summed in the epilogue).
+template <int NTOK> struct TcAcc { static constexpr int n = NTOK <= 32 ? 4 : 1; };
+constexpr int kTcWStages = 4;        // index-byte ring per thread, in groups (3 in flight)
 constexpr size_t kPairTableBytes = 256 * kTcRows * 4;  // 128 KB
 
 struct TcSchedule {
@@ -91,8 +96,10 @@ struct TcSchedule {
     CQ_DEV void row_ptrs(int g, int rt, int t, const uint8_t *&idx, const __half *&cb, int &col) const {
         const int64_t rowbytes = L->K / 2;
         if (L->dual) {
-            const int n = rt * 64 + (t & 63);
-            const bool up = t >= 64;
+            // gate and up rows of one output column in adjacent lanes, so the
+            // epilogue's stores of a warp cover 32 consecutive partial columns
+            const int n = rt * 64 + (t >> 1);
+            const bool up = t & 1;
             idx = (up ? L->idx1 : L->idx0) + (int64_t)g * L->w_stride + (int64_t)n * rowbytes;
             cb = reinterpret_cast<const __half *>(up ? L->cb1 : L->cb0) + (int64_t)g * L->cb_stride + n * 16;
             col = 2 * n + (up ? 1 : 0);
@@ -105,22 +112,71 @@ struct TcSchedule {
     }
 };
 
-// Walks a CTA's units in order: (work item w, chunk ch), dividing only when
-// the walk enters a new item.
-struct TcCursor {
-    int64_t w;
-    int ch;
-    CQ_DEV void init(int64_t u, int C) {
-        w = u / C;
-        ch = (int)(u - w * C);
-    }
-    CQ_DEV void next(int C) {
-        if (++ch == C) {
-            ch = 0;
-            ++w;
+// The chunks a CTA works through, as segments (work item, chunk range) cut
+// into groups of at most kTcG chunks (a group never spans two segments).
+// Stream-K (uniform launches): one contiguous range of units (item x chunk),
+// cut at item boundaries.  Fixed split (routed launches): pieces (item,
+// split) p = blockIdx.x, blockIdx.x + gridDim.x, ... below the number of
+// pieces the routing produced, so the grid stays one CTA per SM whatever the
+// tile count.  Every role of the CTA walks the same sequence.
+struct TcWalk {
+    const LutPlan *P;
+    int64_t w;        // work item of the current segment
+    int c0, gn;       // first chunk (item-relative) and chunk count of the group
+    int c_begin, c_end;
+    int slot;         // partial-sum slot the segment writes
+    int64_t nxt, lim;
+    bool valid;
+
+    CQ_DEV void init(const LutPlan &Pl, int64_t n_pieces) {
+        P = &Pl;
+        if (Pl.streamk) {
+            nxt = (int64_t)blockIdx.x * Pl.units / Pl.grid;
+            lim = ((int64_t)blockIdx.x + 1) * Pl.units / Pl.grid;
+        } else {
+            nxt = blockIdx.x;
+            lim = n_pieces;
         }
+        load();
+    }
+    CQ_DEV void load() {
+        valid = nxt < lim;
+        if (!valid) return;
+        const int C = P->chunks_total;
+        if (P->streamk) {
+            w = nxt / C;
+            c_begin = (int)(nxt - w * C);
+            const int64_t e = min(lim, (w + 1) * C);
+            c_end = (int)(e - w * C);
+            slot = (int)(blockIdx.x - lut_cta_of_unit(*P, w * C));
+            nxt = e;
+        } else {
+            w = nxt / P->splits;
+            const int sp = (int)(nxt - w * P->splits);
+            c_begin = sp * P->chunks_per_split;
+            c_end = min(C, c_begin + P->chunks_per_split);
+            slot = sp;
+            nxt += gridDim.x;
+        }
+        c0 = c_begin;
+        gn = min(kTcG, c_end - c0);
+    }
+    CQ_DEV bool seg_first() const { return c0 == c_begin; }
+    CQ_DEV bool seg_last() const { return c0 + gn == c_end; }
+    CQ_DEV void next() {
+        c0 += gn;
+        if (c0 >= c_end) load();
+        else gn = min(kTcG, c_end - c0);
     }
 };
+
+// Pieces of a fixed-split launch that hold rows (the routing decides how many
+// token tiles there are; the host only knows an upper bound).
+CQ_DEV int64_t tc_pieces(const LutLaunch &L, const LutPlan &P) {
+    if (P.streamk) return 0;
+    const int64_t tiles = min((int64_t)L.grp_tiles[L.G], (int64_t)L.max_tiles);
+    return tiles * P.n_row_tiles * P.splits;
+}
 
 template <int NTOK, bool PAIR>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -131,32 +187,37 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     uint8_t *sm = smem_raw + pad;
     constexpr uint32_t kBSlot = NTOK * 128;  // bytes of one B chunk tile
     constexpr int kTcB = TcB<NTOK>::n;
+    constexpr int kAcc = TcAcc<NTOK>::n;
     uint8_t *bslots = sm;                                     // [kTcB][NTOK][128 B]
     uint8_t *tables = sm + kTcB * kBSlot;                     // PAIR: [256][128 rows] x 4 B
-    uint8_t *wring_raw = tables + (PAIR ? kPairTableBytes : 0);  // [stages][256 thr] x 16 B
-    uint64_t *bars = reinterpret_cast<uint64_t *>(wring_raw + kTcWStages * kTcExpand * 16);
+    uint8_t *wring_raw = tables + (PAIR ? kPairTableBytes : 0);  // [stage][4][256 thr] x 16 B
+    uint64_t *bars = reinterpret_cast<uint64_t *>(wring_raw + kTcWStages * 4 * kTcExpand * 16);
     uint64_t *a_full = bars, *a_empty = bars + kTcA;
-    uint64_t *b_full = bars + 2 * kTcA;
-    uint64_t *d_full = b_full + kTcB, *d_empty = d_full + 1, *fin = d_full + 2;
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(fin + 1);
+    uint64_t *b_full = bars + 2 * kTcA, *b_empty = b_full + kTcB;
+    uint64_t *d_full = b_empty + kTcB, *d_empty = d_full + 1, *fin = d_full + 2;
+    uint64_t *tab_ready = fin + 1;  // [4]: PAIR table of a lane quarter built
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(tab_ready + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    constexpr uint32_t kTmemCols = 512;  // A ring 256 + accumulator NTOK (<= 256)
+    constexpr uint32_t kTmemCols = 512;  // A ring 256 + accumulators kAcc x NTOK (<= 256)
     const TcSchedule S{&L, &P};
-    const int C = P.chunks_total;
 
     if (warp == kWarpMma) {
         tmem_alloc(s_tmem, kTmemCols);
         tmem_relinquish();
         if (lane == 0) {
             for (int s = 0; s < kTcA; s++) {
-                mbar_init(&a_full[s], kTcExpand / 32);  // one arrival per expand warp
+                mbar_init(&a_full[s], kTcExpandWarps);
                 mbar_init(&a_empty[s], 1);
             }
-            for (int s = 0; s < kTcB; s++) mbar_init(&b_full[s], 1);
+            for (int s = 0; s < kTcB; s++) {
+                mbar_init(&b_full[s], 1);
+                mbar_init(&b_empty[s], 1);
+            }
             mbar_init(d_full, 1);
-            mbar_init(d_empty, kTcExpand / 32);
+            mbar_init(d_empty, kTcExpandWarps);
             mbar_init(fin, 1);
+            for (int qq = 0; qq < 4; qq++) mbar_init(&tab_ready[qq], 2);
             fence_barrier_init();
             prefetch_tmap(&tmB);
         }
@@ -165,76 +226,85 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const uint32_t tmem_a = tmem;                // columns [0, 256): A ring (8 x 32)
-    const uint32_t tmem_d = tmem + kTcA * 32;    // columns [256, 256 + NTOK): accumulator
+    const uint32_t tmem_a = tmem;                 // columns [0, 256): A ring (2 x 128)
+    const uint32_t tmem_d = tmem + kTcA * 128;    // columns [256, 256 + kAcc NTOK)
 
-    // ---- this CTA's units
-    int64_t u0, u1;
-    if (P.streamk) {
-        u0 = (int64_t)blockIdx.x * P.units / P.grid;
-        u1 = ((int64_t)blockIdx.x + 1) * P.units / P.grid;
-    } else {
-        const int rt = blockIdx.x % P.n_row_tiles;
-        const int split = blockIdx.x / P.n_row_tiles;
-        const int64_t w = (int64_t)blockIdx.y * P.n_row_tiles + rt;
-        u0 = w * C + (int64_t)split * P.chunks_per_split;
-        u1 = min(u0 + P.chunks_per_split, w * C + C);
-        int g, r0, nr, rtt;
-        S.item(w, g, r0, nr, rtt);
-        if (g < 0) u1 = u0;  // beyond the routed tiles: nothing to do
+    // ---- this CTA's groups and chunks (every thread walks the same sequence)
+    const int64_t n_pieces = tc_pieces(L, P);
+    int ngroups = 0, nchunks = 0;
+    {
+        TcWalk cnt;
+        cnt.init(P, n_pieces);
+        while (cnt.valid) {
+            ngroups += (cnt.c_end - cnt.c_begin + kTcG - 1) / kTcG;
+            nchunks += cnt.c_end - cnt.c_begin;
+            cnt.c0 = cnt.c_end;
+            cnt.next();
+        }
     }
-    const int nchunks = (int)(u1 - u0);
 
     if (warp == kWarpTma) {
         // ====================== B loads (one thread) ======================
         if (lane == 0 && nchunks > 0) {
-            TcCursor bc;
-            bc.init(u0, C);
+            TcWalk bw;
+            bw.init(P, n_pieces);
             int64_t b_item = -1;
             int b_y = 0;
-            for (int j = 0; j < nchunks; j++) {
-                const int s = j % kTcB;
-                if (j >= kTcB) {  // slot s was used by chunk j - kTcB
-                    const int jo = j - kTcB;
-                    if (!mbar_wait(&a_empty[jo % kTcA], (uint32_t)(jo / kTcA) & 1u)) break;
-                }
-                if (bc.w != b_item) {
+            bool ok = true;
+            for (int jc = 0; bw.valid && ok; bw.next()) {
+                if (bw.w != b_item) {
                     int g, row0, nrows, rt;
-                    S.item(bc.w, g, row0, nrows, rt);
-                    b_item = bc.w;
+                    S.item(bw.w, g, row0, nrows, rt);
+                    b_item = bw.w;
                     b_y = b_row_mod > 0 ? row0 % b_row_mod : row0;
                 }
-                mbar_arrive_expect_tx(&b_full[s], kBSlot);
-                tma_load_2d(bslots + s * kBSlot, &tmB, bc.ch * kTcChunk, b_y, &b_full[s]);
-                bc.next(C);
+                for (int i = 0; i < bw.gn; i++, jc++) {
+                    const int s = jc % kTcB;
+                    if (jc >= kTcB && !mbar_wait(&b_empty[s], (uint32_t)(jc / kTcB - 1) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&b_full[s], kBSlot);
+                    tma_load_2d(bslots + s * kBSlot, &tmB, (bw.c0 + i) * kTcChunk, b_y, &b_full[s]);
+                }
             }
         }
     } else if (warp == kWarpMma) {
         // ====================== MMA issuer (one thread) ======================
         if (lane == 0 && nchunks > 0) {
             constexpr uint32_t idesc = idesc_f16(kTcRows, NTOK);
-            TcCursor mc;
-            mc.init(u0, C);
-            int items = 0, consumed = 0;
+            TcWalk mw;
+            mw.init(P, n_pieces);
+            int items = 0, consumed = 0, jc = 0;
             bool ok = true;
-            for (int j = 0; j < nchunks && ok; j++) {
-                const int s = j % kTcA, sb = j % kTcB;
-                const int ch = mc.ch;
-                mc.next(C);
-                const bool first = (j == 0) || ch == 0;
-                const bool last = (j == nchunks - 1) || ch == C - 1;
+            for (int gi = 0; mw.valid && ok; gi++, mw.next()) {
+                const int gs = gi % kTcA;
+                const bool first = mw.seg_first(), last = mw.seg_last();
                 if (first && items > 0) ok = mbar_wait(d_empty, (uint32_t)(items - 1) & 1u);
-                ok = ok && mbar_wait(&a_full[s], (uint32_t)(j / kTcA) & 1u) &&
-                     mbar_wait(&b_full[sb], (uint32_t)(j / kTcB) & 1u);
+                ok = ok && mbar_wait(&a_full[gs], (uint32_t)(gi / kTcA) & 1u);
                 if (!ok) break;
-                consumed++;
                 tc_fence_after();
-                const uint64_t bd = smem_desc_sw128(smem_u32(bslots + sb * kBSlot));
+                for (int i = 0; i < mw.gn; i++, jc++) {
+                    const int sb = jc % kTcB;
+                    if (!mbar_wait(&b_full[sb], (uint32_t)(jc / kTcB) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    consumed++;
+                    tc_fence_after();
+                    const uint64_t bd = smem_desc_sw128(smem_u32(bslots + sb * kBSlot));
+                    const bool fresh = first && i == 0;
 #pragma unroll
-                for (int kk = 0; kk < kTcChunk / 16; kk++)
-                    tc_mma_ts(tmem_d, tmem_a + s * 32 + kk * 8, bd + (uint64_t)(2 * kk), idesc,
-                              (first && kk == 0) ? 0u : 1u);
-                tc_commit(&a_empty[s]);  // frees A slot s and B slot sb
+                    for (int kk = 0; kk < kTcChunk / 16; kk++) {
+                        const uint32_t dcol = (uint32_t)((kk % kAcc) * NTOK);
+                        tc_mma_ts(tmem_d + dcol, tmem_a + gs * 128 + i * 32 + kk * 8,
+                                  bd + (uint64_t)(2 * kk), idesc,
+                                  (fresh && kk < kAcc) ? 0u : 1u);
+                    }
+                    tc_commit(&b_empty[sb]);
+                }
+                if (!ok) break;
+                tc_commit(&a_empty[gs]);
                 if (last) {
                     tc_commit(d_full);
                     items++;
@@ -242,144 +312,172 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
             }
             // nothing may still be writing shared or tensor memory when the CTA
             // leaves: the B loads of chunks not consumed, and all MMAs
-            const int issued_max = nchunks;
-            for (int j = consumed; j < issued_max && j < consumed + kTcB; j++)
+            for (int j = consumed; j < nchunks && j < consumed + kTcB; j++)
                 mbar_wait(&b_full[j % kTcB], (uint32_t)(j / kTcB) & 1u);
             tc_commit(fin);
             mbar_wait(fin, 0);
         }
     } else {
         // ====================== expand warps ======================
-        // warp w: TMEM lane quarter w % 4 (row t), half h = w / 4 of every
-        // 64-k chunk (16 index bytes -> 16 TMEM columns)
-        const int t = (warp & 3) * 32 + lane;  // row within the tile = TMEM lane
-        const int hf = warp >> 2;
-        const uint32_t lane_base = ((uint32_t)((warp & 3) * 32)) << 16;
+        // warp e: TMEM lane quarter q = e % 4 (row t), half h = e / 4 of every
+        // group: chunks 2h and 2h + 1, i.e. 64 index bytes -> 64 TMEM columns
+        const int q = warp & 3, h = warp >> 2;
+        const int t = q * 32 + lane;  // row within the tile = TMEM lane
+        const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
         uint32_t *tab = reinterpret_cast<uint32_t *>(tables) + t;  // entry b at tab[b * 128]
         uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};      // PRMT mode tables
         uint4 *wring = reinterpret_cast<uint4 *>(wring_raw);
-        TcCursor pc;
-        pc.init(u0, C);
+        // producer: this thread's index bytes of the coming groups (3 ahead)
+        TcWalk pw;
+        pw.init(P, n_pieces);
+        int gp = 0;
         int64_t p_item = -1;
         const uint8_t *p_row = nullptr;
-        auto issue_w = [&](int j) {
-            if (pc.w != p_item) {
-                int gg, r0, nr, rtt, cc;
-                S.item(pc.w, gg, r0, nr, rtt);
-                const __half *cbx;
-                S.row_ptrs(max(gg, 0), rtt, t, p_row, cbx, cc);
-                p_item = pc.w;
+        auto issue_group = [&]() {
+            if (pw.valid) {
+                if (pw.w != p_item) {
+                    int gg, r0, nr, rtt, cc;
+                    S.item(pw.w, gg, r0, nr, rtt);
+                    const __half *cbx;
+                    S.row_ptrs(max(gg, 0), rtt, t, p_row, cbx, cc);
+                    p_item = pw.w;
+                }
+                uint4 *dst = wring + (size_t)(gp % kTcWStages) * 4 * kTcExpand + tid;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    // piece i: k = c0*64 + 128h + 32i .. +32 (chunk 2h + i/2 of the group)
+                    const int k0 = pw.c0 * kTcChunk + 128 * h + 32 * i;
+                    const bool live = (2 * h + (i >> 1)) < pw.gn && k0 < L.K;
+                    cp_async16_zfill(dst + i * kTcExpand, live ? p_row + k0 / 2 : p_row,
+                                     live ? 16 : 0);
+                }
+                pw.next();
+                gp++;
             }
-            const int k0 = pc.ch * kTcChunk + hf * 32;
-            pc.next(C);
-            const bool h0 = k0 < L.K;  // ragged last chunk: zeros
-            cp_async16_zfill(wring + (size_t)(j % kTcWStages) * kTcExpand + tid,
-                             h0 ? p_row + k0 / 2 : p_row, h0 ? 16 : 0);
-        };
-        for (int j = 0; j < kTcWStages - 1; j++) {
-            if (j < nchunks) issue_w(j);
             cp_async_commit_group();
-        }
-        int64_t cur_w = -1;
+        };
+        for (int i = 0; i < kTcWStages - 1; i++) issue_group();
+
         int g = 0, row0 = 0, nrows = 0, rt = 0, col = 0, items = 0;
         bool ok = true;
-        TcCursor wc;
-        wc.init(u0, C);
-        for (int j = 0; j < nchunks; j++) {
-            const int64_t w = wc.w;
-            const int ch = wc.ch;
-            wc.next(C);
-            if (w != cur_w) {
-                cur_w = w;
+        TcWalk cw;
+        cw.init(P, n_pieces);
+        for (int gi = 0; cw.valid; gi++, cw.next()) {
+            const int gs = gi % kTcA;
+            if (cw.seg_first()) {
                 const uint8_t *idxp;
                 const __half *cbp;
-                S.item(w, g, row0, nrows, rt);
+                S.item(cw.w, g, row0, nrows, rt);
                 S.row_ptrs(max(g, 0), rt, t, idxp, cbp, col);
-                // the one-time LUT precompute for this row (both halves write the
-                // same table entries; each only reads after its own writes)
+                // the one-time LUT precompute for this row
                 const uint4 c0v = *reinterpret_cast<const uint4 *>(cbp);
                 const uint4 c1v = *reinterpret_cast<const uint4 *>(cbp + 8);
                 const uint32_t cu[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
                 if (PAIR) {
+                    // the two warps of the quarter build half of the table each
 #pragma unroll 1
-                    for (int h = 0; h < 16; h++) {
-                        const uint32_t hv = (uint32_t)__half_as_ushort(cbp[h]);
+                    for (int hh = 8 * h; hh < 8 * h + 8; hh++) {
+                        const uint32_t hv = (uint32_t)__half_as_ushort(cbp[hh]);
 #pragma unroll
                         for (int l = 0; l < 16; l++)
-                            tab[(h * 16 + l) * kTcRows] =
+                            tab[(hh * 16 + l) * kTcRows] =
                                 prmt(cu[l >> 1], hv, (l & 1) ? 0x5432u : 0x5410u);
                     }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tab_ready[q]);
+                    ok = mbar_wait(&tab_ready[q], (uint32_t)items & 1u);
+                    if (!ok) break;
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 4; q++) {
-                        lo[q] = prmt(cu[2 * q], cu[2 * q + 1], 0x6420);
-                        hi[q] = prmt(cu[2 * q], cu[2 * q + 1], 0x7531);
+                    for (int qq = 0; qq < 4; qq++) {
+                        lo[qq] = prmt(cu[2 * qq], cu[2 * qq + 1], 0x6420);
+                        hi[qq] = prmt(cu[2 * qq], cu[2 * qq + 1], 0x7531);
                     }
                 }
             }
             cp_async_wait_group<kTcWStages - 2>();
-            const uint4 wv = wring[(size_t)(j % kTcWStages) * kTcExpand + tid];
-            if (j + kTcWStages - 1 < nchunks) issue_w(j + kTcWStages - 1);
-            cp_async_commit_group();
-            const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
-            // 32 weights -> 16 fp16 pairs (k = 2b, 2b + 1 in column b)
-            uint32_t v[16];
-            if (PAIR) {
+            uint32_t wd[16];
+            {
+                const uint4 *src = wring + (size_t)(gi % kTcWStages) * 4 * kTcExpand + tid;
 #pragma unroll
-                for (int b = 0; b < 16; b++) {
-                    const uint32_t byte = prmt(wd[b >> 2], 0u, 0x4440u | (uint32_t)(b & 3));
-                    v[b] = tab[byte * kTcRows];
-                }
-            } else {
-#pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    uint32_t h4[4];
-                    dequant8(wd[q], lo, hi, h4);
-                    v[4 * q] = h4[0];
-                    v[4 * q + 1] = h4[1];
-                    v[4 * q + 2] = h4[2];
-                    v[4 * q + 3] = h4[3];
+                for (int i = 0; i < 4; i++) {
+                    const uint4 v4 = src[i * kTcExpand];
+                    wd[4 * i] = v4.x;
+                    wd[4 * i + 1] = v4.y;
+                    wd[4 * i + 2] = v4.z;
+                    wd[4 * i + 3] = v4.w;
                 }
             }
-            const int s = j % kTcA;
-            if (j >= kTcA) {
-                ok = mbar_wait(&a_empty[s], (uint32_t)(j / kTcA - 1) & 1u);
+            issue_group();
+            if (2 * h < cw.gn) {
+                // 128 weights -> 64 fp16 pairs (k = 2b, 2b + 1 in column b)
+                uint32_t v[64];
+                if (PAIR) {
+#pragma unroll
+                    for (int b = 0; b < 64; b++) {
+                        const uint32_t byte = prmt(wd[b >> 2], 0u, 0x4440u | (uint32_t)(b & 3));
+                        v[b] = tab[byte * kTcRows];
+                    }
+                } else {
+#pragma unroll
+                    for (int qq = 0; qq < 16; qq++) {
+                        uint32_t h4[4];
+                        dequant8(wd[qq], lo, hi, h4);
+                        v[4 * qq] = h4[0];
+                        v[4 * qq + 1] = h4[1];
+                        v[4 * qq + 2] = h4[2];
+                        v[4 * qq + 3] = h4[3];
+                    }
+                }
+                if (gi >= kTcA) {
+                    ok = mbar_wait(&a_empty[gs], (uint32_t)(gi / kTcA - 1) & 1u);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                const uint32_t ta = tmem_a + lane_base + gs * 128 + h * 64;
+                tmem_st32(ta, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
+                if (2 * h + 1 < cw.gn)
+                    tmem_st32(ta + 32, *reinterpret_cast<const uint32_t(*)[32]>(&v[32]));
+                tmem_wait_st();
+            } else if (gi >= kTcA) {
+                // nothing to store (short group), but the slot must be free
+                // before this warp reports it filled
+                ok = mbar_wait(&a_empty[gs], (uint32_t)(gi / kTcA - 1) & 1u);
                 if (!ok) break;
-                tc_fence_after();
             }
-            tmem_st16(tmem_a + lane_base + s * 32 + hf * 16, v);
-            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[s]);
-            if (ch == C - 1 || j == nchunks - 1) {
-                // item done: this warp's half of the NTOK fp32 columns -> partials
+            if (lane == 0) mbar_arrive(&a_full[gs]);
+            if (cw.seg_last()) {
+                // segment done: this warp's half of the NTOK fp32 columns -> partials
                 ok = mbar_wait(d_full, (uint32_t)items & 1u);
                 if (!ok) break;
                 tc_fence_after();
-                const int slot = P.streamk ? (int)(blockIdx.x - lut_cta_of_unit(P, cur_w * C))
-                                           : (int)(blockIdx.x / P.n_row_tiles);
-                float *out = L.out + (int64_t)slot * L.out_split_stride;
-                constexpr int kHalf = NTOK >= 32 ? NTOK / 2 : 16;
-                const int cbeg = NTOK >= 32 ? hf * kHalf : 0;
-                if (NTOK >= 32 || hf == 0) {
+                float *out = L.out + (int64_t)cw.slot * L.out_split_stride;
+                constexpr int kEpi = NTOK >= 32 ? NTOK / 2 : 16;
+                const int cbeg = h * kEpi;
+                if (cbeg < NTOK) {
 #pragma unroll 1
-                    for (int c0 = cbeg; c0 < cbeg + kHalf; c0 += 16) {
-                        uint32_t d[16];
-                        tmem_ld16(tmem_d + lane_base + c0, d);
+                    for (int c0 = cbeg; c0 < cbeg + kEpi; c0 += 16) {
+                        uint32_t d[kAcc][16];
+#pragma unroll
+                        for (int a = 0; a < kAcc; a++)
+                            tmem_ld16(tmem_d + lane_base + a * NTOK + c0, d[a]);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int q = 0; q < 16; q++)
-                            if (c0 + q < nrows)
-                                out[(int64_t)(row0 + c0 + q) * L.out_row_stride + col] =
-                                    __uint_as_float(d[q]);
+                        for (int qq = 0; qq < 16; qq++) {
+                            float acc = __uint_as_float(d[0][qq]);
+#pragma unroll
+                            for (int a = 1; a < kAcc; a++) acc += __uint_as_float(d[a][qq]);
+                            if (c0 + qq < nrows)
+                                out[(int64_t)(row0 + c0 + qq) * L.out_row_stride + col] = acc;
+                        }
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(d_empty);
                 items++;
-                cur_w = -1;
             }
         }
         cp_async_wait_group<0>();
@@ -455,12 +553,13 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
         splits = std::max(1, std::min(splits, C));
         P.chunks_per_split = (C + splits - 1) / splits;
         P.splits = (C + P.chunks_per_split - 1) / P.chunks_per_split;
-        P.grid = P.n_row_tiles * P.splits;
+        // persistent: at most one CTA per SM, striding over the pieces
+        P.grid = (int)std::min<int64_t>(capacity, base * P.splits);
     }
     const bool pair = ntok <= 16;
     const int nb = ntok <= 128 ? 8 : 4;
     P.smem = 1024 + (size_t)nb * ntok * 128 + (pair ? kPairTableBytes : 0) +
-             (size_t)kTcWStages * kTcExpand * 16 + 512;
+             (size_t)kTcWStages * 4 * kTcExpand * 16 + 512;
     P.tc = 1;
     return P;
 }
@@ -470,8 +569,7 @@ static cudaError_t launch_tc_t(const CUtensorMap &m, const LutLaunch &L, const L
                                int b_row_mod, cudaStream_t st) {
     cudaFuncSetAttribute(k_lut_tc<NTOK, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)P.smem);
-    dim3 grid(P.grid, P.streamk ? 1 : L.max_tiles);
-    k_lut_tc<NTOK, PAIR><<<grid, kTcThreads, P.smem, st>>>(m, L, P, b_row_mod);
+    k_lut_tc<NTOK, PAIR><<<P.grid, kTcThreads, P.smem, st>>>(m, L, P, b_row_mod);
     return cudaGetLastError();
 }
 
@@ -483,7 +581,7 @@ cudaError_t launch_lut_tc(const LutLaunch &L, const LutPlan &P, const void *b_f1
     std::memset(&m, 0, sizeof(m));
     if (!make_b_map(&m, b_f16, b_rows, L.K, ntok)) return cudaErrorInvalidValue;
     const bool timed = timing_on();
-    if (timed) timing_begin(st);
+    if (timed) timing_begin(st, CQ_KERNEL_LUT_TC);
     count_launch();
     cudaError_t e;
     switch (ntok) {

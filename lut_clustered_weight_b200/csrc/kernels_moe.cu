@@ -190,33 +190,53 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
     const int n = n0 + 4 * threadIdx.x;
     if (n >= a.H) return;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < a.topk; j++) {
-        const int p = s_p[j];
-        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp = 0; sp < a.plan_r.splits; sp++) {
-            const float4 v = *reinterpret_cast<const float4 *>(
-                a.part_r + ((int64_t)sp * a.R_routed + p) * a.H + n);
-            y.x += v.x; y.y += v.y; y.z += v.z; y.w += v.w;
+    const int64_t stride_r = a.R_routed * (int64_t)a.H / 4, stride_s = a.R_shared * (int64_t)a.H / 4;
+    // routed rows, four at a time (their split-K slot loads in flight together)
+    for (int j0 = 0; j0 < a.topk; j0 += 4) {
+        float4 y[4];
+        const float4 *pj[4];
+        int nsj[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            y[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int j = min(j0 + u, a.topk - 1);
+            pj[u] = reinterpret_cast<const float4 *>(a.part_r + (int64_t)s_p[j] * a.H + n);
+            nsj[u] = j0 + u < a.topk ? a.plan_r.splits : 0;
         }
-        const float sc = s_sh[j];
-        y.x *= sc; y.y *= sc; y.z *= sc; y.w *= sc;
-        if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + (int64_t)p * a.H + n) = y;
-        const float c = s_c[j];
-        acc.x += c * y.x; acc.y += c * y.y; acc.z += c * y.z; acc.w += c * y.w;
+        sum_slots<4>(pj, nsj, stride_r, y);
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const int j = j0 + u;
+            if (j >= a.topk) break;
+            const float sc = s_sh[j];
+            y[u].x *= sc; y[u].y *= sc; y[u].z *= sc; y[u].w *= sc;
+            if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + (int64_t)s_p[j] * a.H + n) = y[u];
+            const float c = s_c[j];
+            acc.x += c * y[u].x; acc.y += c * y[u].y; acc.z += c * y[u].z; acc.w += c * y[u].w;
+        }
     }
-    for (int s = 0; s < a.n_shared; s++) {
-        const int64_t lp = (int64_t)s * a.T + t;
-        const int ns = s_ns[s][n / rpt - rt0];
-        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp = 0; sp < ns; sp++) {
-            const float4 v = *reinterpret_cast<const float4 *>(
-                a.part_s + ((int64_t)sp * a.R_shared + lp) * a.H + n);
-            y.x += v.x; y.y += v.y; y.z += v.z; y.w += v.w;
+    // shared experts (at most four)
+    if (a.n_shared > 0) {
+        float4 y[4];
+        const float4 *ps[4];
+        int nss[4];
+#pragma unroll
+        for (int s = 0; s < 4; s++) {
+            y[s] = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int64_t lp = (int64_t)min(s, a.n_shared - 1) * a.T + t;
+            ps[s] = reinterpret_cast<const float4 *>(a.part_s + lp * a.H + n);
+            nss[s] = s < a.n_shared ? s_ns[s][n / rpt - rt0] : 0;
         }
-        const float sc = a.h_scales[a.R_routed + lp];
-        y.x *= sc; y.y *= sc; y.z *= sc; y.w *= sc;
-        if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + (a.R_routed + lp) * a.H + n) = y;
-        acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w;
+        sum_slots<4>(ps, nss, stride_s, y);
+#pragma unroll
+        for (int s = 0; s < 4; s++) {
+            if (s >= a.n_shared) break;
+            const int64_t lp = (int64_t)s * a.T + t;
+            const float sc = a.h_scales[a.R_routed + lp];
+            y[s].x *= sc; y[s].y *= sc; y[s].z *= sc; y[s].w *= sc;
+            if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + (a.R_routed + lp) * a.H + n) = y[s];
+            acc.x += y[s].x; acc.y += y[s].y; acc.z += y[s].z; acc.w += y[s].w;
+        }
     }
     *reinterpret_cast<float4 *>(a.out + (int64_t)t * a.H + n) = acc;
 }

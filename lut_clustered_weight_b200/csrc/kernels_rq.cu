@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kRqThreads) k_rq_swiglu(const SwigluArgs a) {
     const int I = routed ? a.I : a.I_shared;
     const int log2b = routed ? a.log2b_i : a.log2b_i_shared;
     const float *part = routed ? a.part_r : a.part_s;
-    const LutPlan &P = routed ? a.plan_r : a.plan_s;
+    const LutPlan P = routed ? a.plan_r : a.plan_s;
     const int64_t rows = routed ? a.R_routed : a.R_shared;
     const int64_t lp = routed ? p : p - a.R_routed;
     const int tok = routed ? a.perm[p] / a.topk : (int)(lp % a.T);
@@ -130,21 +130,17 @@ __global__ void __launch_bounds__(kRqThreads) k_rq_swiglu(const SwigluArgs a) {
     const float *rowp = part + lp * (2 * (int64_t)I);
     for (int i0 = 0; i0 < rp.n; i0 += 4 * kRqThreads) {
         float2 acc[4];
+        const float2 *pf[4];
+        int nsf[4];
 #pragma unroll
         for (int f = 0; f < 4; f++) {
             acc[f] = make_float2(0.f, 0.f);
             const int i = i0 + f * kRqThreads + threadIdx.x;
-            if (i < rp.n) {
-                const int n = rp.e0 + i;
-                const int splits = s_ns[n / P.rows_per_rt - rt0];
-                for (int sp = 0; sp < splits; sp++) {
-                    const float2 v =
-                        *reinterpret_cast<const float2 *>(rowp + sp * slot_stride + 2 * n);
-                    acc[f].x += v.x;
-                    acc[f].y += v.y;
-                }
-            }
+            const int n = rp.e0 + min(i, rp.n - 1);
+            pf[f] = reinterpret_cast<const float2 *>(rowp + 2 * n);
+            nsf[f] = i < rp.n ? s_ns[n / P.rows_per_rt - rt0] : 0;
         }
+        sum_slots<4>(pf, nsf, slot_stride / 2, acc);
 #pragma unroll
         for (int f = 0; f < 4; f++) {
             const int i = i0 + f * kRqThreads + threadIdx.x;
@@ -199,7 +195,7 @@ __global__ void __launch_bounds__(kWarpRows * 32) k_rq_swiglu_warp(const SwigluA
     const int I = routed ? a.I : a.I_shared;
     const int log2b = routed ? a.log2b_i : a.log2b_i_shared;
     const float *part = routed ? a.part_r : a.part_s;
-    const LutPlan &P = routed ? a.plan_r : a.plan_s;
+    const LutPlan P = routed ? a.plan_r : a.plan_s;
     const int64_t rows = routed ? a.R_routed : a.R_shared;
     const int64_t lp = routed ? p : p - a.R_routed;
     const int tok = routed ? a.perm[p] / a.topk : (int)(lp % a.T);
@@ -210,23 +206,23 @@ __global__ void __launch_bounds__(kWarpRows * 32) k_rq_swiglu_warp(const SwigluA
     __syncwarp();
     const int64_t slot_stride = rows * 2 * (int64_t)I;
     const float *rowp = part + lp * (2 * (int64_t)I);
-    for (int n0 = 0; n0 < I; n0 += 4 * 32) {
-        float2 acc[4];
+    // 16 columns per lane per round: the loads of a round are all in flight
+    // together, so a row of I columns costs I / 512 memory round trips
+    constexpr int F = 16;
+    for (int n0 = 0; n0 < I; n0 += F * 32) {
+        float2 acc[F];
+        const float2 *pf[F];
+        int nsf[F];
 #pragma unroll
-        for (int f = 0; f < 4; f++) {
+        for (int f = 0; f < F; f++) {
             acc[f] = make_float2(0.f, 0.f);
             const int n = n0 + f * 32 + lane;
-            if (n < I) {
-                const int ns = s_ns[w][n / P.rows_per_rt];
-                for (int sp = 0; sp < ns; sp++) {
-                    const float2 v = *reinterpret_cast<const float2 *>(rowp + sp * slot_stride + 2 * n);
-                    acc[f].x += v.x;
-                    acc[f].y += v.y;
-                }
-            }
+            pf[f] = reinterpret_cast<const float2 *>(rowp) + min(n, I - 1);
+            nsf[f] = n < I ? s_ns[w][n / P.rows_per_rt] : 0;
         }
+        sum_slots<F>(pf, nsf, slot_stride / 2, acc);
 #pragma unroll
-        for (int f = 0; f < 4; f++) {
+        for (int f = 0; f < F; f++) {
             const int n = n0 + f * 32 + lane;
             if (n < I) {
                 const __half h = __float2half_rn(silu_mul(acc[f].x * sx, acc[f].y * sx));

@@ -208,14 +208,19 @@ CQ_DEV double warp_fwht_absmax(double *buf, int K, int log2b) {
                 v[j] = upper ? (p - v[j]) : (v[j] + p);
             }
         }
-        for (int L = 5; L < log2b; L++) {
-            const int h = 1 << (L - 5);
+        // levels 5..7 pair registers of the same lane; unrolled so that the
+        // register indices are compile-time constants
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                if ((j & h) == 0) {
-                    const double a = v[j], c = v[j + h];
-                    v[j] = a + c;
-                    v[j + h] = a - c;
+        for (int L = 5; L < 8; L++) {
+            if (L < log2b) {
+                const int h = 1 << (L - 5);
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    if ((j & h) == 0) {
+                        const double a = v[j], c = v[j + h];
+                        v[j] = a + c;
+                        v[j + h] = a - c;
+                    }
                 }
             }
         }

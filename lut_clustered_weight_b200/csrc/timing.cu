@@ -17,6 +17,7 @@ static std::atomic<int> g_timing{0};
 static std::mutex g_mu;
 struct EventPair {
     cudaEvent_t a, b;
+    int kind;
 };
 static std::vector<EventPair> g_pending, g_free;
 
@@ -25,7 +26,7 @@ void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 bool timing_on() { return g_timing.load(std::memory_order_relaxed) != 0; }
 
 // Record the opening event of a timed launch (closed by timing_end).
-void timing_begin(cudaStream_t st) {
+void timing_begin(cudaStream_t st, int kind) {
     std::lock_guard<std::mutex> lk(g_mu);
     EventPair p;
     if (!g_free.empty()) {
@@ -38,6 +39,7 @@ void timing_begin(cudaStream_t st) {
             return;
         }
     }
+    p.kind = kind;
     cudaEventRecord(p.a, st);
     g_pending.push_back(p);
 }
@@ -58,6 +60,30 @@ CQ_API int32_t cq_device_error(void) { return cq::read_device_error(); }
 CQ_API cq_status cq_timing_enable(int32_t on) {
     cq::g_timing.store(on ? 1 : 0);
     return CQ_OK;
+}
+
+CQ_API cq_status cq_timing_read_launches(int32_t *kinds, float *ms, int64_t cap, int64_t *n) {
+    if (!n || cap < 0 || (cap > 0 && (!kinds || !ms))) return CQ_ERR_INVALID_ARGUMENT;
+    std::lock_guard<std::mutex> lk(cq::g_mu);
+    int64_t i = 0;
+    cq_status st = CQ_OK;
+    for (auto &p : cq::g_pending) {
+        float t = 0.0f;
+        if (cudaEventSynchronize(p.b) != cudaSuccess ||
+            cudaEventElapsedTime(&t, p.a, p.b) != cudaSuccess) {
+            st = CQ_ERR_CUDA;
+            t = -1.0f;
+        }
+        if (i < cap) {
+            kinds[i] = p.kind;
+            ms[i] = t;
+        }
+        i++;
+        cq::g_free.push_back(p);
+    }
+    cq::g_pending.clear();
+    *n = i;
+    return st;
 }
 
 CQ_API cq_status cq_timing_read(int64_t *launches, double *total_ms) {
