@@ -5,9 +5,9 @@
 Default workload: the Qwen3-4B-shaped dense SwiGLU FFN decode layer (hidden
 2560, intermediate 9728, gate/up 2560->9728, down 9728->2560) in all six
 published variants -- M in {1, 4, 16} tokens x {A4W4, A8W4}.  One step runs
-each variant once (42 tokens) on its own copy of the weights, so a step
-streams 6 x 38 MB of packed indices + codebooks (> the 126 MB L2) and no
-variant finds its weights in L2 from the previous step.
+each variant twice (84 tokens), every call on its own copy of the weights,
+so a step streams 12 x 38 MB of packed indices + codebooks (> 2 x the 126 MB
+L2) and no call finds its weights in L2 from the previous step.
 
 Reported (one JSON line from rank 0):
   value       tokens/s of the whole job (sum over ranks / max time), device
@@ -27,6 +27,7 @@ the timing is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -42,7 +43,7 @@ import numpy as np
 ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
-METRIC = "MoE-FFN tokens/s (LUT-GEMV effective GB/s and HBM roofline fraction in roofline)"
+METRIC = "LUT-GEMV effective GB/s & MoE-FFN tokens/s; fraction of HBM/tensor roofline"
 
 
 # ---------------------------------------------------------------------------
@@ -52,7 +53,10 @@ METRIC = "MoE-FFN tokens/s (LUT-GEMV effective GB/s and HBM roofline fraction in
 def workload_shapes(name):
     import synth
     if name == "qwen3_4b_ffn_decode":
-        return [synth.cfg1(M, b) for (M, b) in synth.CFG1_VARIANTS]
+        # every variant twice, each call on its own weight copy: a step streams
+        # 12 x 38 MB, more than twice the 126 MB L2
+        return [dataclasses.replace(synth.cfg1(M, b), name=f"{synth.cfg1(M, b).name}_w{c}")
+                for c in range(2) for (M, b) in synth.CFG1_VARIANTS]
     if name == "qwen3_30b_a3b_moe_decode":
         return [synth.CFG2]
     if name == "mixtral_8x7b_moe":

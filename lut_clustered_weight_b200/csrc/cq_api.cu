@@ -64,10 +64,12 @@ struct MoePlan {
     int64_t T, H, I, E, k, ns, Is, Rr, Rs, R;
     int bits, Imax, nt, tile_rows, max_tiles_r, tiles_s, tile_rows_s;
     bool tc_r, tc_s, tc_dn_r, tc_dn_s;  // tensor-core kernel per launch
+    bool fused;                         // gate/up launches write h (SwiGLU in their epilogue)
     LutPlan gu_r, gu_s, dn_r, dn_s;
-    size_t o_xq, o_sx, o_ids, o_w, o_counts, o_offsets, o_perm, o_inv, o_tiles;
+    size_t o_xq, o_sx, o_ids, o_w, o_counts, o_offsets, o_perm, o_inv, o_tiles, o_tgrp;
     size_t o_pgu_r, o_pgu_s, o_hq, o_sh, o_pdn_r, o_pdn_s;
     size_t o_bx_r, o_bx_s, o_bh_r, o_bh_s;  // fp16 B operands of tensor-core launches
+    size_t o_hf;                            // fused: h fp16 [R][Imax]
     size_t total;
 };
 
@@ -124,6 +126,10 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
                               (int)m.ns);
         }
     }
+    // SwiGLU moves into the gate/up epilogue when every gate/up launch runs on
+    // the tensor-core kernel with a single partial slot per output
+    m.fused = (m.E == 0 || (m.tc_r && !m.gu_r.streamk && m.gu_r.splits == 1)) &&
+              (m.ns == 0 || (m.tc_s && !m.gu_s.streamk && m.gu_s.splits == 1));
     size_t o = 0;
     auto take = [&](size_t bytes) {
         const size_t at = o;
@@ -139,8 +145,10 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
     m.o_perm = take((size_t)m.Rr * 4);
     m.o_inv = take((size_t)m.Rr * 4);
     m.o_tiles = take((size_t)(m.E + 1) * 4);
-    m.o_pgu_r = take(m.E > 0 ? (size_t)m.gu_r.splits * m.Rr * m.I * 2 * 4 : 0);
-    m.o_pgu_s = take(m.ns > 0 ? (size_t)m.gu_s.splits * m.Rs * m.Is * 2 * 4 : 0);
+    m.o_tgrp = take((size_t)m.max_tiles_r * 4);
+    m.o_pgu_r = take(m.E > 0 && !m.fused ? (size_t)m.gu_r.splits * m.Rr * m.I * 2 * 4 : 0);
+    m.o_pgu_s = take(m.ns > 0 && !m.fused ? (size_t)m.gu_s.splits * m.Rs * m.Is * 2 * 4 : 0);
+    m.o_hf = take(m.fused ? (size_t)m.R * m.Imax * 2 : 0);
     m.o_hq = take((size_t)m.R * code_bytes(m.Imax, m.bits));
     m.o_sh = take((size_t)m.R * 4);
     m.o_pdn_r = take(m.E > 0 ? (size_t)m.dn_r.splits * m.Rr * m.H * 4 : 0);
@@ -317,28 +325,35 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
     int32_t *perm = reinterpret_cast<int32_t *>(ws + m.o_perm);
     int32_t *inv = reinterpret_cast<int32_t *>(ws + m.o_inv);
     int32_t *tiles = reinterpret_cast<int32_t *>(ws + m.o_tiles);
+    int32_t *tgrp = reinterpret_cast<int32_t *>(ws + m.o_tgrp);
     float *pgu_r = reinterpret_cast<float *>(ws + m.o_pgu_r);
     float *pgu_s = reinterpret_cast<float *>(ws + m.o_pgu_s);
     uint8_t *hq = ws + m.o_hq;
     float *sh = reinterpret_cast<float *>(ws + m.o_sh);
     float *pdn_r = reinterpret_cast<float *>(ws + m.o_pdn_r);
     float *pdn_s = reinterpret_cast<float *>(ws + m.o_pdn_s);
+    __half *hf = reinterpret_cast<__half *>(ws + m.o_hf);
     const int64_t ldx = code_bytes(m.H, m.bits), ldh = code_bytes(m.Imax, m.bits);
 
     cudaError_t e = launch_rotate_quantize(x, m.H, T, (int)m.H, ilog2(d->had_block_h), m.bits, xq,
                                            ldx, sx, st);
     if (e == cudaSuccess && m.E > 0)
         e = launch_route(router_logits, (int)T, (int)m.E, (int)m.k, d->renormalize, m.tile_rows,
-                         ids, tw, counts, offsets, perm, inv, tiles, st);
+                         ids, tw, counts, offsets, perm, inv, tiles, tgrp, m.max_tiles_r, st);
     // gate / up (dual) -> partial g, u
     if (e == cudaSuccess && m.E > 0) {
         LutLaunch L{};
         L.codes = xq; L.ld_codes = ldx; L.act_bits = m.bits; L.K = (int)m.H;
         L.map_mode = kMapPerm; L.perm = perm; L.topk = (int)m.k; L.T = (int)T;
-        L.G = (int)m.E; L.grp_rows = offsets; L.grp_tiles = tiles; L.max_tiles = m.max_tiles_r;
+        L.G = (int)m.E; L.grp_rows = offsets; L.grp_tiles = tiles; L.tile_grp = tgrp; L.max_tiles = m.max_tiles_r;
         L.idx0 = w->gate_idx; L.cb0 = w->gate_cb; L.idx1 = w->up_idx; L.cb1 = w->up_cb;
         L.w_stride = m.I * (m.H / 2); L.cb_stride = m.I * 16; L.N = (int)m.I; L.dual = true;
         L.out = pgu_r; L.out_split_stride = m.Rr * m.I * 2; L.out_row_stride = m.I * 2;
+        if (m.fused) {
+            L.scales = sx;
+            L.h_out = hf;
+            L.h_row_stride = m.Imax;
+        }
         if (m.tc_r) {
             void *b = ws + m.o_bx_r;
             e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, m.Rr, kMapPerm, perm, (int)m.k,
@@ -356,6 +371,11 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.idx0 = w->sh_gate_idx; L.cb0 = w->sh_gate_cb; L.idx1 = w->sh_up_idx; L.cb1 = w->sh_up_cb;
         L.w_stride = m.Is * (m.H / 2); L.cb_stride = m.Is * 16; L.N = (int)m.Is; L.dual = true;
         L.out = pgu_s; L.out_split_stride = m.Rs * m.Is * 2; L.out_row_stride = m.Is * 2;
+        if (m.fused) {
+            L.scales = sx;
+            L.h_out = hf + m.Rr * m.Imax;
+            L.h_row_stride = m.Imax;
+        }
         if (m.tc_s) {
             void *b = ws + m.o_bx_s;
             e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, T, kMapIdentity, nullptr, 1,
@@ -366,7 +386,18 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         }
     }
     // SwiGLU + rotate + quantize of h
-    if (e == cudaSuccess) {
+    if (e == cudaSuccess && m.fused) {
+        // h was written by the gate/up epilogues: rotate + quantize its rows
+        if (m.E > 0)
+            e = launch_rotate_quantize(hf, m.Imax, m.Rr, (int)m.I, ilog2(d->had_block_i), m.bits,
+                                       hq, ldh, sh, st);
+        if (e == cudaSuccess && m.ns > 0)
+            e = launch_rotate_quantize(hf + m.Rr * m.Imax, m.Imax, m.Rs, (int)m.Is,
+                                       ilog2(d->had_block_i_shared), m.bits, hq + m.Rr * ldh, ldh,
+                                       sh + m.Rr, st);
+        if (e == cudaSuccess && dbg && dbg->h)
+            e = cudaMemcpyAsync(dbg->h, hf, (size_t)m.R * m.Imax * 2, cudaMemcpyDeviceToDevice, st);
+    } else if (e == cudaSuccess) {
         SwigluArgs a{};
         a.part_r = pgu_r; a.part_s = pgu_s;
         a.plan_r = m.gu_r; a.plan_s = m.gu_s;
@@ -384,7 +415,7 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         LutLaunch L{};
         L.codes = hq; L.ld_codes = ldh; L.act_bits = m.bits; L.K = (int)m.I;
         L.map_mode = kMapIdentity;
-        L.G = (int)m.E; L.grp_rows = offsets; L.grp_tiles = tiles; L.max_tiles = m.max_tiles_r;
+        L.G = (int)m.E; L.grp_rows = offsets; L.grp_tiles = tiles; L.tile_grp = tgrp; L.max_tiles = m.max_tiles_r;
         L.idx0 = w->down_idx; L.cb0 = w->down_cb;
         L.w_stride = m.H * (m.I / 2); L.cb_stride = m.H * 16; L.N = (int)m.H; L.dual = false;
         L.out = pdn_r; L.out_split_stride = m.Rr * m.H; L.out_row_stride = m.H;

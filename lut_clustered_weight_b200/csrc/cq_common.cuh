@@ -50,8 +50,9 @@ CQ_DEV void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// fp32 silu(g) * u
-CQ_DEV float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+// fp32 silu(g) * u with the fast exponential and division (a few ulp in
+// fp32, far below the fp16 rounding of h that follows)
+CQ_DEV float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 // ---------------------------------------------------------------- split-K slot sums
 CQ_DEV void vadd(float &a, float b) { a += b; }

@@ -1,6 +1,7 @@
 // cq_internal.h -- launchers shared between the .cu files of the library.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -36,6 +37,7 @@ struct LutLaunch {
     int uniform_rows;       // > 0: group g = rows [g*u, (g+1)*u); else device arrays
     const int32_t *grp_rows;   // [G+1]
     const int32_t *grp_tiles;  // [G+1] prefix of ceil(rows_g / (8 * plan.nt))
+    const int32_t *tile_grp;   // [max_tiles] group of each token tile (below grp_tiles[G])
     int max_tiles;             // grid.y (upper bound on the tile count)
     // weights: expert g of matrix j at idx[j] + g*w_stride, cb[j] + g*cb_stride
     const uint8_t *idx0;
@@ -51,6 +53,11 @@ struct LutLaunch {
     int64_t out_split_stride;  // floats
     int64_t out_row_stride;    // floats
     bool direct;            // plain, splits == 1: out[r*N+n] = scale * acc
+    // dual tensor-core launches with one partial slot only: instead of the
+    // partials, h[p, n] = fp16(silu(s * g) * (s * u)) with s = scales[code
+    // row of p], written at h_out + p * h_row_stride + n
+    __half *h_out;
+    int64_t h_row_stride;   // elements
 };
 
 // How one LUT GEMM launch is cut into work.  A work item is (token tile,

@@ -43,7 +43,8 @@ struct CombineArgs {
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int tile_rows,
                          int32_t *ids, float *w, int32_t *counts, int32_t *offsets, int32_t *perm,
-                         int32_t *inv_perm, int32_t *grp_tiles, cudaStream_t st);
+                         int32_t *inv_perm, int32_t *grp_tiles, int32_t *tile_grp,
+                         int max_tiles, cudaStream_t st);
 cudaError_t launch_swiglu_rq(const SwigluArgs &a, int64_t rows, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 

@@ -141,12 +141,7 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
                 nrows = min(TT, (g + 1) * L.uniform_rows - row0);
             } else {
                 if (tile >= L.grp_tiles[L.G]) return;  // beyond the routed tiles (fixed mode)
-                int lo = 0, hi = L.G;  // largest g with grp_tiles[g] <= tile
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (L.grp_tiles[mid] <= tile) lo = mid; else hi = mid;
-                }
-                g = lo;
+                g = L.tile_grp[tile];
                 row0 = L.grp_rows[g] + (int)(tile - L.grp_tiles[g]) * TT;
                 nrows = min(TT, L.grp_rows[g + 1] - row0);
             }

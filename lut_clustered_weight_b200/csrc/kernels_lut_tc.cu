@@ -53,9 +53,12 @@ constexpr int kTcRows = 128;         // rows per tile (TMEM lanes)
 constexpr int kTcChunk = 64;         // k per chunk: one B tile, 4 MMAs, 32 TMEM columns
 constexpr int kTcG = 4;              // chunks per group: the expand / A-ring unit (256 k)
 constexpr int kTcA = 2;              // A ring depth in groups (TMEM columns [0, 256))
-// B ring depth in chunks (shared memory, NTOK x 128 B per chunk); a B slot is
-// freed by the commit of the chunk that used it.
-template <int NTOK> struct TcB { static constexpr int n = NTOK <= 128 ? 8 : 4; };
+// B ring (shared memory, NTOK x 128 B per chunk tile): kTcB stages of kBG
+// chunk tiles; a stage is freed by the commit of the MMAs that read it.
+// Small token tiles take a whole group per stage (one wait and one commit
+// per group instead of per chunk).
+template <int NTOK> struct TcB { static constexpr int n = NTOK <= 64 ? 4 : NTOK <= 128 ? 8 : 4; };
+template <int NTOK> struct TcBG { static constexpr int n = NTOK <= 64 ? kTcG : 1; };
 // Independent accumulators: a chain of small MMAs into one accumulator is
 // bound by the MMA latency, so tiles of few tokens spread the four K steps
 // of a chunk over four accumulators (summed in the epilogue).
@@ -82,12 +85,7 @@ struct TcSchedule {
                 row0 = nrows = 0;
                 return;
             }
-            int lo = 0, hi = L->G;
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (L->grp_tiles[mid] <= tile) lo = mid; else hi = mid;
-            }
-            g = lo;
+            g = L->tile_grp[tile];
             row0 = L->grp_rows[g] + (int)(tile - L->grp_tiles[g]) * TT;
             nrows = min(TT, L->grp_rows[g + 1] - row0);
         }
@@ -174,8 +172,18 @@ struct TcWalk {
 // token tiles there are; the host only knows an upper bound).
 CQ_DEV int64_t tc_pieces(const LutLaunch &L, const LutPlan &P) {
     if (P.streamk) return 0;
-    const int64_t tiles = min((int64_t)L.grp_tiles[L.G], (int64_t)L.max_tiles);
+    const int TT = 8 * P.nt;
+    const int64_t tiles = L.uniform_rows > 0
+                              ? (int64_t)L.G * ((L.uniform_rows + TT - 1) / TT)
+                              : min((int64_t)L.grp_tiles[L.G], (int64_t)L.max_tiles);
     return tiles * P.n_row_tiles * P.splits;
+}
+
+// Activation scale of output row p (the row's token).
+CQ_DEV float tc_row_scale(const LutLaunch &L, int64_t p) {
+    const int64_t cr = L.map_mode == kMapPerm ? L.perm[p] / L.topk
+                     : L.map_mode == kMapModT ? p % L.T : p;
+    return L.scales[cr];
 }
 
 template <int NTOK, bool PAIR>
@@ -187,9 +195,10 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     uint8_t *sm = smem_raw + pad;
     constexpr uint32_t kBSlot = NTOK * 128;  // bytes of one B chunk tile
     constexpr int kTcB = TcB<NTOK>::n;
+    constexpr int kBG = TcBG<NTOK>::n;
     constexpr int kAcc = TcAcc<NTOK>::n;
-    uint8_t *bslots = sm;                                     // [kTcB][NTOK][128 B]
-    uint8_t *tables = sm + kTcB * kBSlot;                     // PAIR: [256][128 rows] x 4 B
+    uint8_t *bslots = sm;                                     // [kTcB][kBG][NTOK][128 B]
+    uint8_t *tables = sm + kTcB * kBG * kBSlot;               // PAIR: [256][128 rows] x 4 B
     uint8_t *wring_raw = tables + (PAIR ? kPairTableBytes : 0);  // [stage][4][256 thr] x 16 B
     uint64_t *bars = reinterpret_cast<uint64_t *>(wring_raw + kTcWStages * 4 * kTcExpand * 16);
     uint64_t *a_full = bars, *a_empty = bars + kTcA;
@@ -251,7 +260,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
             int64_t b_item = -1;
             int b_y = 0;
             bool ok = true;
-            for (int jc = 0; bw.valid && ok; bw.next()) {
+            for (int jc = 0, gi = 0; bw.valid && ok; bw.next(), gi++) {
                 if (bw.w != b_item) {
                     int g, row0, nrows, rt;
                     S.item(bw.w, g, row0, nrows, rt);
@@ -259,13 +268,19 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                     b_y = b_row_mod > 0 ? row0 % b_row_mod : row0;
                 }
                 for (int i = 0; i < bw.gn; i++, jc++) {
-                    const int s = jc % kTcB;
-                    if (jc >= kTcB && !mbar_wait(&b_empty[s], (uint32_t)(jc / kTcB - 1) & 1u)) {
-                        ok = false;
-                        break;
+                    // stage js: one chunk (kBG = 1) or the whole group (kBG = kTcG)
+                    const int js = kBG == 1 ? jc : gi;
+                    const int s = js % kTcB;
+                    if (kBG == 1 || i == 0) {
+                        if (js >= kTcB &&
+                            !mbar_wait(&b_empty[s], (uint32_t)(js / kTcB - 1) & 1u)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&b_full[s], kBSlot * (kBG == 1 ? 1 : bw.gn));
                     }
-                    mbar_arrive_expect_tx(&b_full[s], kBSlot);
-                    tma_load_2d(bslots + s * kBSlot, &tmB, (bw.c0 + i) * kTcChunk, b_y, &b_full[s]);
+                    tma_load_2d(bslots + (s * kBG + (kBG == 1 ? 0 : i)) * kBSlot, &tmB,
+                                (bw.c0 + i) * kTcChunk, b_y, &b_full[s]);
                 }
             }
         }
@@ -285,14 +300,17 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 if (!ok) break;
                 tc_fence_after();
                 for (int i = 0; i < mw.gn; i++, jc++) {
-                    const int sb = jc % kTcB;
-                    if (!mbar_wait(&b_full[sb], (uint32_t)(jc / kTcB) & 1u)) {
-                        ok = false;
-                        break;
+                    const int js = kBG == 1 ? jc : gi;
+                    const int sb = js % kTcB;
+                    if (kBG == 1 || i == 0) {
+                        if (!mbar_wait(&b_full[sb], (uint32_t)(js / kTcB) & 1u)) {
+                            ok = false;
+                            break;
+                        }
+                        consumed++;
                     }
-                    consumed++;
-                    tc_fence_after();
-                    const uint64_t bd = smem_desc_sw128(smem_u32(bslots + sb * kBSlot));
+                    const uint64_t bd = smem_desc_sw128(
+                        smem_u32(bslots + (sb * kBG + (kBG == 1 ? 0 : i)) * kBSlot));
                     const bool fresh = first && i == 0;
 #pragma unroll
                     for (int kk = 0; kk < kTcChunk / 16; kk++) {
@@ -301,7 +319,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                                   bd + (uint64_t)(2 * kk), idesc,
                                   (fresh && kk < kAcc) ? 0u : 1u);
                     }
-                    tc_commit(&b_empty[sb]);
+                    if (kBG == 1 || i == mw.gn - 1) tc_commit(&b_empty[sb]);
                 }
                 if (!ok) break;
                 tc_commit(&a_empty[gs]);
@@ -312,7 +330,8 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
             }
             // nothing may still be writing shared or tensor memory when the CTA
             // leaves: the B loads of chunks not consumed, and all MMAs
-            for (int j = consumed; j < nchunks && j < consumed + kTcB; j++)
+            const int nstages = kBG == 1 ? nchunks : ngroups;
+            for (int j = consumed; j < nstages && j < consumed + kTcB; j++)
                 mbar_wait(&b_full[j % kTcB], (uint32_t)(j / kTcB) & 1u);
             tc_commit(fin);
             mbar_wait(fin, 0);
@@ -359,6 +378,13 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
         for (int i = 0; i < kTcWStages - 1; i++) issue_group();
 
         int g = 0, row0 = 0, nrows = 0, rt = 0, col = 0, items = 0;
+        // epilogue: this warp's slice of the NTOK token columns
+        constexpr int kEpi = NTOK >= 32 ? NTOK / 2 : 16;
+        constexpr int kScl = (kEpi + 31) / 32;
+        const int cbeg = h * kEpi;
+        float scl[kScl];  // fused SwiGLU: token scales of the slice, lane l holds c = cbeg + l + 32 i
+#pragma unroll
+        for (int i = 0; i < kScl; i++) scl[i] = 0.0f;
         bool ok = true;
         TcWalk cw;
         cw.init(P, n_pieces);
@@ -369,6 +395,13 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 const __half *cbp;
                 S.item(cw.w, g, row0, nrows, rt);
                 S.row_ptrs(max(g, 0), rt, t, idxp, cbp, col);
+                if (L.h_out) {  // loads in flight during the segment; used by its epilogue
+#pragma unroll
+                    for (int i = 0; i < kScl; i++) {
+                        const int c = cbeg + lane + 32 * i;
+                        scl[i] = (c < nrows && c < cbeg + kEpi) ? tc_row_scale(L, row0 + c) : 0.0f;
+                    }
+                }
                 // the one-time LUT precompute for this row
                 const uint4 c0v = *reinterpret_cast<const uint4 *>(cbp);
                 const uint4 c1v = *reinterpret_cast<const uint4 *>(cbp + 8);
@@ -413,10 +446,12 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 // 128 weights -> 64 fp16 pairs (k = 2b, 2b + 1 in column b)
                 uint32_t v[64];
                 if (PAIR) {
+                    // 64 independent shared loads (32-bit shared addresses)
+                    const uint32_t tab_s = smem_u32(tab);
 #pragma unroll
                     for (int b = 0; b < 64; b++) {
                         const uint32_t byte = prmt(wd[b >> 2], 0u, 0x4440u | (uint32_t)(b & 3));
-                        v[b] = tab[byte * kTcRows];
+                        v[b] = lds32(tab_s + byte * (kTcRows * 4));
                     }
                 } else {
 #pragma unroll
@@ -454,24 +489,58 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 if (!ok) break;
                 tc_fence_after();
                 float *out = L.out + (int64_t)cw.slot * L.out_split_stride;
-                constexpr int kEpi = NTOK >= 32 ? NTOK / 2 : 16;
-                const int cbeg = h * kEpi;
                 if (cbeg < NTOK) {
+                    // kLd 16-column loads in flight per wait; an iteration covers
+                    // at most 32 columns, whose token scales sit in scl[0]
+                    constexpr int kLd = kAcc == 1 ? (kEpi >= 32 ? 2 : 1) : 1;
+                    static_assert(16 * kLd <= 32, "one scale register per iteration");
 #pragma unroll 1
-                    for (int c0 = cbeg; c0 < cbeg + kEpi; c0 += 16) {
-                        uint32_t d[kAcc][16];
+                    for (int it = 0; it < kEpi / (16 * kLd); it++) {
+                        const int c0 = cbeg + it * 16 * kLd;
+                        const float cur = scl[0];
+#pragma unroll
+                        for (int i = 0; i + 1 < kScl; i++) scl[i] = scl[i + 1];
+                        uint32_t d[kAcc * kLd][16];
 #pragma unroll
                         for (int a = 0; a < kAcc; a++)
-                            tmem_ld16(tmem_d + lane_base + a * NTOK + c0, d[a]);
+#pragma unroll
+                            for (int bb = 0; bb < kLd; bb++)
+                                tmem_ld16(tmem_d + lane_base + a * NTOK + c0 + 16 * bb, d[a * kLd + bb]);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int qq = 0; qq < 16; qq++) {
-                            float acc = __uint_as_float(d[0][qq]);
+                        for (int bb = 0; bb < kLd; bb++)
 #pragma unroll
-                            for (int a = 1; a < kAcc; a++) acc += __uint_as_float(d[a][qq]);
-                            if (c0 + qq < nrows)
-                                out[(int64_t)(row0 + c0 + qq) * L.out_row_stride + col] = acc;
-                        }
+                            for (int qq = 0; qq < 16; qq += 2) {
+                                float a0 = __uint_as_float(d[bb][qq]);
+                                float a1 = __uint_as_float(d[bb][qq + 1]);
+#pragma unroll
+                                for (int a = 1; a < kAcc; a++) {
+                                    a0 += __uint_as_float(d[a * kLd + bb][qq]);
+                                    a1 += __uint_as_float(d[a * kLd + bb][qq + 1]);
+                                }
+                                const int c = c0 + 16 * bb + qq;
+                                if (L.h_out) {
+                                    // SwiGLU.  Lanes 2j (gate) and 2j + 1 (up) hold the same
+                                    // output column; the even lane finishes token c and the
+                                    // odd lane token c + 1, after one exchange
+                                    const int odd = lane & 1;
+                                    const float recv =
+                                        __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
+                                    const float gv = odd ? recv : a0, uv = odd ? a1 : recv;
+                                    const float sx =
+                                        __shfl_sync(0xffffffffu, cur, 16 * bb + qq + odd);
+                                    if (c + odd < nrows) {
+                                        const int64_t p = row0 + c + odd;
+                                        L.h_out[p * L.h_row_stride + (col >> 1)] =
+                                            __float2half_rn(silu_mul(gv * sx, uv * sx));
+                                    }
+                                } else {
+                                    if (c < nrows)
+                                        out[(int64_t)(row0 + c) * L.out_row_stride + col] = a0;
+                                    if (c + 1 < nrows)
+                                        out[(int64_t)(row0 + c + 1) * L.out_row_stride + col] = a1;
+                                }
+                            }
                     }
                 }
                 tc_fence_before();
@@ -535,8 +604,11 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
     P.cps_max = P.chunks_total;
     const int capacity = sm_count();  // one CTA per SM
     const int C = P.chunks_total;
-    if (uniform_rows > 0) {
-        const int64_t tiles = (int64_t)n_groups * ((uniform_rows + ntok - 1) / ntok);
+    const int64_t u_tiles =
+        uniform_rows > 0 ? (int64_t)n_groups * ((uniform_rows + ntok - 1) / ntok) : 0;
+    if (uniform_rows > 0 && u_tiles * P.n_row_tiles < 3LL * capacity) {
+        // few work items: stream-K balances them over the SMs
+        const int64_t tiles = u_tiles;
         P.streamk = 1;
         P.uniform_rows = uniform_rows;
         P.units = tiles * P.n_row_tiles * C;
@@ -547,7 +619,10 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
         P.splits = smax;
         P.chunks_per_split = C;
     } else {
+        // many work items (or routed groups): whole items per CTA, split-K only
+        // when there are fewer items than SMs
         P.streamk = 0;
+        P.uniform_rows = uniform_rows;
         const int64_t base = (int64_t)P.n_row_tiles * std::max<int64_t>(est_tiles, 1);
         int splits = base < capacity ? (int)(capacity / base) : 1;
         splits = std::max(1, std::min(splits, C));
@@ -557,7 +632,7 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
         P.grid = (int)std::min<int64_t>(capacity, base * P.splits);
     }
     const bool pair = ntok <= 16;
-    const int nb = ntok <= 128 ? 8 : 4;
+    const int nb = ntok <= 64 ? 4 * kTcG : ntok <= 128 ? 8 : 4;  // chunk tiles in the B ring
     P.smem = 1024 + (size_t)nb * ntok * 128 + (pair ? kPairTableBytes : 0) +
              (size_t)kTcWStages * 4 * kTcExpand * 16 + 512;
     P.tc = 1;

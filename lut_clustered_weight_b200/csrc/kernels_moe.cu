@@ -81,7 +81,8 @@ constexpr int kGroupWarps = kGroupThreads / 32;
 __global__ void __launch_bounds__(kGroupThreads)
 k_group(const int32_t *__restrict__ ids, int T, int E, int k, int tile_rows,
         int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
-        int32_t *__restrict__ inv_perm, int32_t *__restrict__ grp_tiles) {
+        int32_t *__restrict__ inv_perm, int32_t *__restrict__ grp_tiles,
+        int32_t *__restrict__ tile_grp, int max_tiles) {
     __shared__ int32_t hist[kGroupWarps][kMaxExperts];
     __shared__ int32_t s_off[kMaxExperts + 1];
     __shared__ int32_t s_tiles[kMaxExperts + 1];
@@ -131,6 +132,9 @@ k_group(const int32_t *__restrict__ ids, int T, int E, int k, int tile_rows,
         offsets[tid] = s_off[tid];
         grp_tiles[tid] = s_tiles[tid];
     }
+    // tile -> group, so the LUT kernels find a tile's expert with one load
+    if (tid < E)
+        for (int tl = s_tiles[tid]; tl < s_tiles[tid + 1] && tl < max_tiles; tl++) tile_grp[tl] = tid;
     __syncthreads();
     for (int sb = c0; sb < c1; sb += 32) {
         const int sl = sb + lane;
@@ -153,12 +157,13 @@ k_group(const int32_t *__restrict__ ids, int T, int E, int k, int tile_rows,
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int tile_rows,
                          int32_t *ids, float *w, int32_t *counts, int32_t *offsets, int32_t *perm,
-                         int32_t *inv_perm, int32_t *grp_tiles, cudaStream_t st) {
+                         int32_t *inv_perm, int32_t *grp_tiles, int32_t *tile_grp,
+                         int max_tiles, cudaStream_t st) {
     count_launch(2);
     k_topk<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, st>>>(logits, T, E, k,
                                                                           renorm, ids, w);
     k_group<<<1, kGroupThreads, 0, st>>>(ids, T, E, k, tile_rows, counts, offsets, perm, inv_perm,
-                                         grp_tiles);
+                                         grp_tiles, tile_grp, max_tiles);
     return cudaGetLastError();
 }
 

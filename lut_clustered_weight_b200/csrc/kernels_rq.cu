@@ -206,9 +206,9 @@ __global__ void __launch_bounds__(kWarpRows * 32) k_rq_swiglu_warp(const SwigluA
     __syncwarp();
     const int64_t slot_stride = rows * 2 * (int64_t)I;
     const float *rowp = part + lp * (2 * (int64_t)I);
-    // 16 columns per lane per round: the loads of a round are all in flight
-    // together, so a row of I columns costs I / 512 memory round trips
-    constexpr int F = 16;
+    // 8 columns per lane per round: the loads of a round are all in flight
+    // together, so a row of I columns costs I / 256 memory round trips
+    constexpr int F = 8;
     for (int n0 = 0; n0 < I; n0 += F * 32) {
         float2 acc[F];
         const float2 *pf[F];

@@ -188,34 +188,38 @@ __device__ void block_quantize_range(const double *buf, int n, int e0, int bits,
 // ---------------------------------------------------------------- one warp per row
 // Rotation blocks of b <= 256: the whole transform of a 256-aligned chunk is
 // inside one warp (index bits 0-4 across lanes, 5-7 in registers).  buf holds
-// the row (K doubles, K % 256 == 0 or a ragged last chunk); returns max |.|.
+// the row (K doubles; K a multiple of b, so a ragged last chunk holds whole
+// blocks); returns max |.|.
 CQ_DEV double warp_fwht_absmax(double *buf, int K, int log2b) {
     const int lane = threadIdx.x & 31;
     double amax = 0.0;
-    for (int base = 0; base < K; base += 256) {
-        double v[8];
+    // two 256-element chunks per pass: 16 independent butterfly chains
+    for (int base = 0; base < K; base += 512) {
+        double v[16];
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
+        for (int j = 0; j < 16; j++) {
             const int k = base + lane + 32 * j;
             v[j] = k < K ? buf[k] : 0.0;
         }
         for (int L = 0; L < (log2b < 5 ? log2b : 5); L++) {
             const int bit = 1 << L;
-            const bool upper = lane & bit;
+            // partner p: lower lane keeps v + p, upper lane p - v (one
+            // correctly rounded fma with an exact +-1 product)
+            const double sg = (lane & bit) ? -1.0 : 1.0;
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
+            for (int j = 0; j < 16; j++) {
                 const double p = __shfl_xor_sync(0xffffffffu, v[j], bit);
-                v[j] = upper ? (p - v[j]) : (v[j] + p);
+                v[j] = fma(sg, v[j], p);
             }
         }
-        // levels 5..7 pair registers of the same lane; unrolled so that the
-        // register indices are compile-time constants
+        // levels 5..7 pair registers of the same lane (within each 256-chunk);
+        // unrolled so that the register indices are compile-time constants
 #pragma unroll
         for (int L = 5; L < 8; L++) {
             if (L < log2b) {
                 const int h = 1 << (L - 5);
 #pragma unroll
-                for (int j = 0; j < 8; j++) {
+                for (int j = 0; j < 16; j++) {
                     if ((j & h) == 0) {
                         const double a = v[j], c = v[j + h];
                         v[j] = a + c;
@@ -225,7 +229,7 @@ CQ_DEV double warp_fwht_absmax(double *buf, int K, int log2b) {
             }
         }
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
+        for (int j = 0; j < 16; j++) {
             const int k = base + lane + 32 * j;
             if (k < K) {
                 buf[k] = v[j];

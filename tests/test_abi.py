@@ -112,3 +112,14 @@ def test_workspace_sizes_grow_with_tokens():
     c = cq.MoEConfig(2048, 768, 128, 8, 0, 0, 4, 2048, 256, 256)
     assert cq.cq_moe_ffn_workspace_size(c, 64) < cq.cq_moe_ffn_workspace_size(c, 4096)
     assert cq.cq_moe_ffn_workspace_size(c, 64) == cq.cq_moe_ffn_workspace_size(c, 64)
+
+
+def test_timing_record_argument_checks():
+    f = cq.lib.cq_timing_read_launches
+    n = ctypes.c_int64(-1)
+    # empty record: nothing recorded, no CUDA call made
+    assert f(None, None, 0, ctypes.byref(n)) == cq.CQ_OK and n.value == 0
+    assert f(None, None, 0, None) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert f(None, None, -1, ctypes.byref(n)) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert f(None, None, 4, ctypes.byref(n)) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert cq.cq_timing_read_launches() == []

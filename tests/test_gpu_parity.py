@@ -182,6 +182,11 @@ SMALL_MOE = [
                    act_bits=4, had_block_h=128, had_block_i=64),
     synth.MoEShape("moe_many_rows", H=192, I=128, E=4, top_k=2, n_shared=1, T=320, act_bits=8,
                    had_block_h=64, had_block_i=128, I_shared=256),
+    # gate/up with one partial slot: SwiGLU in the tensor-core epilogue (fp16 h)
+    synth.MoEShape("moe_fused_t64", H=384, I=768, E=16, top_k=2, n_shared=0, T=200, act_bits=4,
+                   had_block_h=128, had_block_i=256),
+    synth.MoEShape("moe_fused_i1024", H=256, I=1024, E=8, top_k=2, n_shared=0, T=320,
+                   act_bits=8, had_block_h=256, had_block_i=256, bias_expert=3, bias=0.5),
 ]
 
 
