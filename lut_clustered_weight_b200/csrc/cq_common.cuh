@@ -1,6 +1,8 @@
 // cq_common.cuh -- shared device helpers for the sm_100a CodeQuant kernels.
 #pragma once
 
+#include <utility>
+
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -54,6 +56,17 @@ CQ_DEV void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32
 // fp32, far below the fp16 rounding of h that follows)
 CQ_DEV float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream
+// serialization: it may start while the previous kernel on the stream is
+// still running.  griddep_wait() blocks until that kernel has completed and
+// its writes are visible; nothing that kernel produces may be read, and no
+// global memory may be written, before it.  griddep_launch() lets the next
+// kernel start early (it waits for this one in turn).  Both are no-ops for a
+// kernel launched without the attribute.
+CQ_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+CQ_DEV void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- split-K slot sums
 CQ_DEV void vadd(float &a, float b) { a += b; }
 CQ_DEV void vadd(float2 &a, float2 b) {
@@ -68,27 +81,53 @@ CQ_DEV void vadd(float4 &a, float4 b) {
 }
 
 // acc[f] += p[f][0] + p[f][stride] + ... (ns[f] slots, added in slot order),
-// for F independent sums at once: every round issues the loads of two slots
-// of all F sums before the first add, so 2F loads are in flight instead of a
+// for F independent sums at once: every round issues the loads of U slots of
+// all F sums before the first add, so F * U loads are in flight instead of a
 // chain of dependent round trips.
-template <int F, typename T>
+template <int F, int U = 2, typename T>
 CQ_DEV void sum_slots(const T *const (&p)[F], const int (&ns)[F], int64_t stride, T (&acc)[F]) {
     int nsmax = 0;
 #pragma unroll
     for (int f = 0; f < F; f++) nsmax = max(nsmax, ns[f]);
-    for (int s0 = 0; s0 < nsmax; s0 += 2) {
-        T v[F][2];
+    for (int s0 = 0; s0 < nsmax; s0 += U) {
+        T v[F][U];
 #pragma unroll
         for (int f = 0; f < F; f++)
 #pragma unroll
-            for (int u = 0; u < 2; u++)
+            for (int u = 0; u < U; u++)
                 v[f][u] = s0 + u < ns[f] ? p[f][(int64_t)(s0 + u) * stride] : T{};
 #pragma unroll
         for (int f = 0; f < F; f++)
 #pragma unroll
-            for (int u = 0; u < 2; u++)
+            for (int u = 0; u < U; u++)
                 if (s0 + u < ns[f]) vadd(acc[f], v[f][u]);
     }
+}
+
+// Launch with programmatic stream serialization (and a cluster if cluster_x > 1).
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                     cudaStream_t st, int cluster_x, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    na++;
+    if (cluster_x > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)cluster_x;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        na++;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace cq

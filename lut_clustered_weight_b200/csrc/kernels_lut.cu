@@ -64,6 +64,10 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gq = lane >> 2, cl = lane & 3;
     const int K = L.K;
+    griddep_launch();
+    // routed launches: the group tables come from the previous kernels; uniform
+    // launches prefetch weights and build tables first (see below)
+    if (L.uniform_rows == 0) griddep_wait();
     const int C = P.chunks_total;
     const int64_t rowbytes = K / 2;
     const int tailc = (K & 127) >> 5;  // valid 32-k slices of a ragged last chunk
@@ -175,6 +179,7 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
 #pragma unroll
                 for (int e = 0; e < 4; e++) acc[t][e] = 0.0f;
             __syncthreads();  // previous piece is done with s_code_row / bfrag
+            griddep_wait();   // activations and scales come from the previous kernel
             if (tid < TT) {
                 int cr = -1;
                 if (tid < nrows) {
@@ -345,8 +350,7 @@ static cudaError_t launch_lut_t(const LutLaunch &L, const LutPlan &P, cudaStream
     cudaFuncSetAttribute(k_lut_mma<NT, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)P.smem);
     dim3 grid(P.grid, P.streamk ? 1 : L.max_tiles);
-    k_lut_mma<NT, W><<<grid, W * 32, P.smem, st>>>(L, P);
-    return cudaSuccess;
+    return launch_pdl(k_lut_mma<NT, W>, grid, dim3(W * 32), P.smem, st, 1, L, P);
 }
 
 cudaError_t launch_lut(const LutLaunch &L, const LutPlan &P, cudaStream_t st) {
@@ -368,6 +372,8 @@ __global__ void __launch_bounds__(256) k_reduce_plain(const float *__restrict__ 
                                                       int64_t M, int64_t N, const float *__restrict__ s,
                                                       float *__restrict__ y) {
     __shared__ int s_ns[8];
+    griddep_wait();
+    griddep_launch();
     const int64_t m = blockIdx.y;
     const int n0 = blockIdx.x * 256;
     const int rt0 = n0 / P.rows_per_rt;
@@ -380,7 +386,7 @@ __global__ void __launch_bounds__(256) k_reduce_plain(const float *__restrict__ 
     const float *pp[1] = {part + i};
     const int ns[1] = {s_ns[n / P.rows_per_rt - rt0]};
     float acc[1] = {0.0f};
-    sum_slots<1>(pp, ns, M * N, acc);
+    sum_slots<1, 8>(pp, ns, M * N, acc);
     y[i] = s[m] * acc[0];
 }
 
@@ -390,14 +396,15 @@ cudaError_t launch_reduce_plain(const float *part, const LutPlan &P, int64_t M, 
     if (n == 0) return cudaSuccess;
     count_launch();
     dim3 grid((unsigned)((N + 255) / 256), (unsigned)M);
-    k_reduce_plain<<<grid, 256, 0, st>>>(part, P, M, N, s, y);
-    return cudaGetLastError();
+    return launch_pdl(k_reduce_plain, grid, dim3(256), 0, st, 1, part, P, M, N, s, y);
 }
 
 // ---------------------------------------------------------------- centroid sums (parity)
 // S[m, n, c] = sum_{k : I[n,k] = c} q[m,k]; one thread per (m, n).
 __global__ void k_centroid_sums(const uint8_t *__restrict__ q, int64_t M, int64_t K, int bits,
                                 const uint8_t *__restrict__ w_idx, int64_t N, int32_t *S) {
+    griddep_wait();
+    griddep_launch();
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= M * N) return;
     const int64_t m = i / N, n = i % N;
@@ -426,9 +433,8 @@ cudaError_t launch_centroid_sums(const void *q, int64_t M, int64_t K, int bits,
     const int64_t n = M * N;
     if (n == 0) return cudaSuccess;
     count_launch();
-    k_centroid_sums<<<(unsigned)((n + 127) / 128), 128, 0, st>>>(
-        reinterpret_cast<const uint8_t *>(q), M, K, bits, w_idx, N, S);
-    return cudaGetLastError();
+    return launch_pdl(k_centroid_sums, dim3((unsigned)((n + 127) / 128)), dim3(128), 0, st, 1,
+                      reinterpret_cast<const uint8_t *>(q), M, K, bits, w_idx, N, S);
 }
 
 }  // namespace cq

@@ -234,6 +234,9 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // everything below may read what the previous kernels wrote
+    griddep_wait();
+    griddep_launch();
     const uint32_t tmem = *s_tmem;
     const uint32_t tmem_a = tmem;                 // columns [0, 256): A ring (2 x 128)
     const uint32_t tmem_d = tmem + kTcA * 128;    // columns [256, 256 + kAcc NTOK)
@@ -644,8 +647,8 @@ static cudaError_t launch_tc_t(const CUtensorMap &m, const LutLaunch &L, const L
                                int b_row_mod, cudaStream_t st) {
     cudaFuncSetAttribute(k_lut_tc<NTOK, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)P.smem);
-    k_lut_tc<NTOK, PAIR><<<P.grid, kTcThreads, P.smem, st>>>(m, L, P, b_row_mod);
-    return cudaGetLastError();
+    return launch_pdl(k_lut_tc<NTOK, PAIR>, dim3(P.grid), dim3(kTcThreads), P.smem, st, 1, m, L, P,
+                      b_row_mod);
 }
 
 cudaError_t launch_lut_tc(const LutLaunch &L, const LutPlan &P, const void *b_f16,
@@ -675,6 +678,8 @@ cudaError_t launch_lut_tc(const LutLaunch &L, const LutPlan &P, const void *b_f1
 __global__ void k_codes_to_f16(const uint8_t *__restrict__ codes, int64_t ld_codes, int bits,
                                int K, int64_t rows, int map_mode, const int32_t *__restrict__ perm,
                                int topk, int T, __half *__restrict__ out) {
+    griddep_wait();
+    griddep_launch();
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int per_row = K / 8;
     if (i >= rows * per_row) return;
@@ -704,10 +709,9 @@ cudaError_t launch_codes_to_f16(const void *codes, int64_t ld_codes, int bits, i
     const int64_t n = rows * (K / 8);
     if (n == 0) return cudaSuccess;
     count_launch();
-    k_codes_to_f16<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-        reinterpret_cast<const uint8_t *>(codes), ld_codes, bits, K, rows, map_mode, perm, topk, T,
-        reinterpret_cast<__half *>(out));
-    return cudaGetLastError();
+    return launch_pdl(k_codes_to_f16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, 1,
+                      reinterpret_cast<const uint8_t *>(codes), ld_codes, bits, K, rows, map_mode,
+                      perm, topk, T, reinterpret_cast<__half *>(out));
 }
 
 LutPath lut_path() {

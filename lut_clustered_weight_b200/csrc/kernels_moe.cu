@@ -19,6 +19,8 @@ constexpr int kTopkWarps = 8;
 __global__ void __launch_bounds__(kTopkWarps * 32)
 k_topk(const float *__restrict__ logits, int T, int E, int k, int renorm,
        int32_t *__restrict__ ids, float *__restrict__ w) {
+    griddep_wait();
+    griddep_launch();
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * kTopkWarps + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -86,6 +88,8 @@ k_group(const int32_t *__restrict__ ids, int T, int E, int k, int tile_rows,
     __shared__ int32_t hist[kGroupWarps][kMaxExperts];
     __shared__ int32_t s_off[kMaxExperts + 1];
     __shared__ int32_t s_tiles[kMaxExperts + 1];
+    griddep_wait();
+    griddep_launch();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int S = T * k;
     for (int i = tid; i < kGroupWarps * kMaxExperts; i += kGroupThreads) (&hist[0][0])[i] = 0;
@@ -160,11 +164,12 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
                          int32_t *inv_perm, int32_t *grp_tiles, int32_t *tile_grp,
                          int max_tiles, cudaStream_t st) {
     count_launch(2);
-    k_topk<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, st>>>(logits, T, E, k,
-                                                                          renorm, ids, w);
-    k_group<<<1, kGroupThreads, 0, st>>>(ids, T, E, k, tile_rows, counts, offsets, perm, inv_perm,
-                                         grp_tiles, tile_grp, max_tiles);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(k_topk, dim3((T + kTopkWarps - 1) / kTopkWarps),
+                               dim3(kTopkWarps * 32), 0, st, 1, logits, T, E, k, renorm, ids, w);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_group, dim3(1), dim3(kGroupThreads), 0, st, 1, (const int32_t *)ids, T, E,
+                      k, tile_rows, counts, offsets, perm, inv_perm, grp_tiles, tile_grp,
+                      max_tiles);
 }
 
 // ------------------------------------------------------------------ combine
@@ -176,6 +181,8 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
     __shared__ float s_c[kMaxTopK];   // w[t, j] (scale of row p applied separately)
     __shared__ float s_sh[kMaxTopK];  // h scale of row p
     __shared__ int s_ns[4][24];       // slot counts, shared expert x row tile of this block (<= 17)
+    griddep_wait();
+    griddep_launch();
     const int t = blockIdx.x;
     const int n0 = blockIdx.y * 1024;
     if (threadIdx.x < a.topk) {
@@ -220,28 +227,18 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
             acc.x += c * y[u].x; acc.y += c * y[u].y; acc.z += c * y[u].z; acc.w += c * y[u].w;
         }
     }
-    // shared experts (at most four)
-    if (a.n_shared > 0) {
-        float4 y[4];
-        const float4 *ps[4];
-        int nss[4];
-#pragma unroll
-        for (int s = 0; s < 4; s++) {
-            y[s] = make_float4(0.f, 0.f, 0.f, 0.f);
-            const int64_t lp = (int64_t)min(s, a.n_shared - 1) * a.T + t;
-            ps[s] = reinterpret_cast<const float4 *>(a.part_s + lp * a.H + n);
-            nss[s] = s < a.n_shared ? s_ns[s][n / rpt - rt0] : 0;
-        }
-        sum_slots<4>(ps, nss, stride_s, y);
-#pragma unroll
-        for (int s = 0; s < 4; s++) {
-            if (s >= a.n_shared) break;
-            const int64_t lp = (int64_t)s * a.T + t;
-            const float sc = a.h_scales[a.R_routed + lp];
-            y[s].x *= sc; y[s].y *= sc; y[s].z *= sc; y[s].w *= sc;
-            if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + (a.R_routed + lp) * a.H + n) = y[s];
-            acc.x += y[s].x; acc.y += y[s].y; acc.z += y[s].z; acc.w += y[s].w;
-        }
+    // shared experts (at most four), eight split-K slots per round: a dense
+    // layer's down projection is split over many CTAs at decode
+    for (int s = 0; s < a.n_shared; s++) {
+        const int64_t lp = (int64_t)s * a.T + t;
+        const float4 *ps[1] = {reinterpret_cast<const float4 *>(a.part_s + lp * a.H + n)};
+        const int nss[1] = {s_ns[s][n / rpt - rt0]};
+        float4 y[1] = {make_float4(0.f, 0.f, 0.f, 0.f)};
+        sum_slots<1, 8>(ps, nss, stride_s, y);
+        const float sc = a.h_scales[a.R_routed + lp];
+        y[0].x *= sc; y[0].y *= sc; y[0].z *= sc; y[0].w *= sc;
+        if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + (a.R_routed + lp) * a.H + n) = y[0];
+        acc.x += y[0].x; acc.y += y[0].y; acc.z += y[0].z; acc.w += y[0].w;
     }
     *reinterpret_cast<float4 *>(a.out + (int64_t)t * a.H + n) = acc;
 }
@@ -249,8 +246,8 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
     if ((int64_t)a.T * a.H == 0) return cudaSuccess;
     count_launch();
-    k_combine<<<dim3((unsigned)a.T, (unsigned)((a.H + 1023) / 1024)), 256, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k_combine, dim3((unsigned)a.T, (unsigned)((a.H + 1023) / 1024)), dim3(256), 0,
+                      st, 1, a);
 }
 
 }  // namespace cq

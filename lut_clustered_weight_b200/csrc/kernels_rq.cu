@@ -81,6 +81,8 @@ k_rq_x(const __half *__restrict__ x, int64_t ldx, int K, int log2b, int bits,
        uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s) {
     extern __shared__ __align__(16) double buf[];
     int cs, rank;
+    griddep_wait();
+    griddep_launch();
     cluster_pos<CLUSTER>(cs, rank);
     const int64_t m = blockIdx.x / cs;
     const RowPart part = row_part(K, log2b, rank, cs);
@@ -105,6 +107,8 @@ k_rq_x(const __half *__restrict__ x, int64_t ldx, int K, int log2b, int bits,
 template <bool CLUSTER>
 __global__ void __launch_bounds__(kRqThreads) k_rq_swiglu(const SwigluArgs a) {
     extern __shared__ __align__(16) double buf[];
+    griddep_wait();
+    griddep_launch();
     int cs, rank;
     cluster_pos<CLUSTER>(cs, rank);
     const int64_t p = blockIdx.x / cs;
@@ -140,7 +144,7 @@ __global__ void __launch_bounds__(kRqThreads) k_rq_swiglu(const SwigluArgs a) {
             pf[f] = reinterpret_cast<const float2 *>(rowp + 2 * n);
             nsf[f] = i < rp.n ? s_ns[n / P.rows_per_rt - rt0] : 0;
         }
-        sum_slots<4>(pf, nsf, slot_stride / 2, acc);
+        sum_slots<4, 4>(pf, nsf, slot_stride / 2, acc);
 #pragma unroll
         for (int f = 0; f < 4; f++) {
             const int i = i0 + f * kRqThreads + threadIdx.x;
@@ -165,6 +169,8 @@ __global__ void __launch_bounds__(kWarpRows * 32)
 k_rq_x_warp(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log2b, int bits,
             uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s) {
     extern __shared__ __align__(16) double wbuf[];
+    griddep_wait();
+    griddep_launch();
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int64_t m = (int64_t)blockIdx.x * kWarpRows + w;
     if (m >= M) return;
@@ -188,6 +194,8 @@ k_rq_x_warp(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log
 __global__ void __launch_bounds__(kWarpRows * 32) k_rq_swiglu_warp(const SwigluArgs a, int64_t R) {
     extern __shared__ __align__(16) double wbuf[];
     __shared__ int s_ns[kWarpRows][kMaxK / 64];
+    griddep_wait();
+    griddep_launch();
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int64_t p = (int64_t)blockIdx.x * kWarpRows + w;
     if (p >= R) return;
@@ -260,25 +268,8 @@ static cudaError_t launch_clustered(Kern kern, int64_t rows, int cs, size_t smem
                                     cudaStream_t st, Args... args) {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)(kMaxK * sizeof(double)));
-    if (cs == 1) {  // one CTA per row: a plain launch
-        count_launch();
-        kern<<<(unsigned)rows, kRqThreads, smem, st>>>(args...);
-        return cudaGetLastError();
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(rows * cs));
-    cfg.blockDim = dim3(kRqThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     count_launch();
-    return cudaLaunchKernelEx(&cfg, kern, args...);
+    return launch_pdl(kern, dim3((unsigned)(rows * cs)), dim3(kRqThreads), smem, st, cs, args...);
 }
 
 cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K, int log2b,
@@ -289,10 +280,9 @@ cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K,
         cudaFuncSetAttribute(k_rq_x_warp, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(kWarpRows * 4096 * sizeof(double)));
         count_launch();
-        k_rq_x_warp<<<(unsigned)((M + kWarpRows - 1) / kWarpRows), kWarpRows * 32, smem, st>>>(
-            reinterpret_cast<const __half *>(x), ldx, M, K, log2b, bits,
-            reinterpret_cast<uint8_t *>(q), ldq, s);
-        return cudaGetLastError();
+        return launch_pdl(k_rq_x_warp, dim3((unsigned)((M + kWarpRows - 1) / kWarpRows)),
+                          dim3(kWarpRows * 32), smem, st, 1, reinterpret_cast<const __half *>(x),
+                          ldx, M, K, log2b, bits, reinterpret_cast<uint8_t *>(q), ldq, s);
     }
     const int cs = cluster_size(M, K, log2b);
     auto kern = cs == 1 ? k_rq_x<false> : k_rq_x<true>;
@@ -310,9 +300,8 @@ cudaError_t launch_swiglu_rq(const SwigluArgs &a, int64_t rows, cudaStream_t st)
         cudaFuncSetAttribute(k_rq_swiglu_warp, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(kWarpRows * 4096 * sizeof(double)));
         count_launch();
-        k_rq_swiglu_warp<<<(unsigned)((rows + kWarpRows - 1) / kWarpRows), kWarpRows * 32, smem,
-                           st>>>(a, rows);
-        return cudaGetLastError();
+        return launch_pdl(k_rq_swiglu_warp, dim3((unsigned)((rows + kWarpRows - 1) / kWarpRows)),
+                          dim3(kWarpRows * 32), smem, st, 1, a, rows);
     }
     // one cluster size for the launch: the coarser of the two row kinds
     int cs = kMaxCluster;
