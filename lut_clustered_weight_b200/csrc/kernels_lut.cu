@@ -58,7 +58,6 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint2 *bfrag = reinterpret_cast<uint2 *>(smem_raw);
     uint4 *ring = reinterpret_cast<uint4 *>(smem_raw + (size_t)P.cps_max * NT * 2048);
-    __shared__ int s_code_row[kTokTile];
     __shared__ float s_scale[kTokTile];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -87,6 +86,8 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
     }
 
     float acc[NT][4];
+    uint4 cbv[4];          // codebook rows A and B of a new item, loaded ahead
+    bool tables_pending = false;
     int64_t cur_w = -1;
     int cur_s = 0, row0 = 0, nrows = 0, nA = 0, nB = 0;
     const uint8_t *pA = nullptr, *pB = nullptr;
@@ -166,29 +167,33 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
                 cA = reinterpret_cast<const __half *>(L.cb0) + (int64_t)g * L.cb_stride + nA * 16;
                 cB = cA + 8 * 16;
             }
-            // weight stream first, so HBM latency overlaps the set-up below
+            // the 64 codebook bytes go out ahead of the weight stream (behind
+            // several KB of weights per lane they would wait in the DRAM queues),
+            // then the stream, whose latency overlaps the set-up below
+            cbv[0] = *reinterpret_cast<const uint4 *>(cA);
+            cbv[1] = *reinterpret_cast<const uint4 *>(cA + 8);
+            cbv[2] = *reinterpret_cast<const uint4 *>(cB);
+            cbv[3] = *reinterpret_cast<const uint4 *>(cB + 8);
+            tables_pending = true;  // built once the activation loads are out too
 #pragma unroll
             for (int sl = 0; sl < kStages - 1; sl++) {
                 if (sl < nch) issue(ch_lo + sl, sl);
                 cp_async_commit();
             }
-            build_tables(cA, loA, hiA);
-            build_tables(cB, loB, hiB);
 #pragma unroll
             for (int t = 0; t < NT; t++)
 #pragma unroll
                 for (int e = 0; e < 4; e++) acc[t][e] = 0.0f;
-            __syncthreads();  // previous piece is done with s_code_row / bfrag
+            __syncthreads();  // previous piece is done with s_scale / bfrag
             griddep_wait();   // activations and scales come from the previous kernel
-            if (tid < TT) {
+            if (tid < TT && L.direct) {
                 int cr = -1;
                 if (tid < nrows) {
                     const int p = row0 + tid;
                     cr = L.map_mode == kMapPerm ? L.perm[p] / L.topk
                        : L.map_mode == kMapModT ? p % L.T : p;
                 }
-                s_code_row[tid] = cr;
-                s_scale[tid] = (cr >= 0 && L.direct) ? L.scales[cr] : 0.0f;
+                s_scale[tid] = cr >= 0 ? L.scales[cr] : 0.0f;
             }
         } else {
 #pragma unroll
@@ -197,7 +202,7 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
                 cp_async_commit();
             }
         }
-        __syncthreads();  // s_code_row visible; bfrag free
+        __syncthreads();  // bfrag free (the first piece of an item synchronised above)
 
         // ---- activation fragments for chunks [ch_lo, ch_hi).  An item is the
         // 32 consecutive k of one token that one lane consumes (lane = 4*(token
@@ -214,7 +219,13 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
                     const int it = it0 + f * W * 32;
                     if (it < items) {
                         const int ln = it & 31, nt = (it >> 5) % NT, ch = (it >> 5) / NT;
-                        const int cr = s_code_row[8 * nt + (ln >> 2)];
+                        const int tok = 8 * nt + (ln >> 2);
+                        int cr = -1;
+                        if (tok < nrows) {
+                            const int p = row0 + tok;
+                            cr = L.map_mode == kMapPerm ? L.perm[p] / L.topk
+                               : L.map_mode == kMapModT ? p % L.T : p;
+                        }
                         const int k0 = (ch_lo + ch) * 128 + 32 * (ln & 3);
                         if (cr >= 0 && k0 < K) {
                             const uint8_t *src = L.codes + (int64_t)cr * L.ld_codes;
@@ -226,6 +237,11 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
                             }
                         }
                     }
+                }
+                if (tables_pending) {  // the codebook loads went out with the weights
+                    build_tables(cbv[0], cbv[1], loA, hiA);
+                    build_tables(cbv[2], cbv[3], loB, hiB);
+                    tables_pending = false;
                 }
 #pragma unroll
                 for (int f = 0; f < FB; f++) {
@@ -255,6 +271,11 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
                     }
                 }
             }
+        }
+        if (tables_pending) {  // no activation items for this thread
+            build_tables(cbv[0], cbv[1], loA, hiA);
+            build_tables(cbv[2], cbv[3], loB, hiB);
+            tables_pending = false;
         }
         __syncthreads();
 

@@ -9,15 +9,17 @@ namespace cq {
 
 // Byte-plane tables of one codebook row: lo[j] holds the low bytes of
 // C[4j..4j+3], hi[j] the high bytes.
-CQ_DEV void build_tables(const __half *cb, uint32_t (&lo)[4], uint32_t (&hi)[4]) {
-    const uint4 a = *reinterpret_cast<const uint4 *>(cb);
-    const uint4 b = *reinterpret_cast<const uint4 *>(cb + 8);
+CQ_DEV void build_tables(const uint4 a, const uint4 b, uint32_t (&lo)[4], uint32_t (&hi)[4]) {
     const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int j = 0; j < 4; j++) {
         lo[j] = prmt(u[2 * j], u[2 * j + 1], 0x6420);
         hi[j] = prmt(u[2 * j], u[2 * j + 1], 0x7531);
     }
+}
+CQ_DEV void build_tables(const __half *cb, uint32_t (&lo)[4], uint32_t (&hi)[4]) {
+    build_tables(*reinterpret_cast<const uint4 *>(cb), *reinterpret_cast<const uint4 *>(cb + 8), lo,
+                 hi);
 }
 
 // Eight 4-bit indices (nibble i of w = index of element i) -> four half2:
