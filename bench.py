@@ -385,6 +385,22 @@ class DeviceLayer:
         return c.cpu().numpy()
 
 
+def max_over_ranks(ms, dist, world, device="cuda"):
+    """The slowest rank's time: every rank gets the max (replicas are timed
+    on the device and the job is as slow as its slowest GPU)."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_step, steps, world, ms):
+    """Whole-job rate: the units all ranks processed over the max-over-ranks time."""
+    return units_per_step * steps * world / (ms / 1e3)
+
+
 def timed(fn, steps, dist, world):
     """Device time (ms) of `steps` calls of fn on the current stream,
     bracketed by barrier + synchronize on both sides; max over ranks."""
@@ -401,12 +417,7 @@ def timed(fn, steps, dist, world):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return max_over_ranks(e0.elapsed_time(e1), dist, world)
 
 
 def main():
@@ -481,7 +492,7 @@ def main():
         ms = timed(run, args.steps, dist, world)
     clocks = clk.summary()
     ms_step = ms / args.steps
-    value = tokens_per_step * args.steps * world / (ms / 1e3)
+    value = job_throughput(tokens_per_step, args.steps, world, ms)
 
     # ---- the LUT GEMM kernel, CUDA-event timed launch by launch (eager steps).
     # A spin kernel ahead of every step keeps the GPU busy while the host
@@ -514,7 +525,7 @@ def main():
     for _ in range(args.warmup):
         step_e2e()
     ms_e2e = timed(step_e2e, args.steps, dist, world)
-    e2e = {"value": tokens_per_step * args.steps * world / (ms_e2e / 1e3), "unit": "tokens/s",
+    e2e = {"value": job_throughput(tokens_per_step, args.steps, world, ms_e2e), "unit": "tokens/s",
            "h2d_bytes_per_step": sum(L.h2d for L in layers),
            "d2h_bytes_per_step": sum(L.d2h for L in layers),
            "ms_per_step": ms_e2e / args.steps}
