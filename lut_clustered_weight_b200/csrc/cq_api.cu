@@ -70,6 +70,7 @@ struct MoePlan {
     size_t o_pgu_r, o_pgu_s, o_hq, o_sh, o_pdn_r, o_pdn_s;
     size_t o_bx_r, o_bx_s, o_bh_r, o_bh_s;  // fp16 B operands of tensor-core launches
     size_t o_hf;                            // fused: h fp16 [R][Imax]
+    size_t o_rs;                            // fused: x scale per routed row [Rr]
     size_t total;
 };
 
@@ -149,6 +150,7 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
     m.o_pgu_r = take(m.E > 0 && !m.fused ? (size_t)m.gu_r.splits * m.Rr * m.I * 2 * 4 : 0);
     m.o_pgu_s = take(m.ns > 0 && !m.fused ? (size_t)m.gu_s.splits * m.Rs * m.Is * 2 * 4 : 0);
     m.o_hf = take(m.fused ? (size_t)m.R * m.Imax * 2 : 0);
+    m.o_rs = take(m.fused && m.E > 0 ? (size_t)m.Rr * 4 : 0);
     m.o_hq = take((size_t)m.R * code_bytes(m.Imax, m.bits));
     m.o_sh = take((size_t)m.R * 4);
     m.o_pdn_r = take(m.E > 0 ? (size_t)m.dn_r.splits * m.Rr * m.H * 4 : 0);
@@ -333,6 +335,7 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
     float *pdn_r = reinterpret_cast<float *>(ws + m.o_pdn_r);
     float *pdn_s = reinterpret_cast<float *>(ws + m.o_pdn_s);
     __half *hf = reinterpret_cast<__half *>(ws + m.o_hf);
+    float *rsc = reinterpret_cast<float *>(ws + m.o_rs);
     const int64_t ldx = code_bytes(m.H, m.bits), ldh = code_bytes(m.Imax, m.bits);
 
     cudaError_t e = launch_rotate_quantize(x, m.H, T, (int)m.H, ilog2(d->had_block_h), m.bits, xq,
@@ -351,13 +354,14 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.out = pgu_r; L.out_split_stride = m.Rr * m.I * 2; L.out_row_stride = m.I * 2;
         if (m.fused) {
             L.scales = sx;
+            L.row_scales = rsc;
             L.h_out = hf;
             L.h_row_stride = m.Imax;
         }
         if (m.tc_r) {
             void *b = ws + m.o_bx_r;
             e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, m.Rr, kMapPerm, perm, (int)m.k,
-                                    (int)T, b, st);
+                                    (int)T, b, st, m.fused ? sx : nullptr, rsc);
             if (e == cudaSuccess) e = launch_lut_tc(L, m.gu_r, b, m.Rr, 0, st);
         } else {
             e = launch_lut(L, m.gu_r, st);

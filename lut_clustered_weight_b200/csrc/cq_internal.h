@@ -58,6 +58,7 @@ struct LutLaunch {
     // row of p], written at h_out + p * h_row_stride + n
     __half *h_out;
     int64_t h_row_stride;   // elements
+    const float *row_scales;  // fused, kMapPerm: scale of output row p, gathered
 };
 
 // How one LUT GEMM launch is cut into work.  A work item is (token tile,
@@ -129,9 +130,11 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
 cudaError_t launch_lut_tc(const LutLaunch &L, const LutPlan &P, const void *b_f16, int64_t b_rows,
                           int b_row_mod, cudaStream_t st);
 // fp16 copies of activation codes (B operand), rows mapped like LutLaunch::map_mode.
+// scales_in != nullptr: also writes scales_out[p] = scales_in[code row of p].
 cudaError_t launch_codes_to_f16(const void *codes, int64_t ld_codes, int bits, int K,
                                 int64_t rows, int map_mode, const int32_t *perm, int topk, int T,
-                                void *out, cudaStream_t st);
+                                void *out, cudaStream_t st, const float *scales_in = nullptr,
+                                float *scales_out = nullptr);
 // Reads and clears the device error word (-1 if the read failed).
 int read_device_error();
 // Which LUT kernel a launch uses: "mma" (mma.sync, register tables), "tc"

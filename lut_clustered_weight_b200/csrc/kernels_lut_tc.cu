@@ -180,10 +180,14 @@ CQ_DEV int64_t tc_pieces(const LutLaunch &L, const LutPlan &P) {
 }
 
 // Activation scale of output row p (the row's token).
+// Issued as a volatile load at segment start, so the compiler cannot sink it to
+// the epilogue, where it would stall the drain of the accumulator.
 CQ_DEV float tc_row_scale(const LutLaunch &L, int64_t p) {
-    const int64_t cr = L.map_mode == kMapPerm ? L.perm[p] / L.topk
-                     : L.map_mode == kMapModT ? p % L.T : p;
-    return L.scales[cr];
+    const float *src = L.row_scales ? L.row_scales + p
+                     : L.scales + (L.map_mode == kMapModT ? p % L.T : p);
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(src));
+    return v;
 }
 
 template <int NTOK, bool PAIR>
@@ -510,40 +514,51 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                             for (int bb = 0; bb < kLd; bb++)
                                 tmem_ld16(tmem_d + lane_base + a * NTOK + c0 + 16 * bb, d[a * kLd + bb]);
                         tmem_wait_ld();
+                        if (L.h_out) {
+                            // SwiGLU.  Lanes 2j (gate) and 2j + 1 (up) hold the same output
+                            // column; the even lane finishes token c and the odd lane token
+                            // c + 1 after one exchange.  All values first (independent
+                            // chains, no branches), then the predicated stores.
+                            const int odd = lane & 1;
+                            __half hv[kLd * 8];
 #pragma unroll
-                        for (int bb = 0; bb < kLd; bb++)
+                            for (int bb = 0; bb < kLd; bb++)
 #pragma unroll
-                            for (int qq = 0; qq < 16; qq += 2) {
-                                float a0 = __uint_as_float(d[bb][qq]);
-                                float a1 = __uint_as_float(d[bb][qq + 1]);
+                                for (int qq = 0; qq < 16; qq += 2) {
+                                    float a0 = __uint_as_float(d[bb][qq]);
+                                    float a1 = __uint_as_float(d[bb][qq + 1]);
 #pragma unroll
-                                for (int a = 1; a < kAcc; a++) {
-                                    a0 += __uint_as_float(d[a * kLd + bb][qq]);
-                                    a1 += __uint_as_float(d[a * kLd + bb][qq + 1]);
-                                }
-                                const int c = c0 + 16 * bb + qq;
-                                if (L.h_out) {
-                                    // SwiGLU.  Lanes 2j (gate) and 2j + 1 (up) hold the same
-                                    // output column; the even lane finishes token c and the
-                                    // odd lane token c + 1, after one exchange
-                                    const int odd = lane & 1;
+                                    for (int a = 1; a < kAcc; a++) {
+                                        a0 += __uint_as_float(d[a * kLd + bb][qq]);
+                                        a1 += __uint_as_float(d[a * kLd + bb][qq + 1]);
+                                    }
                                     const float recv =
                                         __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
                                     const float gv = odd ? recv : a0, uv = odd ? a1 : recv;
                                     const float sx =
                                         __shfl_sync(0xffffffffu, cur, 16 * bb + qq + odd);
-                                    if (c + odd < nrows) {
-                                        const int64_t p = row0 + c + odd;
-                                        L.h_out[p * L.h_row_stride + (col >> 1)] =
-                                            __float2half_rn(silu_mul(gv * sx, uv * sx));
-                                    }
-                                } else {
+                                    hv[bb * 8 + qq / 2] = __float2half_rn(silu_mul(gv * sx, uv * sx));
+                                }
+#pragma unroll
+                            for (int j = 0; j < kLd * 8; j++) {
+                                const int c = c0 + 2 * j + odd;
+                                if (c < nrows)
+                                    L.h_out[(int64_t)(row0 + c) * L.h_row_stride + (col >> 1)] = hv[j];
+                            }
+                        } else {
+#pragma unroll
+                            for (int bb = 0; bb < kLd; bb++)
+#pragma unroll
+                                for (int qq = 0; qq < 16; qq++) {
+                                    float a0 = __uint_as_float(d[bb][qq]);
+#pragma unroll
+                                    for (int a = 1; a < kAcc; a++)
+                                        a0 += __uint_as_float(d[a * kLd + bb][qq]);
+                                    const int c = c0 + 16 * bb + qq;
                                     if (c < nrows)
                                         out[(int64_t)(row0 + c) * L.out_row_stride + col] = a0;
-                                    if (c + 1 < nrows)
-                                        out[(int64_t)(row0 + c + 1) * L.out_row_stride + col] = a1;
                                 }
-                            }
+                        }
                     }
                 }
                 tc_fence_before();
@@ -677,7 +692,8 @@ cudaError_t launch_lut_tc(const LutLaunch &L, const LutPlan &P, const void *b_f1
 // tensor-core kernel.  One thread per 8 codes.
 __global__ void k_codes_to_f16(const uint8_t *__restrict__ codes, int64_t ld_codes, int bits,
                                int K, int64_t rows, int map_mode, const int32_t *__restrict__ perm,
-                               int topk, int T, __half *__restrict__ out) {
+                               int topk, int T, __half *__restrict__ out,
+                               const float *__restrict__ scales_in, float *__restrict__ scales_out) {
     griddep_wait();
     griddep_launch();
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -686,6 +702,7 @@ __global__ void k_codes_to_f16(const uint8_t *__restrict__ codes, int64_t ld_cod
     const int64_t p = i / per_row;
     const int k = (int)(i - p * per_row) * 8;
     const int64_t cr = map_mode == kMapPerm ? perm[p] / topk : map_mode == kMapModT ? p % T : p;
+    if (scales_in && k == 0) scales_out[p] = scales_in[cr];
     const uint8_t *src = codes + cr * ld_codes;
     __align__(16) __half v[8];
     if (bits == 4) {
@@ -705,13 +722,14 @@ __global__ void k_codes_to_f16(const uint8_t *__restrict__ codes, int64_t ld_cod
 
 cudaError_t launch_codes_to_f16(const void *codes, int64_t ld_codes, int bits, int K,
                                 int64_t rows, int map_mode, const int32_t *perm, int topk, int T,
-                                void *out, cudaStream_t st) {
+                                void *out, cudaStream_t st, const float *scales_in,
+                                float *scales_out) {
     const int64_t n = rows * (K / 8);
     if (n == 0) return cudaSuccess;
     count_launch();
     return launch_pdl(k_codes_to_f16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, 1,
                       reinterpret_cast<const uint8_t *>(codes), ld_codes, bits, K, rows, map_mode,
-                      perm, topk, T, reinterpret_cast<__half *>(out));
+                      perm, topk, T, reinterpret_cast<__half *>(out), scales_in, scales_out);
 }
 
 LutPath lut_path() {
