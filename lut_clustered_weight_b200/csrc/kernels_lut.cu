@@ -175,11 +175,10 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
             cbv[2] = *reinterpret_cast<const uint4 *>(cB);
             cbv[3] = *reinterpret_cast<const uint4 *>(cB + 8);
             tables_pending = true;  // built once the activation loads are out too
-#pragma unroll
-            for (int sl = 0; sl < kStages - 1; sl++) {
-                if (sl < nch) issue(ch_lo + sl, sl);
-                cp_async_commit();
-            }
+            // first stage of the weight stream now; the rest once the set-up
+            // loads are out, so they do not queue behind the whole burst
+            if (nch > 0) issue(ch_lo, 0);
+            cp_async_commit();
 #pragma unroll
             for (int t = 0; t < NT; t++)
 #pragma unroll
@@ -196,11 +195,8 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
                 s_scale[tid] = cr >= 0 ? L.scales[cr] : 0.0f;
             }
         } else {
-#pragma unroll
-            for (int sl = 0; sl < kStages - 1; sl++) {
-                if (sl < nch) issue(ch_lo + sl, sl);
-                cp_async_commit();
-            }
+            if (nch > 0) issue(ch_lo, 0);
+            cp_async_commit();
         }
         __syncthreads();  // bfrag free (the first piece of an item synchronised above)
 
@@ -276,6 +272,11 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 4) k_lut_mma(const LutLau
             build_tables(cbv[0], cbv[1], loA, hiA);
             build_tables(cbv[2], cbv[3], loB, hiB);
             tables_pending = false;
+        }
+#pragma unroll
+        for (int sl = 1; sl < kStages - 1; sl++) {
+            if (sl < nch) issue(ch_lo + sl, sl);
+            cp_async_commit();
         }
         __syncthreads();
 
