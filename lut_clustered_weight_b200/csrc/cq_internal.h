@@ -62,28 +62,32 @@ struct LutLaunch {
 };
 
 // How one LUT GEMM launch is cut into work.  A work item is (token tile,
-// row tile); its contraction is cut into 128-k chunks, and the units
-// (work item, chunk) are shared out in one of two ways:
-//   fixed    every work item is split into `splits` equal chunk ranges; the
-//            grid is (row tiles * splits) x (token tiles).  Used when the
-//            token tiles are only known on the device (routed experts).
+// row tile); its contraction is cut into chunks (128 k for the mma.sync
+// kernel, 64 k for the tensor-memory kernel), and the units (work item,
+// chunk) are shared out in one of two ways:
+//   fixed    every work item is split into `splits` equal chunk ranges.  The
+//            mma.sync kernel's grid is (row tiles * splits) x (token tiles);
+//            the tensor-memory kernel runs one CTA per SM that strides over
+//            the (item, split) pieces.  Used when the token tiles are only
+//            known on the device (routed experts), and by the tensor-memory
+//            kernel whenever there are many work items.
 //   stream-K the W*C units of all work items are dealt out in equal
 //            contiguous ranges to `grid` CTAs (one wave), so no SM waits on
 //            a tail.  A work item is then covered by a variable number of
 //            CTAs; its partial sums occupy slots 0..n-1.
 struct LutPlan {
     int nt;             // n8 token tiles per CTA (1 or 2): a token tile has 8*nt rows
-    int warps;          // warps per CTA (4 or 8)
+    int warps;          // mma.sync kernel: warps per CTA (4 or 8)
     int rows_per_rt;    // plain: weight rows per row tile; dual: output columns
     int n_row_tiles;
-    int chunks_total;   // C = ceil(K / 128)
+    int chunks_total;   // C = ceil(K / chunk)
     int cps_max;        // most chunks one CTA stages at a time (shared memory)
     int streamk;
-    int grid;           // CTAs (stream-K) / row_tiles * splits (fixed)
+    int grid;           // CTAs (x dimension)
     int splits;         // fixed: chunk ranges per work item; partial slots allocated
     int chunks_per_split;
     int64_t units;      // stream-K: total units (work items * C)
-    int uniform_rows;   // stream-K: rows per group (token tiles of a group are consecutive)
+    int uniform_rows;   // rows per group of a uniform launch (token tiles of a group are consecutive)
     int tc;             // 1: tensor-memory kernel (64-k chunks, 128-row tiles)
     size_t smem;
 };

@@ -7,28 +7,31 @@
 // held in shared memory followed by table lookups.  Here:
 //  * Two threads per weight row: row t of a 128-row tile is lane t of tensor
 //    memory (TMEM); of the eight "expand" warps, warps w and w + 4 both serve
-//    TMEM lane quarter w, one taking the low and one the high 32 k of every
-//    64-k chunk.
-//  * PAIR mode (decode): the one-time precompute is a 256-entry pair table per
-//    row in shared memory -- entry b holds the two fp16 centroids selected by
-//    an index byte b (low nibble = even k).  Entry b of thread t sits at
-//    b * 512 + 4 t, so the 32 lanes of a warp always hit 32 different banks,
-//    whatever the indices.  One byte (two weights) costs one byte extract,
-//    one address multiply-add and one 4-byte shared load.
-//  * PRMT mode (prefill): the codebook is held as two byte-plane tables in
-//    registers and looked up with byte permutes; no shared memory is spent on
-//    tables, which leaves room for wide activation tiles.
-//  * The looked-up fp16 weights of a 64-k chunk are stored to TMEM
-//    (tcgen05.st, 32 columns per row and chunk) and used as the A operand of
-//    tcgen05.mma kind::f16; the activations (int codes converted to fp16,
-//    exact) are the B operand, a 128-byte-swizzled shared tile loaded by TMA.
-//    The fp32 accumulator lives in TMEM and is read back with tcgen05.ld.
+//    TMEM lane quarter w, one taking the low and one the high 128 k of every
+//    4-chunk (256-k) group.
+//  * PAIR mode (16-token tiles): the one-time precompute is a 256-entry pair
+//    table per row in shared memory -- entry b holds the two fp16 centroids
+//    selected by an index byte b (low nibble = even k).  Entry b of thread t
+//    sits at b * 512 + 4 t, so the 32 lanes of a warp always hit 32 different
+//    banks, whatever the indices.  One byte (two weights) costs one byte
+//    extract, one address multiply-add and one 4-byte shared load.
+//  * PRMT mode (64- to 256-token tiles): the codebook is held as two
+//    byte-plane tables in registers and looked up with byte permutes; no
+//    shared memory is spent on tables, which leaves room for wide B tiles.
+//  * The looked-up fp16 weights of a group are stored to TMEM (tcgen05.st,
+//    32 columns per row and chunk, a 2-group ring) and used as the A operand
+//    of tcgen05.mma kind::f16; the activations (int codes converted to fp16,
+//    exact) are the B operand, 128-byte-swizzled shared tiles loaded by TMA.
+//    The fp32 accumulator lives in TMEM and is read back with tcgen05.ld; the
+//    epilogue writes fp32 partial sums, or fp16 h = silu(s g) (s u) when the
+//    launch has one partial slot per output (SwiGLU fused).
 //  * Roles: warps 0-7 expand (each thread streams its row's index bytes
-//    through a private cp.async ring) and write the accumulator back; lane 0
-//    of warp 8 issues the MMAs; lane 0 of warp 9 issues the TMA loads of the
+//    through a private cp.async ring) and drain the accumulator; lane 0 of
+//    warp 8 issues the MMAs; lane 0 of warp 9 issues the TMA loads of the
 //    activation tiles.  mbarriers connect them; every wait is bounded.
-//  * Work is cut into (128-row tile x token tile) items and 64-k chunks,
-//    shared out like the mma.sync kernel (stream-K for uniform launches).
+//  * Persistent: one CTA per SM works through (128-row tile x token tile)
+//    items cut into 64-k chunks -- contiguous stream-K ranges when there are
+//    few items, else whole (item, split) pieces strided over the CTAs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -615,7 +618,6 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
     LutPlan P{};
     const int ntok = tc_ntok_for(max_rows_per_group);
     P.nt = ntok / 8;
-    P.warps = 4;
     P.rows_per_rt = dual ? 64 : kTcRows;
     P.n_row_tiles = N / P.rows_per_rt;
     P.chunks_total = (K + kTcChunk - 1) / kTcChunk;
