@@ -401,6 +401,41 @@ def job_throughput(units_per_step, steps, world, ms):
     return units_per_step * steps * world / (ms / 1e3)
 
 
+def bf16_dense_context(shapes, dev, stream, steps, warmup, dist, world):
+    """tokens/s of the same dense SwiGLU FFN calls done in bf16 by torch
+    (F.linear on dense weights, one weight copy per call), replayed from a
+    CUDA graph and timed like the main leg."""
+    import torch
+    import torch.nn.functional as F
+    g = torch.Generator(device=dev).manual_seed(0)
+    calls = []
+    for s in shapes:
+        wgu = torch.randn((2 * s.I_shared, s.H), generator=g, device=dev, dtype=torch.bfloat16)
+        wd = torch.randn((s.H, s.I_shared), generator=g, device=dev, dtype=torch.bfloat16)
+        x = torch.randn((s.T, s.H), generator=g, device=dev, dtype=torch.bfloat16)
+        calls.append((x, wgu.mul_(0.02), wd.mul_(0.02), s.I_shared))
+
+    def step():
+        for x, wgu, wd, i in calls:
+            gu = F.linear(x, wgu)
+            F.linear(F.silu(gu[:, :i]) * gu[:, i:], wd)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    for _ in range(warmup):
+        graph.replay()
+    ms = timed(graph.replay, steps, dist, world)
+    tokens = sum(s.T for s in shapes)
+    return {"value": job_throughput(tokens, steps, world, ms), "unit": "tokens/s",
+            "ms_per_step": ms / steps,
+            "what": "torch bf16 F.linear dense SwiGLU FFN, same shapes and tokens, "
+                    "own dense weight copy per call, CUDA graph"}
+
+
 def timed(fn, steps, dist, world):
     """Device time (ms) of `steps` calls of fn on the current stream,
     bracketed by barrier + synchronize on both sides; max over ranks."""
@@ -431,6 +466,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    ap.add_argument("--no-bf16", action="store_true", help="skip the torch bf16 context leg")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -530,6 +566,14 @@ def main():
            "d2h_bytes_per_step": sum(L.d2h for L in layers),
            "ms_per_step": ms_e2e / args.steps}
 
+    # ---- context: the same dense FFN step in bf16 with torch (F.linear, dense
+    # weights, own weight copy per call, CUDA graph) -- the pages compare
+    # their decode kernel against BF16
+    bf16 = None
+    if all(s.E == 0 for s in shapes) and not args.no_bf16:
+        bf16 = bf16_dense_context(shapes, dev, stream, args.steps, args.warmup, dist, world)
+        bf16["speedup_of_value"] = value / bf16["value"]
+
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -553,7 +597,7 @@ def main():
                        "parallelism": f"replicas x{world}"},
             "effective_gbs": alg_bytes_step / (ms_step / 1e3) / 1e9,
             "alg_bytes_per_step": alg_bytes_step, "alg_flops_per_step": alg_flops_step,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "bf16_context": bf16,
             "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
             "dtype_note": "int4/int8 codes and 4-bit indices; looked-up weights as fp16 "
                           "into mma.sync (decode) or tcgen05 kind::f16 (more than 16 "
