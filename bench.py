@@ -577,9 +577,15 @@ def main():
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
+        import oracle
         n, dt, desc = cpu_oracle_sample(shapes, inputs, args.cpu_seconds)
         cpu = {"value": n / dt, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
                "sample": desc}
+        oracle.set_threads(1)
+        n1, dt1, desc1 = cpu_oracle_sample(shapes, inputs, args.cpu_seconds / 3)
+        oracle.set_threads(oracle_threads())
+        cpu["single_thread"] = {"value": n1 / dt1, "unit": "tokens/s", "cores": 1,
+                                "sample": desc1}
 
     if world > 1:
         dist.barrier()

@@ -47,6 +47,11 @@ def build(force: bool = False) -> Path:
     return _LIB
 
 
+def set_threads(n: int) -> None:
+    """Host threads the oracle's row loops may use (timing only)."""
+    lib().orc_set_threads(int(n))
+
+
 def lib():
     global _lib
     if _lib is None:
@@ -57,6 +62,8 @@ def lib():
         _lib.orc_f64_to_f16.argtypes = [D]
         _lib.orc_f64_to_f16.restype = ctypes.c_uint16
         _lib.orc_hadamard_matrix.argtypes = [I64, P]
+        _lib.orc_set_threads.argtypes = [I32]
+        _lib.orc_set_threads.restype = None
         _lib.orc_rotate.argtypes = [P, I64, I64, I64, P]
         _lib.orc_quantize.argtypes = [P, I64, I64, I64, I32, P, P]
         _lib.orc_rotate_quantize.argtypes = [P, I64, I64, I64, I32, P, P]

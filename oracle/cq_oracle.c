@@ -38,6 +38,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_OK 0
 #define ORC_EINVAL 1
@@ -390,4 +393,14 @@ void orc_combine(const double *y_slot, const double *w, int64_t T, int64_t k, in
                 acc += y_shared[(s * T + t) * H + h];
             out[t * H + h] = acc;
         }
+}
+
+/* Host threads the loops above may use (timing only; results do not depend on it). */
+void orc_set_threads(int n)
+{
+#ifdef _OPENMP
+    omp_set_num_threads(n > 0 ? n : 1);
+#else
+    (void)n;
+#endif
 }
