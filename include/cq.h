@@ -280,6 +280,15 @@ CQ_API int64_t cq_launch_count(void);
  * read.
  */
 CQ_API int32_t cq_device_error(void);
+
+/*
+ * cq_selftest_wait_timeout -- runs one kernel whose bounded wait can never be
+ * satisfied (an mbarrier nothing arrives on): it gives up after about one
+ * second, sets the device error word to 1 and returns, leaving the context
+ * usable.  Exercises the error path of the tensor-core kernels' waits for
+ * tests.  Asynchronous on stream; CQ_ERR_CUDA if the launch failed.
+ */
+CQ_API cq_status cq_selftest_wait_timeout(cq_stream_t stream);
 CQ_API cq_status cq_timing_enable(int32_t on);
 CQ_API cq_status cq_timing_read(int64_t *launches, double *total_ms);
 CQ_API cq_status cq_timing_read_launches(int32_t *kinds, float *ms, int64_t cap, int64_t *n);

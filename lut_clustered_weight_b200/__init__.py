@@ -20,7 +20,7 @@ LIB_PATH = _PKG / "libcq_b200.so"
 EXPORTS = ("cq_status_string", "cq_version", "cq_rotate_quantize", "cq_lut_gemm_workspace_size",
            "cq_lut_gemm", "cq_moe_ffn_workspace_size", "cq_moe_ffn", "cq_launch_count",
            "cq_timing_enable", "cq_timing_read", "cq_lut_gemm_noalloc", "cq_device_error",
-           "cq_timing_read_launches")
+           "cq_timing_read_launches", "cq_selftest_wait_timeout")
 
 CQ_OK, CQ_ERR_INVALID_ARGUMENT, CQ_ERR_UNSUPPORTED, CQ_ERR_WORKSPACE, CQ_ERR_CUDA = range(5)
 
@@ -85,6 +85,8 @@ lib.cq_timing_enable.argtypes = [_I32]
 lib.cq_timing_enable.restype = ctypes.c_int
 lib.cq_timing_read.argtypes = [ctypes.POINTER(_I64), ctypes.POINTER(ctypes.c_double)]
 lib.cq_timing_read.restype = ctypes.c_int
+lib.cq_selftest_wait_timeout.argtypes = [_P]
+lib.cq_selftest_wait_timeout.restype = ctypes.c_int
 lib.cq_timing_read_launches.argtypes = [_P, _P, _I64, ctypes.POINTER(_I64)]
 lib.cq_timing_read_launches.restype = ctypes.c_int
 
@@ -109,6 +111,12 @@ def cq_timing_read() -> tuple[int, float]:
     ms = ctypes.c_double(0.0)
     _check(lib.cq_timing_read(ctypes.byref(n), ctypes.byref(ms)), "cq_timing_read")
     return int(n.value), float(ms.value)
+
+
+def cq_selftest_wait_timeout(stream=None) -> None:
+    """Launch the kernel whose bounded wait always runs out (about 1 s); it sets
+    the device error word read by cq_device_error()."""
+    _check(lib.cq_selftest_wait_timeout(_stream(stream)), "cq_selftest_wait_timeout")
 
 
 KERNEL_KINDS = {0: "k_lut_mma", 1: "k_lut_tc"}   # cq_kernel_kind

@@ -139,6 +139,8 @@ cudaError_t launch_codes_to_f16(const void *codes, int64_t ld_codes, int bits, i
                                 int64_t rows, int map_mode, const int32_t *perm, int topk, int T,
                                 void *out, cudaStream_t st, const float *scales_in = nullptr,
                                 float *scales_out = nullptr);
+// Launches the bounded-wait self-test kernel (sets the device error word).
+cudaError_t launch_selftest_wait(cudaStream_t st);
 // Reads and clears the device error word (-1 if the read failed).
 int read_device_error();
 // Which LUT kernel a launch uses: "mma" (mma.sync, register tables), "tc"

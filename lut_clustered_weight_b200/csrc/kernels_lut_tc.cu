@@ -744,6 +744,24 @@ LutPath lut_path() {
     return p;
 }
 
+// One thread waits on an mbarrier that nothing ever arrives on: the bounded
+// wait gives up after about a second, records kErrWaitTimeout and the kernel
+// returns -- the error path every tensor-core kernel takes when a wait runs out.
+__global__ void k_selftest_wait() {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        mbar_wait(&bar, 0);
+    }
+}
+
+cudaError_t launch_selftest_wait(cudaStream_t st) {
+    count_launch();
+    k_selftest_wait<<<1, 32, 0, st>>>();
+    return cudaGetLastError();
+}
+
 int read_device_error() {
     int v = 0;
     if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return -1;

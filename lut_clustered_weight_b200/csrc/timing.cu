@@ -57,6 +57,12 @@ CQ_API int64_t cq_launch_count(void) { return cq::g_launches.load(); }
 
 CQ_API int32_t cq_device_error(void) { return cq::read_device_error(); }
 
+CQ_API cq_status cq_selftest_wait_timeout(cq_stream_t stream) {
+    return cq::launch_selftest_wait(reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? CQ_OK
+               : CQ_ERR_CUDA;
+}
+
 CQ_API cq_status cq_timing_enable(int32_t on) {
     cq::g_timing.store(on ? 1 : 0);
     return CQ_OK;
