@@ -1,5 +1,5 @@
 // sm100.cuh -- thin wrappers over the sm_100a PTX used by the tensor-memory
-// LUT kernel: mbarriers (with bounded waits), TMA tile loads (no multicast),
+// LUT kernel: mbarriers (with bounded waits), TMA tile loads into this CTA only,
 // tcgen05 tensor-memory allocation, MMA, commit, loads and stores.
 #pragma once
 
@@ -94,7 +94,7 @@ CQ_DEV void cp_async_wait_group() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// ---------------------------------------------------------------- TMA (tiled, no multicast)
+// ---------------------------------------------------------------- TMA (tiled, this CTA only)
 CQ_DEV void tma_load_2d(void *dst, const void *tmap, int x, int y, uint64_t *bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
