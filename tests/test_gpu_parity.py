@@ -225,6 +225,17 @@ def test_config3_mixtral_moe(cq):
 
 
 @pytest.mark.slow
+def test_dense_prefill_fused_epilogue(cq):
+    """A dense SwiGLU FFN at prefill size: the gate/up launch takes whole work
+    items per CTA with one partial slot, so SwiGLU runs in its epilogue."""
+    s = synth.MoEShape("dense_prefill_fused", H=128, I=4096, E=0, top_k=0, n_shared=1, T=2048,
+                       act_bits=4, had_block_h=128, had_block_i=256)
+    inp = moe_inputs_cached(s)
+    g = run_moe(inp)
+    check_moe(inp, g, sample_rows=8, sample_tokens=8)
+
+
+@pytest.mark.slow
 def test_config4_prefill_moe(cq):
     inp = moe_inputs_cached(synth.CFG4)
     g = run_moe(inp)
