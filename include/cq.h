@@ -23,7 +23,11 @@
  *               the end of this header it keeps no state between calls.
  *   Streams     work is enqueued on `stream` (NULL = legacy default stream)
  *               and the call returns without synchronizing.  Kernel faults
- *               surface at the caller's next synchronization.
+ *               surface at the caller's next synchronization.  Kernels are
+ *               launched with programmatic stream serialization: one may start
+ *               while the previous kernel on the stream is finishing, and it
+ *               waits for that kernel to complete before it reads any output
+ *               of it or writes global memory.
  *   Layout      row-major, densely packed (leading dimension = row length).
  *               Packed 4-bit data: element 2j in the LOW nibble of byte j,
  *               element 2j+1 in the high nibble.  int4 activation codes are
@@ -103,8 +107,10 @@ CQ_API cq_status cq_rotate_quantize(const void *x, int64_t M, int64_t K, int32_t
  *   centroid_sums[m,n,c] = sum over k with I[n,k] = c of q[m,k]  (if non-NULL)
  * Passage: CodeQuant2 Figure 3 (codebook + assignment matrices) and Figure 4
  * (one-time LUT precompute, then lookups).  The codebook is expanded once per
- * row tile into register-resident byte-plane tables; q is applied exactly
- * (int codes as fp16) and the sum is accumulated in fp32.  Error bound per
+ * row tile into lookup tables (register byte planes, or a byte-pair table in
+ * shared memory); M <= 16 runs on mma.sync, larger M on the tcgen05 kernel
+ * with the looked-up weights in tensor memory as the MMA's A operand.  q is
+ * applied exactly (int codes as fp16) and the sum is accumulated in fp32.  Error bound per
  * output: |y - y_exact| <= 1e-4 * |s_x[m]| * sum_k |C[n,I[n,k]] q[m,k]| + 1e-6.
  *
  * q          codes as written by cq_rotate_quantize (act_bits 4: uint8 [M, K/2];
