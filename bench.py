@@ -146,11 +146,12 @@ def lut_roofline(launch_alg, timed, steps, ms_step, peak_gbs, peak_tf, peak_kind
         e[3] += 1
     kern = max(per, key=lambda k: per[k][2])
     b, f, ms, n = per[kern]
-    src = {"k_lut_mma": "kernels_lut.cu", "k_lut_tc": "kernels_lut_tc.cu"}[kern]
+    src = {"k_lut_mma": "kernels_lut.cu", "k_lut_tc": "kernels_lut_tc.cu",
+           "k_lut_ts": "lut_ts.cuh"}[kern]
     common = {"kernel": kern, "avg_launch_us": 1e3 * ms / n, "launches_timed": n,
               "share_of_step": (ms / steps) / ms_step,
               "kernels_timed": {k: {"launches": v[3], "ms": v[2]} for k, v in per.items()}}
-    if kern == "k_lut_mma":
+    if kern in ("k_lut_mma", "k_lut_ts"):
         a = b / (ms / 1e3) / 1e9
         return {"bound": "hbm", "achieved": a, "peak": peak_gbs, "unit": "GB/s",
                 "frac": a / peak_gbs, "peak_source": f"{peak_kind} hbm_gbs",

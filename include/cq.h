@@ -274,7 +274,8 @@ CQ_API cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *ro
  */
 enum cq_kernel_kind {
     CQ_KERNEL_LUT_MMA = 0, /* mma.sync kernel, register / shared lookup tables */
-    CQ_KERNEL_LUT_TC = 1   /* tcgen05 kernel, looked-up weights in tensor memory */
+    CQ_KERNEL_LUT_TC = 1,  /* tcgen05 kernel for wide token tiles (> 32 rows per group) */
+    CQ_KERNEL_LUT_TS = 2   /* tcgen05 decode kernel (<= 32 rows per group): pair tables */
 };
 CQ_API int64_t cq_launch_count(void);
 

@@ -119,7 +119,7 @@ def cq_selftest_wait_timeout(stream=None) -> None:
     _check(lib.cq_selftest_wait_timeout(_stream(stream)), "cq_selftest_wait_timeout")
 
 
-KERNEL_KINDS = {0: "k_lut_mma", 1: "k_lut_tc"}   # cq_kernel_kind
+KERNEL_KINDS = {0: "k_lut_mma", 1: "k_lut_tc", 2: "k_lut_ts"}   # cq_kernel_kind
 
 
 def cq_timing_read_launches(cap: int = 1 << 16) -> list[tuple[str, float]]:

@@ -20,29 +20,40 @@ int ilog2(int64_t v) {
     return l;
 }
 cq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA; }
-size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 int64_t code_bytes(int64_t K, int bits) { return bits == 4 ? K / 2 : K; }
 
 // ------------------------------------------------------------------ LUT GEMM plan
-struct LutGemmPlan {
-    LutPlan p;
-    int tiles;
-    size_t ws;
-    size_t b_off;  // tensor-core path: fp16 activations at workspace + b_off
-};
+// (plan_gemm / run_lut_gemm are shared with the no-allocation entry point)
 
-// Tensor-core (tcgen05) kernel for groups of more than 16 rows, mma.sync
-// with register tables for decode-sized groups.  rows = typical rows per group.
-bool use_tc(int64_t rows, int64_t N, bool dual) {
-    if (dual ? N % 64 : N % 128) return false;  // 128 weight rows per tile
-    const LutPath p = lut_path();
-    if (p != kPathAuto) return p == kPathTc;
-    return rows > 16;
+}  // namespace
+
+namespace cq {
+
+// Which LUT GEMM kernel serves groups of `rows` typical rows: the tensor-memory
+// kernels need whole 128-row weight tiles (64 output columns for gate||up);
+// groups of at most 32 rows run on the decode kernel, wider ones on the
+// wide-token-tile kernel; other shapes on mma.sync.
+LutKernel pick_kernel(int64_t rows, int64_t N, bool dual) {
+    if (dual ? N % 64 : N % kTcTileRows) return kKernMma;
+    switch (lut_path()) {
+    case kPathMma: return kKernMma;
+    case kPathTc: return kKernTc;
+    default: break;
+    }
+    return rows <= 32 ? kKernTs : kKernTc;
 }
 
 LutGemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
-    LutGemmPlan g;
-    if (use_tc(M, N, false)) {
+    LutGemmPlan g{};
+    const LutKernel k = pick_kernel(M, N, false);
+    if (k == kKernTs) {
+        const int ntok = ts_ntok_for((int)M);
+        g.tiles = (int)((M + ntok - 1) / ntok);
+        g.p = plan_lut_ts((int)N, (int)K, false, (int)M, g.tiles, (int)M, 1);
+        g.ws = align256((size_t)g.p.splits * M * N * sizeof(float));
+        return g;
+    }
+    if (k == kKernTc) {
         const int mr = (int)std::min<int64_t>(M, 256);
         const int ntok = tc_ntok_for(mr);
         g.tiles = (int)((M + ntok - 1) / ntok);
@@ -59,11 +70,53 @@ LutGemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
     return g;
 }
 
+cudaError_t run_lut_gemm(const LutGemmPlan &g, const void *q, const float *s_x, int64_t M,
+                         int64_t K, int act_bits, const uint8_t *w_idx, const void *codebook,
+                         int64_t N, float *y, void *scratch, cudaStream_t st) {
+    LutLaunch L{};
+    L.codes = reinterpret_cast<const uint8_t *>(q);
+    L.ld_codes = act_bits == 4 ? K / 2 : K;
+    L.scales = s_x;
+    L.act_bits = act_bits;
+    L.K = (int)K;
+    L.map_mode = kMapIdentity;
+    L.G = 1;
+    L.uniform_rows = (int)M;
+    L.max_tiles = g.tiles;
+    L.idx0 = w_idx;
+    L.cb0 = codebook;
+    L.w_stride = 0;
+    L.cb_stride = 0;
+    L.N = (int)N;
+    L.dual = false;
+    L.out_row_stride = N;
+    L.direct = false;
+    L.out = reinterpret_cast<float *>(scratch);
+    L.out_split_stride = M * N;
+    cudaError_t e;
+    if (g.p.tc == 2) {
+        e = launch_lut_ts(L, g.p, st);
+    } else if (g.p.tc == 1) {
+        void *b = reinterpret_cast<uint8_t *>(scratch) + g.b_off;
+        e = launch_codes_to_f16(q, L.ld_codes, act_bits, (int)K, M, kMapIdentity, nullptr, 1, 1,
+                                b, st);
+        if (e == cudaSuccess) e = launch_lut_tc(L, g.p, b, M, 0, st);
+    } else {
+        e = launch_lut(L, g.p, st);
+    }
+    if (e == cudaSuccess) e = launch_reduce_plain(L.out, g.p, M, N, s_x, y, st);
+    return e;
+}
+
+}  // namespace cq
+
+namespace {
+
 // ------------------------------------------------------------------ MoE plan
 struct MoePlan {
     int64_t T, H, I, E, k, ns, Is, Rr, Rs, R;
     int bits, Imax, nt, tile_rows, max_tiles_r, tiles_s, tile_rows_s;
-    bool tc_r, tc_s, tc_dn_r, tc_dn_s;  // tensor-core kernel per launch
+    LutKernel k_r, k_s;                 // kernel of the routed / shared launches
     bool fused;                         // gate/up launches write h (SwiGLU in their epilogue)
     LutPlan gu_r, gu_s, dn_r, dn_s;
     size_t o_xq, o_sx, o_ids, o_w, o_counts, o_offsets, o_perm, o_inv, o_tiles, o_tgrp;
@@ -89,48 +142,48 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
     m.bits = d->act_bits;
     m.Imax = (int)std::max<int64_t>(m.E > 0 ? m.I : 0, m.Is);
     m.nt = T <= 8 ? 1 : 2;
-    // routed experts: typical rows per expert decide the kernel and tile size
+    // routed experts: typical rows per expert decide the kernel and tile size;
+    // gate||up and down share one token tiling per group (the routing tables)
     const int64_t avg_r = m.E > 0 ? (m.Rr + m.E - 1) / m.E : 0;
-    m.tc_r = m.E > 0 && use_tc(avg_r, m.I, true);
-    m.tc_dn_r = m.tc_r && use_tc(avg_r, m.H, false);
-    if (m.tc_r != m.tc_dn_r) m.tc_r = m.tc_dn_r = false;  // one token tiling per group
     const int rows_r = (int)std::min<int64_t>(T, std::max<int64_t>(2 * avg_r, 1));
-    m.tile_rows = m.tc_r ? tc_ntok_for(rows_r) : 8 * m.nt;
+    if (m.E > 0) {
+        m.k_r = pick_kernel(rows_r, m.I, true);
+        if (pick_kernel(rows_r, m.H, false) != m.k_r) m.k_r = kKernMma;
+    }
+    m.tile_rows = m.k_r == kKernTs ? ts_ntok_for(rows_r)
+                : m.k_r == kKernTc ? tc_ntok_for(rows_r) : 8 * m.nt;
     const int64_t nonempty = std::min<int64_t>(m.E, m.Rr);
     m.max_tiles_r = (int)(m.Rr / m.tile_rows + nonempty);
     // shared experts: every token
-    m.tc_s = m.ns > 0 && use_tc(T, m.Is, true);
-    m.tc_dn_s = m.ns > 0 && use_tc(T, m.H, false);
-    if (m.tc_s != m.tc_dn_s) m.tc_s = m.tc_dn_s = false;
-    m.tile_rows_s = m.tc_s ? tc_ntok_for((int)std::min<int64_t>(T, 256)) : 8 * m.nt;
+    const int rows_s = (int)std::min<int64_t>(T, 256);
+    if (m.ns > 0) {
+        m.k_s = pick_kernel(rows_s, m.Is, true);
+        if (pick_kernel(rows_s, m.H, false) != m.k_s) m.k_s = kKernMma;
+    }
+    m.tile_rows_s = m.k_s == kKernTs ? ts_ntok_for(rows_s)
+                  : m.k_s == kKernTc ? tc_ntok_for(rows_s) : 8 * m.nt;
     m.tiles_s = (int)(m.ns * ((T + m.tile_rows_s - 1) / m.tile_rows_s));
     const int rows_per_group = (int)std::min<int64_t>(T, 16);
+    auto plan_for = [&](LutKernel k, int N, int K, bool dual, int tile_rows, int64_t tiles,
+                        int uniform_rows, int n_groups) {
+        if (k == kKernTs) return plan_lut_ts(N, K, dual, tile_rows, tiles, uniform_rows, n_groups);
+        if (k == kKernTc) return plan_lut_tc(N, K, dual, tile_rows, tiles, uniform_rows, n_groups);
+        return plan_lut(N, K, dual, rows_per_group, tiles, uniform_rows, n_groups);
+    };
     if (m.E > 0) {
-        if (m.tc_r) {
-            m.gu_r = plan_lut_tc((int)m.I, (int)m.H, true, m.tile_rows, m.max_tiles_r);
-            m.dn_r = plan_lut_tc((int)m.H, (int)m.I, false, m.tile_rows, m.max_tiles_r);
-        } else {
-            m.gu_r = plan_lut((int)m.I, (int)m.H, true, rows_per_group, m.max_tiles_r);
-            m.dn_r = plan_lut((int)m.H, (int)m.I, false, rows_per_group, m.max_tiles_r);
-        }
+        m.gu_r = plan_for(m.k_r, (int)m.I, (int)m.H, true, m.tile_rows, m.max_tiles_r, 0, 1);
+        m.dn_r = plan_for(m.k_r, (int)m.H, (int)m.I, false, m.tile_rows, m.max_tiles_r, 0, 1);
     }
     if (m.ns > 0) {
-        if (m.tc_s) {
-            m.gu_s = plan_lut_tc((int)m.Is, (int)m.H, true, m.tile_rows_s, m.tiles_s, (int)T,
-                                 (int)m.ns);
-            m.dn_s = plan_lut_tc((int)m.H, (int)m.Is, false, m.tile_rows_s, m.tiles_s, (int)T,
-                                 (int)m.ns);
-        } else {
-            m.gu_s = plan_lut((int)m.Is, (int)m.H, true, rows_per_group, m.tiles_s, (int)T,
-                              (int)m.ns);
-            m.dn_s = plan_lut((int)m.H, (int)m.Is, false, rows_per_group, m.tiles_s, (int)T,
-                              (int)m.ns);
-        }
+        m.gu_s = plan_for(m.k_s, (int)m.Is, (int)m.H, true, m.tile_rows_s, m.tiles_s, (int)T,
+                          (int)m.ns);
+        m.dn_s = plan_for(m.k_s, (int)m.H, (int)m.Is, false, m.tile_rows_s, m.tiles_s, (int)T,
+                          (int)m.ns);
     }
     // SwiGLU moves into the gate/up epilogue when every gate/up launch runs on
     // the tensor-core kernel with a single partial slot per output
-    m.fused = (m.E == 0 || (m.tc_r && !m.gu_r.streamk && m.gu_r.splits == 1)) &&
-              (m.ns == 0 || (m.tc_s && !m.gu_s.streamk && m.gu_s.splits == 1));
+    m.fused = (m.E == 0 || (m.k_r == kKernTc && !m.gu_r.streamk && m.gu_r.splits == 1)) &&
+              (m.ns == 0 || (m.k_s == kKernTc && !m.gu_s.streamk && m.gu_s.splits == 1));
     size_t o = 0;
     auto take = [&](size_t bytes) {
         const size_t at = o;
@@ -155,10 +208,11 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
     m.o_sh = take((size_t)m.R * 4);
     m.o_pdn_r = take(m.E > 0 ? (size_t)m.dn_r.splits * m.Rr * m.H * 4 : 0);
     m.o_pdn_s = take(m.ns > 0 ? (size_t)m.dn_s.splits * m.Rs * m.H * 4 : 0);
-    m.o_bx_r = take(m.tc_r ? (size_t)m.Rr * m.H * 2 : 0);
-    m.o_bx_s = take(m.tc_s ? (size_t)T * m.H * 2 : 0);
-    m.o_bh_r = take(m.tc_r ? (size_t)m.Rr * m.I * 2 : 0);
-    m.o_bh_s = take(m.tc_s ? (size_t)m.Rs * m.Is * 2 : 0);
+    const bool wide_r = m.k_r == kKernTc, wide_s = m.k_s == kKernTc;
+    m.o_bx_r = take(wide_r ? (size_t)m.Rr * m.H * 2 : 0);
+    m.o_bx_s = take(wide_s ? (size_t)T * m.H * 2 : 0);
+    m.o_bh_r = take(wide_r ? (size_t)m.Rr * m.I * 2 : 0);
+    m.o_bh_s = take(wide_s ? (size_t)m.Rs * m.Is * 2 : 0);
     m.total = o;
     return m;
 }
@@ -246,36 +300,7 @@ cq_status cq_lut_gemm(const void *q, const float *s_x, int64_t M, int64_t K, int
     const LutGemmPlan g = plan_gemm(M, N, K);
     if (g.ws > 0 && (!workspace || workspace_bytes < g.ws)) return CQ_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    LutLaunch L{};
-    L.codes = reinterpret_cast<const uint8_t *>(q);
-    L.ld_codes = code_bytes(K, act_bits);
-    L.scales = s_x;
-    L.act_bits = act_bits;
-    L.K = (int)K;
-    L.map_mode = kMapIdentity;
-    L.G = 1;
-    L.uniform_rows = (int)M;
-    L.max_tiles = g.tiles;
-    L.idx0 = w_idx;
-    L.cb0 = codebook;
-    L.w_stride = 0;
-    L.cb_stride = 0;
-    L.N = (int)N;
-    L.dual = false;
-    L.out_row_stride = N;
-    L.direct = false;
-    L.out = reinterpret_cast<float *>(workspace);
-    L.out_split_stride = M * N;
-    cudaError_t e;
-    if (g.p.tc) {
-        void *b = reinterpret_cast<uint8_t *>(workspace) + g.b_off;
-        e = launch_codes_to_f16(q, code_bytes(K, act_bits), act_bits, (int)K, M, kMapIdentity,
-                                nullptr, 1, 1, b, st);
-        if (e == cudaSuccess) e = launch_lut_tc(L, g.p, b, M, 0, st);
-    } else {
-        e = launch_lut(L, g.p, st);
-    }
-    if (e == cudaSuccess) e = launch_reduce_plain(L.out, g.p, M, N, s_x, y, st);
+    cudaError_t e = run_lut_gemm(g, q, s_x, M, K, act_bits, w_idx, codebook, N, y, workspace, st);
     if (e == cudaSuccess && centroid_sums)
         e = launch_centroid_sums(q, M, K, act_bits, w_idx, N, centroid_sums, st);
     return cuda_status(e);
@@ -358,7 +383,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
             L.h_out = hf;
             L.h_row_stride = m.Imax;
         }
-        if (m.tc_r) {
+        if (m.k_r == kKernTs) {
+            e = launch_lut_ts(L, m.gu_r, st);
+        } else if (m.k_r == kKernTc) {
             void *b = ws + m.o_bx_r;
             e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, m.Rr, kMapPerm, perm, (int)m.k,
                                     (int)T, b, st, m.fused ? sx : nullptr, rsc);
@@ -380,7 +407,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
             L.h_out = hf + m.Rr * m.Imax;
             L.h_row_stride = m.Imax;
         }
-        if (m.tc_s) {
+        if (m.k_s == kKernTs) {
+            e = launch_lut_ts(L, m.gu_s, st);
+        } else if (m.k_s == kKernTc) {
             void *b = ws + m.o_bx_s;
             e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, T, kMapIdentity, nullptr, 1,
                                     (int)T, b, st);
@@ -423,7 +452,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.idx0 = w->down_idx; L.cb0 = w->down_cb;
         L.w_stride = m.H * (m.I / 2); L.cb_stride = m.H * 16; L.N = (int)m.H; L.dual = false;
         L.out = pdn_r; L.out_split_stride = m.Rr * m.H; L.out_row_stride = m.H;
-        if (m.tc_dn_r) {
+        if (m.k_r == kKernTs) {
+            e = launch_lut_ts(L, m.dn_r, st);
+        } else if (m.k_r == kKernTc) {
             void *b = ws + m.o_bh_r;
             e = launch_codes_to_f16(hq, ldh, m.bits, (int)m.I, m.Rr, kMapIdentity, nullptr, 1, 1,
                                     b, st);
@@ -440,7 +471,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.idx0 = w->sh_down_idx; L.cb0 = w->sh_down_cb;
         L.w_stride = m.H * (m.Is / 2); L.cb_stride = m.H * 16; L.N = (int)m.H; L.dual = false;
         L.out = pdn_s; L.out_split_stride = m.Rs * m.H; L.out_row_stride = m.H;
-        if (m.tc_dn_s) {
+        if (m.k_s == kKernTs) {
+            e = launch_lut_ts(L, m.dn_s, st);
+        } else if (m.k_s == kKernTc) {
             void *b = ws + m.o_bh_s;
             e = launch_codes_to_f16(hq + m.Rr * ldh, ldh, m.bits, (int)m.Is, m.Rs, kMapIdentity,
                                     nullptr, 1, 1, b, st);

@@ -88,7 +88,8 @@ struct LutPlan {
     int chunks_per_split;
     int64_t units;      // stream-K: total units (work items * C)
     int uniform_rows;   // rows per group of a uniform launch (token tiles of a group are consecutive)
-    int tc;             // 1: tensor-memory kernel (64-k chunks, 128-row tiles)
+    int tc;             // 0: mma.sync kernel; 1: tensor-memory kernel (wide token
+                        // tiles); 2: tensor-memory decode kernel (64-k chunks, 128-row tiles)
     size_t smem;
 };
 
@@ -125,6 +126,28 @@ LutPlan plan_lut(int N, int K, bool dual, int max_rows_per_group, int64_t est_ti
                  int uniform_rows = 0, int n_groups = 1);
 cudaError_t launch_lut(const LutLaunch &L, const LutPlan &P, cudaStream_t st);
 
+// The LUT GEMM kernels and which one serves a launch.
+enum LutKernel : int { kKernMma = 0, kKernTc = 1, kKernTs = 2 };
+constexpr int kTcTileRows = 128;  // weight rows per tensor-memory tile
+LutKernel pick_kernel(int64_t rows, int64_t N, bool dual);
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// A planned cq_lut_gemm call: the launch plan, the token tiles, the scratch
+// it needs (split-K partial sums, then for the wide-tile kernel fp16 codes at
+// b_off) and its launches.  Shared by the workspace and no-allocation entry
+// points, so both run exactly the same kernels with the same partition.
+struct LutGemmPlan {
+    LutPlan p;
+    int tiles;
+    size_t ws;
+    size_t b_off;
+};
+LutGemmPlan plan_gemm(int64_t M, int64_t N, int64_t K);
+cudaError_t run_lut_gemm(const LutGemmPlan &g, const void *q, const float *s_x, int64_t M,
+                         int64_t K, int act_bits, const uint8_t *w_idx, const void *codebook,
+                         int64_t N, float *y, void *scratch, cudaStream_t st);
+
 // Tensor-memory (tcgen05) LUT GEMM.  The activations are read as fp16 rows
 // b_f16 [b_rows][K]; the GEMM row p of a token tile maps to B row
 // (b_row_mod > 0 ? p % b_row_mod : p).
@@ -133,6 +156,13 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
                     int uniform_rows = 0, int n_groups = 1);
 cudaError_t launch_lut_tc(const LutLaunch &L, const LutPlan &P, const void *b_f16, int64_t b_rows,
                           int b_row_mod, cudaStream_t st);
+// Tensor-memory decode kernel (groups of at most 32 rows): thread-per-row pair
+// tables, index bytes by TMA, B tiles converted from the int codes in-kernel
+// (rows mapped like LutLaunch::map_mode), so it needs no fp16 copy.
+int ts_ntok_for(int max_rows_per_group);
+LutPlan plan_lut_ts(int N, int K, bool dual, int max_rows_per_group, int64_t est_tiles,
+                    int uniform_rows = 0, int n_groups = 1);
+cudaError_t launch_lut_ts(const LutLaunch &L, const LutPlan &P, cudaStream_t st);
 // fp16 copies of activation codes (B operand), rows mapped like LutLaunch::map_mode.
 // scales_in != nullptr: also writes scales_out[p] = scales_in[code row of p].
 cudaError_t launch_codes_to_f16(const void *codes, int64_t ld_codes, int bits, int K,
@@ -145,7 +175,7 @@ cudaError_t launch_selftest_wait(cudaStream_t st);
 int read_device_error();
 // Which LUT kernel a launch uses: "mma" (mma.sync, register tables), "tc"
 // (tcgen05 / tensor memory), or automatic (default).
-enum LutPath : int { kPathAuto = 0, kPathMma = 1, kPathTc = 2 };
+enum LutPath : int { kPathAuto = 0, kPathMma = 1, kPathTc = 2, kPathTs = 3 };
 LutPath lut_path();
 
 // y[m, n] = s[m] * sum_{s < n(m, n)} part[s][m][n]

@@ -44,6 +44,8 @@
 #include "cq_internal.h"
 #include "lut_lookup.cuh"
 #include "sm100.cuh"
+#include "tc_walk.cuh"
+#include "lut_ts.cuh"
 
 namespace cq {
 
@@ -52,9 +54,6 @@ constexpr int kTcExpand = kTcExpandWarps * 32;
 constexpr int kWarpMma = 8;          // TMEM allocation + MMA issue (lane 0)
 constexpr int kWarpTma = 9;          // B tile loads (lane 0)
 constexpr int kTcThreads = 320;
-constexpr int kTcRows = 128;         // rows per tile (TMEM lanes)
-constexpr int kTcChunk = 64;         // k per chunk: one B tile, 4 MMAs, 32 TMEM columns
-constexpr int kTcG = 4;              // chunks per group: the expand / A-ring unit (256 k)
 constexpr int kTcA = 2;              // A ring depth in groups (TMEM columns [0, 256))
 // B ring (shared memory, NTOK x 128 B per chunk tile): kTcB stages of kBG
 // chunk tiles; a stage is freed by the commit of the MMAs that read it.
@@ -68,130 +67,6 @@ template <int NTOK> struct TcBG { static constexpr int n = NTOK <= 64 ? kTcG : 1
 template <int NTOK> struct TcAcc { static constexpr int n = NTOK <= 32 ? 4 : 1; };
 constexpr int kTcWStages = 4;        // index-byte ring per thread, in groups (3 in flight)
 constexpr size_t kPairTableBytes = 256 * kTcRows * 4;  // 128 KB
-
-struct TcSchedule {
-    const LutLaunch *L;
-    const LutPlan *P;
-    // work item -> (group, first row, rows, row tile)
-    CQ_DEV void item(int64_t w, int &g, int &row0, int &nrows, int &rt) const {
-        const int TT = 8 * P->nt;
-        const int64_t tile = w / P->n_row_tiles;
-        rt = (int)(w - tile * P->n_row_tiles);
-        if (L->uniform_rows > 0) {
-            const int tpg = (L->uniform_rows + TT - 1) / TT;
-            g = (int)(tile / tpg);
-            row0 = g * L->uniform_rows + (int)(tile - (int64_t)g * tpg) * TT;
-            nrows = min(TT, (g + 1) * L->uniform_rows - row0);
-        } else {
-            if (tile >= L->grp_tiles[L->G]) {
-                g = -1;
-                row0 = nrows = 0;
-                return;
-            }
-            g = L->tile_grp[tile];
-            row0 = L->grp_rows[g] + (int)(tile - L->grp_tiles[g]) * TT;
-            nrows = min(TT, L->grp_rows[g + 1] - row0);
-        }
-    }
-    // this thread's weight row: index bytes and codebook (t = 0..127)
-    CQ_DEV void row_ptrs(int g, int rt, int t, const uint8_t *&idx, const __half *&cb, int &col) const {
-        const int64_t rowbytes = L->K / 2;
-        if (L->dual) {
-            // gate and up rows of one output column in adjacent lanes, so the
-            // epilogue's stores of a warp cover 32 consecutive partial columns
-            const int n = rt * 64 + (t >> 1);
-            const bool up = t & 1;
-            idx = (up ? L->idx1 : L->idx0) + (int64_t)g * L->w_stride + (int64_t)n * rowbytes;
-            cb = reinterpret_cast<const __half *>(up ? L->cb1 : L->cb0) + (int64_t)g * L->cb_stride + n * 16;
-            col = 2 * n + (up ? 1 : 0);
-        } else {
-            const int n = rt * kTcRows + t;
-            idx = L->idx0 + (int64_t)g * L->w_stride + (int64_t)n * rowbytes;
-            cb = reinterpret_cast<const __half *>(L->cb0) + (int64_t)g * L->cb_stride + n * 16;
-            col = n;
-        }
-    }
-};
-
-// The chunks a CTA works through, as segments (work item, chunk range) cut
-// into groups of at most kTcG chunks (a group never spans two segments).
-// Stream-K (uniform launches): one contiguous range of units (item x chunk),
-// cut at item boundaries.  Fixed split (routed launches): pieces (item,
-// split) p = blockIdx.x, blockIdx.x + gridDim.x, ... below the number of
-// pieces the routing produced, so the grid stays one CTA per SM whatever the
-// tile count.  Every role of the CTA walks the same sequence.
-struct TcWalk {
-    const LutPlan *P;
-    int64_t w;        // work item of the current segment
-    int c0, gn;       // first chunk (item-relative) and chunk count of the group
-    int c_begin, c_end;
-    int slot;         // partial-sum slot the segment writes
-    int64_t nxt, lim;
-    bool valid;
-
-    CQ_DEV void init(const LutPlan &Pl, int64_t n_pieces) {
-        P = &Pl;
-        if (Pl.streamk) {
-            nxt = (int64_t)blockIdx.x * Pl.units / Pl.grid;
-            lim = ((int64_t)blockIdx.x + 1) * Pl.units / Pl.grid;
-        } else {
-            nxt = blockIdx.x;
-            lim = n_pieces;
-        }
-        load();
-    }
-    CQ_DEV void load() {
-        valid = nxt < lim;
-        if (!valid) return;
-        const int C = P->chunks_total;
-        if (P->streamk) {
-            w = nxt / C;
-            c_begin = (int)(nxt - w * C);
-            const int64_t e = min(lim, (w + 1) * C);
-            c_end = (int)(e - w * C);
-            slot = (int)(blockIdx.x - lut_cta_of_unit(*P, w * C));
-            nxt = e;
-        } else {
-            w = nxt / P->splits;
-            const int sp = (int)(nxt - w * P->splits);
-            c_begin = sp * P->chunks_per_split;
-            c_end = min(C, c_begin + P->chunks_per_split);
-            slot = sp;
-            nxt += gridDim.x;
-        }
-        c0 = c_begin;
-        gn = min(kTcG, c_end - c0);
-    }
-    CQ_DEV bool seg_first() const { return c0 == c_begin; }
-    CQ_DEV bool seg_last() const { return c0 + gn == c_end; }
-    CQ_DEV void next() {
-        c0 += gn;
-        if (c0 >= c_end) load();
-        else gn = min(kTcG, c_end - c0);
-    }
-};
-
-// Pieces of a fixed-split launch that hold rows (the routing decides how many
-// token tiles there are; the host only knows an upper bound).
-CQ_DEV int64_t tc_pieces(const LutLaunch &L, const LutPlan &P) {
-    if (P.streamk) return 0;
-    const int TT = 8 * P.nt;
-    const int64_t tiles = L.uniform_rows > 0
-                              ? (int64_t)L.G * ((L.uniform_rows + TT - 1) / TT)
-                              : min((int64_t)L.grp_tiles[L.G], (int64_t)L.max_tiles);
-    return tiles * P.n_row_tiles * P.splits;
-}
-
-// Activation scale of output row p (the row's token).
-// Issued as a volatile load at segment start, so the compiler cannot sink it to
-// the epilogue, where it would stall the drain of the accumulator.
-CQ_DEV float tc_row_scale(const LutLaunch &L, int64_t p) {
-    const float *src = L.row_scales ? L.row_scales + p
-                     : L.scales + (L.map_mode == kMapModT ? p % L.T : p);
-    float v;
-    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(src));
-    return v;
-}
 
 template <int NTOK, bool PAIR>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -689,6 +564,91 @@ cudaError_t launch_lut_tc(const LutLaunch &L, const LutPlan &P, const void *b_f1
     return e;
 }
 
+// ---------------------------------------------------------------- decode kernel (lut_ts.cuh)
+// Tensor map over packed index bytes uint8 [rows][K/2] (row stride K/2), box
+// [box_rows rows][128 B] (one 256-k group), 128-byte swizzle; bytes past K/2
+// read as zero.
+static bool make_idx_map(CUtensorMap *m, const void *base, int64_t rows, int K, int box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int ts_ntok_for(int max_rows_per_group) { return max_rows_per_group <= 16 ? 16 : 32; }
+
+LutPlan plan_lut_ts(int N, int K, bool dual, int max_rows_per_group, int64_t est_tiles,
+                    int uniform_rows, int n_groups) {
+    LutPlan P{};
+    const int ntok = ts_ntok_for(max_rows_per_group);
+    P.nt = ntok / 8;
+    P.rows_per_rt = dual ? 64 : kTcRows;
+    P.n_row_tiles = N / P.rows_per_rt;
+    P.chunks_total = (K + kTcChunk - 1) / kTcChunk;
+    P.cps_max = P.chunks_total;
+    const int capacity = sm_count();  // one CTA per SM
+    const int C = P.chunks_total;
+    P.uniform_rows = uniform_rows;
+    if (uniform_rows > 0) {
+        // stream-K: every SM gets the same number of chunks
+        const int64_t tiles = (int64_t)n_groups * ((uniform_rows + ntok - 1) / ntok);
+        P.streamk = 1;
+        P.units = tiles * P.n_row_tiles * C;
+        P.grid = (int)std::min<int64_t>(capacity, P.units);
+        int smax = 1;
+        const int64_t items = tiles * P.n_row_tiles;
+        for (int64_t w = 0; w < items; w++) smax = std::max(smax, lut_item_splits(P, w));
+        P.splits = smax;
+        P.chunks_per_split = C;
+    } else {
+        // routed groups: whole (item, split) pieces strided over the CTAs,
+        // split-K only when there are fewer items than SMs
+        P.streamk = 0;
+        const int64_t base = (int64_t)P.n_row_tiles * std::max<int64_t>(est_tiles, 1);
+        int splits = base < capacity ? (int)(capacity / base) : 1;
+        splits = std::max(1, std::min(splits, C));
+        P.chunks_per_split = (C + splits - 1) / splits;
+        P.splits = (C + P.chunks_per_split - 1) / P.chunks_per_split;
+        P.grid = (int)std::min<int64_t>(capacity, base * P.splits);
+    }
+    P.smem = ntok == 16 ? TsShape<16>::smem : TsShape<32>::smem;
+    P.tc = 2;
+    return P;
+}
+
+template <int NTOK>
+static cudaError_t launch_ts_t(const CUtensorMap &m0, const CUtensorMap &m1, const LutLaunch &L,
+                               const LutPlan &P, cudaStream_t st) {
+    cudaFuncSetAttribute(k_lut_ts<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)P.smem);
+    return launch_pdl(k_lut_ts<NTOK>, dim3(P.grid), dim3(TsShape<NTOK>::threads), P.smem, st, 1,
+                      m0, m1, L, P);
+}
+
+cudaError_t launch_lut_ts(const LutLaunch &L, const LutPlan &P, cudaStream_t st) {
+    if (P.grid == 0 || (!P.streamk && L.max_tiles == 0)) return cudaSuccess;
+    const int64_t rows = (int64_t)std::max(L.G, 1) * L.N;
+    const int box = L.dual ? 64 : kTcRows;
+    CUtensorMap m0, m1;
+    std::memset(&m0, 0, sizeof(m0));
+    std::memset(&m1, 0, sizeof(m1));
+    if (!make_idx_map(&m0, L.idx0, rows, L.K, box)) return cudaErrorInvalidValue;
+    if (L.dual && !make_idx_map(&m1, L.idx1, rows, L.K, box)) return cudaErrorInvalidValue;
+    const bool timed = timing_on();
+    if (timed) timing_begin(st, CQ_KERNEL_LUT_TS);
+    count_launch();
+    const cudaError_t e = P.nt == 2 ? launch_ts_t<16>(m0, L.dual ? m1 : m0, L, P, st)
+                                    : launch_ts_t<32>(m0, L.dual ? m1 : m0, L, P, st);
+    if (timed) timing_end(st);
+    return e;
+}
+
 // ---------------------------------------------------------------- codes -> fp16 rows
 // out[p, k] = fp16(code of row map(p), position k): the B operand of the
 // tensor-core kernel.  One thread per 8 codes.
@@ -739,6 +699,7 @@ LutPath lut_path() {
         const char *e = getenv("CQ_LUT_PATH");
         if (e && !strcmp(e, "mma")) return kPathMma;
         if (e && !strcmp(e, "tc")) return kPathTc;
+        if (e && !strcmp(e, "ts")) return kPathTs;
         return kPathAuto;
     }();
     return p;
@@ -773,3 +734,10 @@ int read_device_error() {
 }
 
 }  // namespace cq
+
+#ifdef CQ_TS_TRACE
+// Copies the decode kernel's timeline stamps to host memory (tuning builds only).
+extern "C" CQ_API int cq_ts_trace_read(void *dst, size_t bytes) {
+    return cudaMemcpyFromSymbol(dst, cq::g_ts_trace, bytes) == cudaSuccess ? 0 : 1;
+}
+#endif

@@ -72,37 +72,13 @@ extern "C" CQ_API cq_status cq_lut_gemm_noalloc(const void *q, const float *s_x,
         return CQ_ERR_UNSUPPORTED;
     if (M == 0) return CQ_OK;
 
-    // the mma.sync kernel with the plan cq_lut_gemm uses for it (M <= 16)
-    const int nt = M <= 8 ? 1 : 2;
-    const int tiles = (int)((M + 8 * nt - 1) / (8 * nt));
-    const LutPlan P = plan_lut((int)N, (int)K, false, (int)std::min<int64_t>(M, 16), tiles,
-                               (int)M, 1);
-    const size_t need = (size_t)P.splits * M * N * sizeof(float);
-    if (need > kNoAllocScratchBytes) return CQ_ERR_UNSUPPORTED;  // beyond the fixed scratch
+    // exactly the plan and kernels of cq_lut_gemm, with the scratch in the array
+    const LutGemmPlan g = plan_gemm(M, N, K);
+    if (g.ws > kNoAllocScratchBytes) return CQ_ERR_UNSUPPORTED;  // beyond the fixed scratch
 
     void *p = nullptr;
     if (scratch_on_current_device(&p) != cudaSuccess) return CQ_ERR_CUDA;
-    float *scratch = reinterpret_cast<float *>(p);
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    LutLaunch L{};
-    L.codes = reinterpret_cast<const uint8_t *>(q);
-    L.ld_codes = act_bits == 4 ? K / 2 : K;
-    L.scales = s_x;
-    L.act_bits = act_bits;
-    L.K = (int)K;
-    L.map_mode = kMapIdentity;
-    L.G = 1;
-    L.uniform_rows = (int)M;
-    L.max_tiles = tiles;
-    L.idx0 = w_idx;
-    L.cb0 = codebook;
-    L.N = (int)N;
-    L.dual = false;
-    L.out_row_stride = N;
-    L.direct = false;
-    L.out = scratch;
-    L.out_split_stride = M * N;
-    cudaError_t e = launch_lut(L, P, st);
-    if (e == cudaSuccess) e = launch_reduce_plain(scratch, P, M, N, s_x, y, st);
+    const cudaError_t e = run_lut_gemm(g, q, s_x, M, K, act_bits, w_idx, codebook, N, y, p,
+                                       reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }

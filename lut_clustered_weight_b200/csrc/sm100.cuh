@@ -181,6 +181,24 @@ CQ_DEV void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
         : "memory");
 }
 
+// 8 / 32 consecutive 32-bit columns of this thread's TMEM lane (warp-wide).
+CQ_DEV void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7])
+        : "r"(taddr)
+        : "memory");
+}
+CQ_DEV void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[8]) { tmem_ld8(taddr, v); }
+CQ_DEV void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[16]) { tmem_ld16(taddr, v); }
+
+// Generic-proxy shared-memory writes of this thread become visible to the
+// async proxy (the tensor core reading a descriptor-addressed operand).
+CQ_DEV void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, rows of 128 B,
 // 8-row groups 1024 B apart (stride byte offset), sm_100 descriptor version 1.
 CQ_DEV uint64_t smem_desc_sw128(uint32_t saddr) {
