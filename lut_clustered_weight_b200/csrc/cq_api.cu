@@ -30,27 +30,36 @@ int64_t code_bytes(int64_t K, int bits) { return bits == 4 ? K / 2 : K; }
 namespace cq {
 
 // Which LUT GEMM kernel serves groups of `rows` typical rows: the tensor-memory
-// kernels need whole 128-row weight tiles (64 output columns for gate||up);
-// groups of at most 32 rows run on the decode kernel, wider ones on the
-// wide-token-tile kernel; other shapes on mma.sync.
-LutKernel pick_kernel(int64_t rows, int64_t N, bool dual) {
+// kernels need whole 128-row weight tiles (64 output columns for gate||up).
+// Measured on B200: uniform launches of at most 16 rows (dense decode) are as
+// fast on mma.sync and need no fp16 copy of the activations; routed groups of
+// at most 32 rows (MoE decode) are faster on the tensor-memory decode kernel;
+// wider groups run on the wide-token-tile kernel.
+LutKernel pick_kernel(int64_t rows, int64_t N, bool dual, int64_t K, int64_t tiles_bound,
+                      bool routed) {
     if (dual ? N % 64 : N % kTcTileRows) return kKernMma;
+    // the tensor-memory kernels count their work in 32 bits
+    const int64_t units = tiles_bound * (N / (dual ? 64 : kTcTileRows)) * ((K + 63) / 64);
+    if (units * sm_count() >= (int64_t(1) << 31)) return kKernMma;
     switch (lut_path()) {
     case kPathMma: return kKernMma;
     case kPathTc: return kKernTc;
+    case kPathTs: return rows <= 32 ? kKernTs : kKernTc;
     default: break;
     }
+    if (rows <= 16 && !routed) return kKernMma;
     return rows <= 32 ? kKernTs : kKernTc;
 }
 
 LutGemmPlan plan_gemm(int64_t M, int64_t N, int64_t K) {
     LutGemmPlan g{};
-    const LutKernel k = pick_kernel(M, N, false);
+    const LutKernel k = pick_kernel(M, N, false, K, (M + 15) / 16, false);
     if (k == kKernTs) {
         const int ntok = ts_ntok_for((int)M);
         g.tiles = (int)((M + ntok - 1) / ntok);
         g.p = plan_lut_ts((int)N, (int)K, false, (int)M, g.tiles, (int)M, 1);
-        g.ws = align256((size_t)g.p.splits * M * N * sizeof(float));
+        g.b_off = align256((size_t)g.p.splits * M * N * sizeof(float));
+        g.ws = g.b_off + align256((size_t)M * K * 2);
         return g;
     }
     if (k == kKernTc) {
@@ -94,13 +103,13 @@ cudaError_t run_lut_gemm(const LutGemmPlan &g, const void *q, const float *s_x, 
     L.out = reinterpret_cast<float *>(scratch);
     L.out_split_stride = M * N;
     cudaError_t e;
-    if (g.p.tc == 2) {
-        e = launch_lut_ts(L, g.p, st);
-    } else if (g.p.tc == 1) {
+    if (g.p.tc != 0) {
+        // tensor-memory kernels read the activations as fp16 rows
         void *b = reinterpret_cast<uint8_t *>(scratch) + g.b_off;
         e = launch_codes_to_f16(q, L.ld_codes, act_bits, (int)K, M, kMapIdentity, nullptr, 1, 1,
                                 b, st);
-        if (e == cudaSuccess) e = launch_lut_tc(L, g.p, b, M, 0, st);
+        if (e == cudaSuccess)
+            e = g.p.tc == 2 ? launch_lut_ts(L, g.p, b, M, 0, st) : launch_lut_tc(L, g.p, b, M, 0, st);
     } else {
         e = launch_lut(L, g.p, st);
     }
@@ -147,8 +156,9 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
     const int64_t avg_r = m.E > 0 ? (m.Rr + m.E - 1) / m.E : 0;
     const int rows_r = (int)std::min<int64_t>(T, std::max<int64_t>(2 * avg_r, 1));
     if (m.E > 0) {
-        m.k_r = pick_kernel(rows_r, m.I, true);
-        if (pick_kernel(rows_r, m.H, false) != m.k_r) m.k_r = kKernMma;
+        const int64_t tb = m.Rr / 16 + m.E;
+        m.k_r = pick_kernel(rows_r, m.I, true, m.H, tb, true);
+        if (pick_kernel(rows_r, m.H, false, m.I, tb, true) != m.k_r) m.k_r = kKernMma;
     }
     m.tile_rows = m.k_r == kKernTs ? ts_ntok_for(rows_r)
                 : m.k_r == kKernTc ? tc_ntok_for(rows_r) : 8 * m.nt;
@@ -157,8 +167,9 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
     // shared experts: every token
     const int rows_s = (int)std::min<int64_t>(T, 256);
     if (m.ns > 0) {
-        m.k_s = pick_kernel(rows_s, m.Is, true);
-        if (pick_kernel(rows_s, m.H, false) != m.k_s) m.k_s = kKernMma;
+        const int64_t tb = m.ns * ((T + 15) / 16);
+        m.k_s = pick_kernel(rows_s, m.Is, true, m.H, tb, false);
+        if (pick_kernel(rows_s, m.H, false, m.Is, tb, false) != m.k_s) m.k_s = kKernMma;
     }
     m.tile_rows_s = m.k_s == kKernTs ? ts_ntok_for(rows_s)
                   : m.k_s == kKernTc ? tc_ntok_for(rows_s) : 8 * m.nt;
@@ -208,7 +219,7 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
     m.o_sh = take((size_t)m.R * 4);
     m.o_pdn_r = take(m.E > 0 ? (size_t)m.dn_r.splits * m.Rr * m.H * 4 : 0);
     m.o_pdn_s = take(m.ns > 0 ? (size_t)m.dn_s.splits * m.Rs * m.H * 4 : 0);
-    const bool wide_r = m.k_r == kKernTc, wide_s = m.k_s == kKernTc;
+    const bool wide_r = m.k_r != kKernMma, wide_s = m.k_s != kKernMma;  // fp16 B rows
     m.o_bx_r = take(wide_r ? (size_t)m.Rr * m.H * 2 : 0);
     m.o_bx_s = take(wide_s ? (size_t)T * m.H * 2 : 0);
     m.o_bh_r = take(wide_r ? (size_t)m.Rr * m.I * 2 : 0);
@@ -383,13 +394,13 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
             L.h_out = hf;
             L.h_row_stride = m.Imax;
         }
-        if (m.k_r == kKernTs) {
-            e = launch_lut_ts(L, m.gu_r, st);
-        } else if (m.k_r == kKernTc) {
+        if (m.k_r != kKernMma) {
             void *b = ws + m.o_bx_r;
             e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, m.Rr, kMapPerm, perm, (int)m.k,
                                     (int)T, b, st, m.fused ? sx : nullptr, rsc);
-            if (e == cudaSuccess) e = launch_lut_tc(L, m.gu_r, b, m.Rr, 0, st);
+            if (e == cudaSuccess)
+                e = m.k_r == kKernTs ? launch_lut_ts(L, m.gu_r, b, m.Rr, 0, st)
+                                     : launch_lut_tc(L, m.gu_r, b, m.Rr, 0, st);
         } else {
             e = launch_lut(L, m.gu_r, st);
         }
@@ -407,13 +418,13 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
             L.h_out = hf + m.Rr * m.Imax;
             L.h_row_stride = m.Imax;
         }
-        if (m.k_s == kKernTs) {
-            e = launch_lut_ts(L, m.gu_s, st);
-        } else if (m.k_s == kKernTc) {
+        if (m.k_s != kKernMma) {
             void *b = ws + m.o_bx_s;
             e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, T, kMapIdentity, nullptr, 1,
                                     (int)T, b, st);
-            if (e == cudaSuccess) e = launch_lut_tc(L, m.gu_s, b, T, (int)T, st);
+            if (e == cudaSuccess)
+                e = m.k_s == kKernTs ? launch_lut_ts(L, m.gu_s, b, T, (int)T, st)
+                                     : launch_lut_tc(L, m.gu_s, b, T, (int)T, st);
         } else {
             e = launch_lut(L, m.gu_s, st);
         }
@@ -452,13 +463,13 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.idx0 = w->down_idx; L.cb0 = w->down_cb;
         L.w_stride = m.H * (m.I / 2); L.cb_stride = m.H * 16; L.N = (int)m.H; L.dual = false;
         L.out = pdn_r; L.out_split_stride = m.Rr * m.H; L.out_row_stride = m.H;
-        if (m.k_r == kKernTs) {
-            e = launch_lut_ts(L, m.dn_r, st);
-        } else if (m.k_r == kKernTc) {
+        if (m.k_r != kKernMma) {
             void *b = ws + m.o_bh_r;
             e = launch_codes_to_f16(hq, ldh, m.bits, (int)m.I, m.Rr, kMapIdentity, nullptr, 1, 1,
                                     b, st);
-            if (e == cudaSuccess) e = launch_lut_tc(L, m.dn_r, b, m.Rr, 0, st);
+            if (e == cudaSuccess)
+                e = m.k_r == kKernTs ? launch_lut_ts(L, m.dn_r, b, m.Rr, 0, st)
+                                     : launch_lut_tc(L, m.dn_r, b, m.Rr, 0, st);
         } else {
             e = launch_lut(L, m.dn_r, st);
         }
@@ -471,13 +482,13 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.idx0 = w->sh_down_idx; L.cb0 = w->sh_down_cb;
         L.w_stride = m.H * (m.Is / 2); L.cb_stride = m.H * 16; L.N = (int)m.H; L.dual = false;
         L.out = pdn_s; L.out_split_stride = m.Rs * m.H; L.out_row_stride = m.H;
-        if (m.k_s == kKernTs) {
-            e = launch_lut_ts(L, m.dn_s, st);
-        } else if (m.k_s == kKernTc) {
+        if (m.k_s != kKernMma) {
             void *b = ws + m.o_bh_s;
             e = launch_codes_to_f16(hq + m.Rr * ldh, ldh, m.bits, (int)m.Is, m.Rs, kMapIdentity,
                                     nullptr, 1, 1, b, st);
-            if (e == cudaSuccess) e = launch_lut_tc(L, m.dn_s, b, m.Rs, 0, st);
+            if (e == cudaSuccess)
+                e = m.k_s == kKernTs ? launch_lut_ts(L, m.dn_s, b, m.Rs, 0, st)
+                                     : launch_lut_tc(L, m.dn_s, b, m.Rs, 0, st);
         } else {
             e = launch_lut(L, m.dn_s, st);
         }

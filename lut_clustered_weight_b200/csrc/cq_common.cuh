@@ -1,7 +1,9 @@
 // cq_common.cuh -- shared device helpers for the sm_100a CodeQuant kernels.
 #pragma once
 
+#include <mutex>
 #include <utility>
+#include <vector>
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -104,10 +106,35 @@ CQ_DEV void sum_slots(const T *const (&p)[F], const int (&ns)[F], int64_t stride
     }
 }
 
+// Once per kernel and device (host): allow the largest dynamic shared memory a
+// CTA may have and ask for the full shared-memory carveout.  Every kernel of
+// the library then runs with the same L1 / shared-memory split, so the SMs
+// never re-split it between consecutive kernels, and no launch pays a
+// cudaFuncSetAttribute call.
+inline void configure_kernel_once(const void *kern) {
+    static std::mutex mu;
+    static std::vector<std::pair<const void *, int>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return;
+    std::lock_guard<std::mutex> lk(mu);
+    for (const auto &d : done)
+        if (d.first == kern && d.second == dev) return;
+    int optin = 0;
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, kern);  // dynamic + static shared memory <= opt-in limit
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         optin - (int)fa.sharedSizeBytes);
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+    done.emplace_back(kern, dev);
+}
+
 // Launch with programmatic stream serialization (and a cluster if cluster_x > 1).
 template <typename... KArgs, typename... Args>
 static inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                                      cudaStream_t st, int cluster_x, Args &&...args) {
+    configure_kernel_once(reinterpret_cast<const void *>(kern));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;

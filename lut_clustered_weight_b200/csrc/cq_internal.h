@@ -129,7 +129,10 @@ cudaError_t launch_lut(const LutLaunch &L, const LutPlan &P, cudaStream_t st);
 // The LUT GEMM kernels and which one serves a launch.
 enum LutKernel : int { kKernMma = 0, kKernTc = 1, kKernTs = 2 };
 constexpr int kTcTileRows = 128;  // weight rows per tensor-memory tile
-LutKernel pick_kernel(int64_t rows, int64_t N, bool dual);
+// tiles_bound: an upper bound on the token tiles of the launch; routed: the
+// groups are routed experts (token tiles known on the device only).
+LutKernel pick_kernel(int64_t rows, int64_t N, bool dual, int64_t K, int64_t tiles_bound,
+                      bool routed);
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -157,12 +160,14 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
 cudaError_t launch_lut_tc(const LutLaunch &L, const LutPlan &P, const void *b_f16, int64_t b_rows,
                           int b_row_mod, cudaStream_t st);
 // Tensor-memory decode kernel (groups of at most 32 rows): thread-per-row pair
-// tables, index bytes by TMA, B tiles converted from the int codes in-kernel
-// (rows mapped like LutLaunch::map_mode), so it needs no fp16 copy.
+// tables, index bytes by TMA.  The activations are read like the wide-tile
+// kernel's: fp16 rows b_f16 [b_rows][K], GEMM row p of a token tile at B row
+// (b_row_mod > 0 ? p % b_row_mod : p).
 int ts_ntok_for(int max_rows_per_group);
 LutPlan plan_lut_ts(int N, int K, bool dual, int max_rows_per_group, int64_t est_tiles,
                     int uniform_rows = 0, int n_groups = 1);
-cudaError_t launch_lut_ts(const LutLaunch &L, const LutPlan &P, cudaStream_t st);
+cudaError_t launch_lut_ts(const LutLaunch &L, const LutPlan &P, const void *b_f16,
+                          int64_t b_rows, int b_row_mod, cudaStream_t st);
 // fp16 copies of activation codes (B operand), rows mapped like LutLaunch::map_mode.
 // scales_in != nullptr: also writes scales_out[p] = scales_in[code row of p].
 cudaError_t launch_codes_to_f16(const void *codes, int64_t ld_codes, int bits, int K,

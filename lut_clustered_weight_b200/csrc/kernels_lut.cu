@@ -369,8 +369,6 @@ LutPlan plan_lut(int N, int K, bool dual, int max_rows_per_group, int64_t est_ti
 
 template <int NT, int W>
 static cudaError_t launch_lut_t(const LutLaunch &L, const LutPlan &P, cudaStream_t st) {
-    cudaFuncSetAttribute(k_lut_mma<NT, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)P.smem);
     dim3 grid(P.grid, P.streamk ? 1 : L.max_tiles);
     return launch_pdl(k_lut_mma<NT, W>, grid, dim3(W * 32), P.smem, st, 1, L, P);
 }

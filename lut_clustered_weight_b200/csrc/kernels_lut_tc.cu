@@ -124,7 +124,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     const uint32_t tmem_d = tmem + kTcA * 128;    // columns [256, 256 + kAcc NTOK)
 
     // ---- this CTA's groups and chunks (every thread walks the same sequence)
-    const int64_t n_pieces = tc_pieces(L, P);
+    const int n_pieces = tc_pieces(L, P);
     int ngroups = 0, nchunks = 0;
     {
         TcWalk cnt;
@@ -142,7 +142,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
         if (lane == 0 && nchunks > 0) {
             TcWalk bw;
             bw.init(P, n_pieces);
-            int64_t b_item = -1;
+            int b_item = -1;
             int b_y = 0;
             bool ok = true;
             for (int jc = 0, gi = 0; bw.valid && ok; bw.next(), gi++) {
@@ -235,7 +235,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
         TcWalk pw;
         pw.init(P, n_pieces);
         int gp = 0;
-        int64_t p_item = -1;
+        int p_item = -1;
         const uint8_t *p_row = nullptr;
         auto issue_group = [&]() {
             if (pw.valid) {
@@ -537,8 +537,6 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
 template <int NTOK, bool PAIR>
 static cudaError_t launch_tc_t(const CUtensorMap &m, const LutLaunch &L, const LutPlan &P,
                                int b_row_mod, cudaStream_t st) {
-    cudaFuncSetAttribute(k_lut_tc<NTOK, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)P.smem);
     return launch_pdl(k_lut_tc<NTOK, PAIR>, dim3(P.grid), dim3(kTcThreads), P.smem, st, 1, m, L, P,
                       b_row_mod);
 }
@@ -623,28 +621,32 @@ LutPlan plan_lut_ts(int N, int K, bool dual, int max_rows_per_group, int64_t est
 }
 
 template <int NTOK>
-static cudaError_t launch_ts_t(const CUtensorMap &m0, const CUtensorMap &m1, const LutLaunch &L,
-                               const LutPlan &P, cudaStream_t st) {
-    cudaFuncSetAttribute(k_lut_ts<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)P.smem);
-    return launch_pdl(k_lut_ts<NTOK>, dim3(P.grid), dim3(TsShape<NTOK>::threads), P.smem, st, 1,
-                      m0, m1, L, P);
+static cudaError_t launch_ts_t(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &mb,
+                               const LutLaunch &L, const LutPlan &P, int b_row_mod,
+                               cudaStream_t st) {
+    return launch_pdl(k_lut_ts<NTOK>, dim3(P.grid), dim3(kTsThreads), P.smem, st, 1, m0, m1, mb,
+                      L, P, b_row_mod);
 }
 
-cudaError_t launch_lut_ts(const LutLaunch &L, const LutPlan &P, cudaStream_t st) {
+cudaError_t launch_lut_ts(const LutLaunch &L, const LutPlan &P, const void *b_f16,
+                          int64_t b_rows, int b_row_mod, cudaStream_t st) {
     if (P.grid == 0 || (!P.streamk && L.max_tiles == 0)) return cudaSuccess;
     const int64_t rows = (int64_t)std::max(L.G, 1) * L.N;
     const int box = L.dual ? 64 : kTcRows;
-    CUtensorMap m0, m1;
+    const int ntok = 8 * P.nt;
+    CUtensorMap m0, m1, mb;
     std::memset(&m0, 0, sizeof(m0));
     std::memset(&m1, 0, sizeof(m1));
+    std::memset(&mb, 0, sizeof(mb));
     if (!make_idx_map(&m0, L.idx0, rows, L.K, box)) return cudaErrorInvalidValue;
     if (L.dual && !make_idx_map(&m1, L.idx1, rows, L.K, box)) return cudaErrorInvalidValue;
+    if (!make_b_map(&mb, b_f16, b_rows, L.K, ntok)) return cudaErrorInvalidValue;
     const bool timed = timing_on();
     if (timed) timing_begin(st, CQ_KERNEL_LUT_TS);
     count_launch();
-    const cudaError_t e = P.nt == 2 ? launch_ts_t<16>(m0, L.dual ? m1 : m0, L, P, st)
-                                    : launch_ts_t<32>(m0, L.dual ? m1 : m0, L, P, st);
+    const CUtensorMap &m1r = L.dual ? m1 : m0;
+    const cudaError_t e = ntok == 16 ? launch_ts_t<16>(m0, m1r, mb, L, P, b_row_mod, st)
+                                     : launch_ts_t<32>(m0, m1r, mb, L, P, b_row_mod, st);
     if (timed) timing_end(st);
     return e;
 }

@@ -266,8 +266,6 @@ static size_t part_smem(int K, int log2b, int cs) {
 template <class Kern, class... Args>
 static cudaError_t launch_clustered(Kern kern, int64_t rows, int cs, size_t smem,
                                     cudaStream_t st, Args... args) {
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)(kMaxK * sizeof(double)));
     count_launch();
     return launch_pdl(kern, dim3((unsigned)(rows * cs)), dim3(kRqThreads), smem, st, cs, args...);
 }
@@ -277,8 +275,6 @@ cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K,
     if (M == 0) return cudaSuccess;
     if (use_warp_rows(M, K, log2b)) {
         const size_t smem = (size_t)kWarpRows * K * sizeof(double);
-        cudaFuncSetAttribute(k_rq_x_warp, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(kWarpRows * 4096 * sizeof(double)));
         count_launch();
         return launch_pdl(k_rq_x_warp, dim3((unsigned)((M + kWarpRows - 1) / kWarpRows)),
                           dim3(kWarpRows * 32), smem, st, 1, reinterpret_cast<const __half *>(x),
@@ -297,8 +293,6 @@ cudaError_t launch_swiglu_rq(const SwigluArgs &a, int64_t rows, cudaStream_t st)
     const bool warp_s = a.R_shared == 0 || use_warp_rows(rows, a.I_shared, a.log2b_i_shared);
     if (warp_r && warp_s) {
         const size_t smem = (size_t)kWarpRows * a.Imax * sizeof(double);
-        cudaFuncSetAttribute(k_rq_swiglu_warp, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(kWarpRows * 4096 * sizeof(double)));
         count_launch();
         return launch_pdl(k_rq_swiglu_warp, dim3((unsigned)((rows + kWarpRows - 1) / kWarpRows)),
                           dim3(kWarpRows * 32), smem, st, 1, a, rows);

@@ -15,9 +15,9 @@
 //
 // The looked-up pairs are stored to tensor memory (row t = TMEM lane t) and
 // are the A operand of tcgen05.mma kind::f16 (M = 128, K = 16); the tokens are
-// N (16 or 32).  On B200 such an MMA issues every ~50 cycles for any N <= 64,
-// which is 41 weights per cycle per SM -- ~0.9 of the HBM rate of 4-bit
-// indices -- so the weight stream, not the multiply, sets the pace.
+// N (16 or 32), their int codes as fp16 (exact) the B operand.  On B200 such
+// an MMA issues every ~50-60 cycles for any N <= 64: 2048 weights, i.e. ~0.8
+// of the HBM rate of 4-bit indices per SM.
 //
 // Roles (one CTA per SM, persistent over stream-K or fixed-split work):
 //   warps 0-7   expand: warp w serves TMEM lane quarter w % 4 and half
@@ -25,14 +25,14 @@
 //               builds the pair tables, looks up, stores A, drains the
 //               accumulator (fp32 partial sums) once a segment is done
 //   warp 8      lane 0 issues the MMAs; the warp owns the TMEM allocation
-//   warp 9      lane 0 loads the index bytes: one 2-D TMA tile (128 rows x
-//               128 B, 128-byte swizzle) per group into a 3-stage ring
-//   warps 10-   convert the int activation codes of the group's token rows
-//               (gathered through the launch's row map) to fp16 B tiles in
-//               the 128-byte-swizzled K-major layout the MMA descriptor reads
-// Rings: index stages (3), A slots in TMEM (3 groups, columns [0, 384)), B
-// stages (2 groups), accumulators (2 x NTOK columns after the A ring, so a
-// segment's drain overlaps the next segment's MMAs).  Every wait is bounded.
+//   warp 9      lane 0 streams the index bytes: one 2-D TMA tile (128 rows x
+//               128 B, 128-byte swizzle) per group into a 4-stage ring
+//   warp 10     lane 0 loads the B tiles (fp16 codes, 64 k x NTOK rows,
+//               128-byte swizzle) per group into their own ring, ahead of
+//               the MMAs, which consume them later than the index bytes
+// Rings: index stages (4), A slots in TMEM (3 groups, columns [0, 384)), B
+// stages, accumulators (2 x NTOK columns after the A ring, so a segment's
+// drain overlaps the next segment's MMAs).  Every wait is bounded.
 #pragma once
 
 namespace cq {
@@ -42,99 +42,85 @@ namespace cq {
 #ifdef CQ_TS_TRACE
 constexpr int kTsTraceSlots = 2048;
 __device__ unsigned long long g_ts_trace[160 * kTsTraceSlots];
+// slot 2047: global timer at the start of the CTA; other slots: SM clock
 #define TS_TRACE(slot)                                                              \
     do {                                                                            \
         const int s_ = (slot);                                                      \
         if (s_ >= 0 && s_ < kTsTraceSlots && blockIdx.x < 160)                      \
-            g_ts_trace[blockIdx.x * kTsTraceSlots + s_] = globaltimer_ns();         \
+            g_ts_trace[blockIdx.x * kTsTraceSlots + s_] = clock64();                \
+    } while (0)
+#define TS_TRACE_ANCHOR()                                                           \
+    do {                                                                            \
+        if (blockIdx.x < 160)                                                       \
+            g_ts_trace[blockIdx.x * kTsTraceSlots + 2047] = globaltimer_ns();       \
     } while (0)
 #else
 #define TS_TRACE(slot) \
     do {               \
+    } while (0)
+#define TS_TRACE_ANCHOR() \
+    do {                  \
     } while (0)
 #endif
 
 constexpr int kTsExpandWarps = 8;
 constexpr int kTsWarpMma = 8;
 constexpr int kTsWarpTma = 9;
-constexpr int kTsWarpConv = 10;
+constexpr int kTsWarpB = 10;
+constexpr int kTsThreads = 32 * 11;
 constexpr int kTsA = 3;                      // A slots (groups) in TMEM
-constexpr int kTsI = 3;                      // index stages
+constexpr int kTsI = 4;                      // index stages
 constexpr uint32_t kTsIStage = kTcRows * 128;  // one group of 128 rows: 16 KB
-constexpr int kTsB = 2;                      // B stages (groups)
 constexpr uint32_t kTsTableBytes = 256 * kTcRows * 4;  // 128 KB
 
 template <int NTOK>
 struct TsShape {
     static_assert(NTOK == 16 || NTOK == 32, "token tiles of 16 or 32 rows");
-    static constexpr int conv_warps = NTOK / 16;
-    static constexpr int threads = 32 * (kTsWarpConv + conv_warps);
+    static constexpr int nb = NTOK == 16 ? 4 : 2;          // B stages (groups)
     static constexpr uint32_t b_chunk = NTOK * 128;        // one 64-k chunk tile
     static constexpr uint32_t b_stage = kTcG * b_chunk;    // one group
-    static constexpr size_t smem =
-        1024 + kTsI * kTsIStage + kTsB * b_stage + kTsTableBytes + 512;
+    static constexpr size_t smem = 1024 + kTsI * kTsIStage + nb * b_stage + kTsTableBytes + 512;
 };
 
-// fp16 value of 8 activation codes at k0 .. k0 + 7 of one code row: 4 bytes
-// (int4, low nibble first) or 8 bytes (int8).  Exact: |code| <= 127.
-CQ_DEV uint4 codes8_to_half(uint32_t lo, uint32_t hi, int bits) {
-    __align__(16) __half v[8];
-    if (bits == 4) {
-#pragma unroll
-        for (int e = 0; e < 8; e++) v[e] = __short2half_rn((short)(((int)(lo << (28 - 4 * e))) >> 28));
-    } else {
-#pragma unroll
-        for (int e = 0; e < 4; e++) {
-            v[e] = __short2half_rn((short)(((int)(lo << (24 - 8 * e))) >> 24));
-            v[4 + e] = __short2half_rn((short)(((int)(hi << (24 - 8 * e))) >> 24));
-        }
-    }
-    return *reinterpret_cast<const uint4 *>(v);
-}
-
-// Code row (row of L.codes) of output row p of the launch, -1 if none.
-CQ_DEV int ts_code_row(const LutLaunch &L, int p) {
-    return L.map_mode == kMapPerm ? L.perm[p] / L.topk : L.map_mode == kMapModT ? p % L.T : p;
-}
-
 template <int NTOK>
-__global__ void __launch_bounds__(TsShape<NTOK>::threads, 1)
+__global__ void __launch_bounds__(kTsThreads, 1)
 k_lut_ts(const __grid_constant__ CUtensorMap tmI0, const __grid_constant__ CUtensorMap tmI1,
-         const LutLaunch L, const LutPlan P) {
+         const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPlan P,
+         int b_row_mod) {
     using Sh = TsShape<NTOK>;
+    constexpr int NB = Sh::nb;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
     uint8_t *istages = sm;                                   // [kTsI][128 rows][128 B]
-    uint8_t *bstages = istages + kTsI * kTsIStage;           // [kTsB][4 chunks][NTOK][128 B]
-    uint8_t *tables = bstages + kTsB * Sh::b_stage;          // [256 entries][128 rows] x 4 B
+    uint8_t *bstages = istages + kTsI * kTsIStage;           // [NB][4 chunks][NTOK][128 B]
+    uint8_t *tables = bstages + NB * Sh::b_stage;            // [256 entries][128 rows] x 4 B
     uint64_t *i_full = reinterpret_cast<uint64_t *>(tables + kTsTableBytes);
     uint64_t *i_empty = i_full + kTsI;
     uint64_t *a_full = i_empty + kTsI, *a_empty = a_full + kTsA;
-    uint64_t *b_full = a_empty + kTsA, *b_empty = b_full + kTsB;
-    uint64_t *d_full = b_empty + kTsB, *d_empty = d_full + 2;
+    uint64_t *b_full = a_empty + kTsA, *b_empty = b_full + NB;
+    uint64_t *d_full = b_empty + NB, *d_empty = d_full + 2;
     uint64_t *tab_free = d_empty + 2, *tab_ready = tab_free + 4, *fin = tab_ready + 4;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(fin + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const TcSchedule S{&L, &P};
     const bool tr0 = tid == 0;  // trace: expand warp 0
-    if (tr0) TS_TRACE(0);
+    if (tr0) {
+        TS_TRACE(0);
+        TS_TRACE_ANCHOR();
+    }
 
     if (warp == kTsWarpMma) {
         tmem_alloc(s_tmem, 512);
         tmem_relinquish();
         if (lane == 0) {
-            for (int s = 0; s < kTsI; s++) {
-                mbar_init(&i_full[s], 1);
-                mbar_init(&i_empty[s], kTsExpandWarps);
-            }
             for (int s = 0; s < kTsA; s++) {
                 mbar_init(&a_full[s], kTsExpandWarps);
                 mbar_init(&a_empty[s], 1);
             }
-            for (int s = 0; s < kTsB; s++) {
-                mbar_init(&b_full[s], Sh::conv_warps);
+            for (int s = 0; s < NB; s++) {
+                mbar_init(&b_full[s], 1);
                 mbar_init(&b_empty[s], 1);
             }
             for (int s = 0; s < 2; s++) {
@@ -149,50 +135,69 @@ k_lut_ts(const __grid_constant__ CUtensorMap tmI0, const __grid_constant__ CUten
             fence_barrier_init();
         }
     }
+    // routed launches: the group tables come from the previous kernels.  A
+    // uniform launch reads only weights until its activations (B loads) and
+    // outputs (drains), so its set-up overlaps the previous kernel.
+    const bool routed = L.uniform_rows == 0;
+    // index stream: the first stages go out before the CTA barrier (uniform
+    // launches), the HBM latency of the weights overlaps the set-up
+    TcWalk tw;
+    int tgi = 0;
+    auto issue_index = [&]() {
+        const int s = tgi % kTsI;
+        int g, row0, nrows, rt;
+        S.item(tw.w, g, row0, nrows, rt);
+        mbar_arrive_expect_tx(&i_full[s], kTsIStage);
+        uint8_t *dst = istages + s * kTsIStage;
+        const int x = tw.c0 * (kTcChunk / 2);  // byte offset of the group in a row
+        if (L.dual) {
+            const int y = max(g, 0) * L.N + rt * 64;
+            tma_load_2d(dst, &tmI0, x, y, &i_full[s]);
+            tma_load_2d(dst + kTsIStage / 2, &tmI1, x, y, &i_full[s]);
+        } else {
+            tma_load_2d(dst, &tmI0, x, max(g, 0) * L.N + rt * kTcRows, &i_full[s]);
+        }
+        TS_TRACE(1400 + tgi);
+        tgi++;
+        tw.next();
+    };
     if (warp == kTsWarpTma && lane == 0) {
+        for (int s = 0; s < kTsI; s++) {
+            mbar_init(&i_full[s], 1);
+            mbar_init(&i_empty[s], kTsExpandWarps);
+        }
+        fence_barrier_init();
         prefetch_tmap(&tmI0);
         if (L.dual) prefetch_tmap(&tmI1);
+        if (!routed) {
+            tw.init(P, 0);
+            while (tw.valid && tgi < kTsI) issue_index();
+        }
     }
+    if (warp == kTsWarpB && lane == 0) prefetch_tmap(&tmB);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     griddep_launch();
-    // routed launches: the group tables come from the previous kernels.  A
-    // uniform launch reads only weights until its activations (converters)
-    // and outputs (drains), so its set-up overlaps the previous kernel.
-    const bool routed = L.uniform_rows == 0;
     if (routed) griddep_wait();
     const uint32_t tmem = *s_tmem;
     const uint32_t tmem_a = tmem;                      // columns [0, 384): A slots
     const uint32_t tmem_d = tmem + kTsA * 128;         // [384, 384 + 2 NTOK): accumulators
-    const int64_t n_pieces = tc_pieces(L, P);
+    const int n_pieces = tc_pieces(L, P);
     if (tr0) TS_TRACE(1);
 
     if (warp == kTsWarpTma) {
         // ====================== index stream (one thread) ======================
         if (lane == 0) {
-            TcWalk w;
-            w.init(P, n_pieces);
-            int gi = 0;
-            for (; w.valid; w.next(), gi++) {
-                const int s = gi % kTsI;
-                if (gi >= kTsI && !mbar_wait(&i_empty[s], (uint32_t)(gi / kTsI - 1) & 1u)) break;
-                int g, row0, nrows, rt;
-                S.item(w.w, g, row0, nrows, rt);
-                mbar_arrive_expect_tx(&i_full[s], kTsIStage);
-                uint8_t *dst = istages + s * kTsIStage;
-                const int x = w.c0 * (kTcChunk / 2);  // byte offset of the group in a row
-                if (L.dual) {
-                    const int y = max(g, 0) * L.N + rt * 64;
-                    tma_load_2d(dst, &tmI0, x, y, &i_full[s]);
-                    tma_load_2d(dst + kTsIStage / 2, &tmI1, x, y, &i_full[s]);
-                } else {
-                    tma_load_2d(dst, &tmI0, x, max(g, 0) * L.N + rt * kTcRows, &i_full[s]);
-                }
-                TS_TRACE(1400 + gi);
+            if (routed) tw.init(P, n_pieces);
+            TS_TRACE(1399);
+            while (tw.valid) {
+                const int s = tgi % kTsI;
+                if (tgi >= kTsI && !mbar_wait(&i_empty[s], (uint32_t)(tgi / kTsI - 1) & 1u)) break;
+                issue_index();
             }
             // loads still in flight land before the CTA may leave
-            for (int j = max(0, gi - kTsI); j < gi; j++)
+            for (int j = max(0, tgi - kTsI); j < tgi; j++)
                 mbar_wait(&i_full[j % kTsI], (uint32_t)(j / kTsI) & 1u);
         }
     } else if (warp == kTsWarpMma) {
@@ -204,14 +209,14 @@ k_lut_ts(const __grid_constant__ CUtensorMap tmI0, const __grid_constant__ CUten
             int segs = 0;
             bool ok = true;
             for (int gi = 0; mw.valid && ok; gi++, mw.next()) {
-                const int slot = gi % kTsA, bs = gi % kTsB;
+                const int slot = gi % kTsA, bs = gi % NB;
                 const bool first = mw.seg_first(), last = mw.seg_last();
                 const int buf = segs & 1;
                 if (first && segs >= 2)
-                    ok = mbar_wait(&d_empty[buf], (uint32_t)(segs / 2 - 1) & 1u);
-                ok = ok && mbar_wait(&a_full[slot], (uint32_t)(gi / kTsA) & 1u);
+                    ok = mbar_wait(&d_empty[buf], (uint32_t)(segs / 2 - 1) & 1u, 32);
+                ok = ok && mbar_wait(&a_full[slot], (uint32_t)(gi / kTsA) & 1u, 32);
                 TS_TRACE(700 + 3 * gi);
-                ok = ok && mbar_wait(&b_full[bs], (uint32_t)(gi / kTsB) & 1u);
+                ok = ok && mbar_wait(&b_full[bs], (uint32_t)(gi / NB) & 1u, 32);
                 TS_TRACE(701 + 3 * gi);
                 if (!ok) break;
                 tc_fence_after();
@@ -303,6 +308,7 @@ k_lut_ts(const __grid_constant__ CUtensorMap tmI0, const __grid_constant__ CUten
                     ok = mbar_wait(&tab_free[q], (uint32_t)(segs - 1) & 1u);
                     if (!ok) break;
                 }
+                if (tr0) TS_TRACE(650 + segs);
                 const uint4 c0v = cbn0, c1v = cbn1;
                 {
                     TcWalk nx = cw;  // prefetch the next segment's codebook
@@ -313,9 +319,11 @@ k_lut_ts(const __grid_constant__ CUtensorMap tmI0, const __grid_constant__ CUten
                 // the one-time LUT precompute: this warp builds entries
                 // [128 h, 128 h + 128) of its 32 rows' pair tables
                 const uint32_t cu[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
-#pragma unroll 1
-                for (int hh = 8 * h; hh < 8 * h + 8; hh++) {
-                    const uint32_t hv = (hh & 1) ? (cu[hh >> 1] >> 16) : (cu[hh >> 1] & 0xFFFFu);
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const int hh = 8 * h + i;  // high nibble of the entries
+                    const uint32_t wv = h ? cu[4 + (i >> 1)] : cu[i >> 1];
+                    const uint32_t hv = (i & 1) ? (wv >> 16) : (wv & 0xFFFFu);
 #pragma unroll
                     for (int l = 0; l < 16; l++)
                         tab[(hh * 16 + l) * kTcRows] =
@@ -393,103 +401,28 @@ k_lut_ts(const __grid_constant__ CUtensorMap tmI0, const __grid_constant__ CUten
             }
         }
         if (pend && ok) drain();
-    } else {
-        // ====================== B tiles from the activation codes ======================
-        // lane: 16-byte piece j (8 k) of token rows 16 wc + (lane >> 3) + 4 i
-        const int wc = warp - kTsWarpConv;
-        const int j = lane & 7;
-        if (!routed) griddep_wait();  // the codes come from the previous kernel
-        int rr[4];
-#pragma unroll
-        for (int i = 0; i < 4; i++) rr[i] = 16 * wc + (lane >> 3) + 4 * i;
-        const int bits = L.act_bits;
-        const int cb = bits == 4 ? 4 : 8;  // code bytes per 8 k
-        // codes of one group: [chunk][row] (int8 uses .y as well)
-        uint2 raw[kTcG][4], nxt[kTcG][4];
-        const uint8_t *crp[4], *ncrp[4];  // code rows of the current / next group's segment
-        auto rows_of = [&](const TcWalk &wk, const uint8_t *(&cr)[4]) {
-            int g, row0, nrows, rt;
-            S.item(wk.w, g, row0, nrows, rt);
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                cr[i] = nullptr;
-                if (rr[i] < nrows) {
-                    const int c = ts_code_row(L, row0 + rr[i]);
-                    cr[i] = L.codes + (int64_t)c * L.ld_codes;
+    } else if (warp == kTsWarpB) {
+        // ====================== B tiles (one thread) ======================
+        if (lane == 0) {
+            if (!routed) griddep_wait();  // the fp16 codes come from the previous kernel
+            TcWalk w;
+            w.init(P, n_pieces);
+            int gi = 0, b_y = 0;
+            for (; w.valid; w.next(), gi++) {
+                const int s = gi % NB;
+                if (gi >= NB && !mbar_wait(&b_empty[s], (uint32_t)(gi / NB - 1) & 1u)) break;
+                if (w.seg_first()) {
+                    int g, row0, nrows, rt;
+                    S.item(w.w, g, row0, nrows, rt);
+                    b_y = b_row_mod > 0 ? row0 % b_row_mod : row0;
                 }
+                mbar_arrive_expect_tx(&b_full[s], Sh::b_chunk * w.gn);
+                for (int i = 0; i < w.gn; i++)
+                    tma_load_2d(bstages + s * Sh::b_stage + i * Sh::b_chunk, &tmB,
+                                (w.c0 + i) * kTcChunk, b_y, &b_full[s]);
             }
-        };
-        auto fetch = [&](const TcWalk &wk, const uint8_t *const (&cr)[4], uint2 (&dst)[kTcG][4]) {
-#pragma unroll
-            for (int c = 0; c < kTcG; c++) {
-                const int k0 = (wk.c0 + c) * kTcChunk + 8 * j;
-                const bool kin = c < wk.gn && k0 < L.K;
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    dst[c][i] = make_uint2(0, 0);
-                    if (kin && cr[i]) {
-                        const uint8_t *src = cr[i] + (int64_t)k0 * cb / 8;
-                        if (bits == 4)
-                            dst[c][i].x = __ldg(reinterpret_cast<const unsigned int *>(src));
-                        else
-                            dst[c][i] = __ldg(reinterpret_cast<const uint2 *>(src));
-                    }
-                }
-            }
-        };
-        TcWalk bw, pw;  // convert / prefetch (one group ahead)
-        bw.init(P, n_pieces);
-        pw = bw;
-        bool ok = true;
-        if (bw.valid) {
-            rows_of(bw, crp);
-            fetch(bw, crp, raw);
-            pw.next();
-            if (pw.valid) {
-                if (pw.seg_first()) rows_of(pw, ncrp);
-                else
-#pragma unroll
-                    for (int i = 0; i < 4; i++) ncrp[i] = crp[i];
-            }
-        }
-        for (int gi = 0; bw.valid && ok; gi++) {
-            // next group's codes in flight while this one is converted
-            if (pw.valid) fetch(pw, ncrp, nxt);
-            const int s = gi % kTsB;
-            if (gi >= kTsB) {
-                ok = mbar_wait(&b_empty[s], (uint32_t)(gi / kTsB - 1) & 1u);
-                if (!ok) break;
-            }
-            if (tid == 32 * kTsWarpConv) TS_TRACE(1100 + 2 * gi);
-            uint8_t *dst = bstages + s * Sh::b_stage;
-#pragma unroll
-            for (int c = 0; c < kTcG; c++) {
-                if (c < bw.gn) {
-#pragma unroll
-                    for (int i = 0; i < 4; i++) {
-                        const int r = rr[i];
-                        *reinterpret_cast<uint4 *>(dst + c * Sh::b_chunk + r * 128 +
-                                                   ((j ^ (r & 7)) << 4)) =
-                            codes8_to_half(raw[c][i].x, raw[c][i].y, bits);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&b_full[s]);
-            if (tid == 32 * kTsWarpConv) TS_TRACE(1101 + 2 * gi);
-            // advance: the prefetched group becomes current
-            bw = pw;
-#pragma unroll
-            for (int c = 0; c < kTcG; c++)
-#pragma unroll
-                for (int i = 0; i < 4; i++) raw[c][i] = nxt[c][i];
-#pragma unroll
-            for (int i = 0; i < 4; i++) crp[i] = ncrp[i];
-            if (pw.valid) {
-                pw.next();
-                if (pw.valid && pw.seg_first()) rows_of(pw, ncrp);
-            }
+            for (int j = max(0, gi - NB); j < gi; j++)
+                mbar_wait(&b_full[j % NB], (uint32_t)(j / NB) & 1u);
         }
     }
     // ---- teardown: all MMAs and tensor-memory reads are complete

@@ -60,15 +60,19 @@ CQ_DEV uint64_t globaltimer_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Wait for the phase with the given parity to complete.  Gives up after about
-// one second, records kErrWaitTimeout and returns false.
-CQ_DEV bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete.  A thread that has to
+// wait sleeps between polls (16 ns doubling up to max_sleep_ns), so waiting
+// warps leave the issue slots and the shared-memory pipe to the working ones.
+// Gives up after about one second, records kErrWaitTimeout and returns false.
+CQ_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t max_sleep_ns = 256) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (true) {
-        for (int i = 0; i < 64; i++)
-            if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > 1000000000ull) break;
+    uint32_t ns = 16;
+    for (uint32_t i = 1;; i++) {
+        __nanosleep(ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        ns = min(2 * ns, max_sleep_ns);
+        if ((i & 63) == 0 && globaltimer_ns() - t0 > 1000000000ull) break;
     }
     atomicExch(&g_device_error, kErrWaitTimeout);
     return false;

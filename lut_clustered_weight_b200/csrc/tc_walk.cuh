@@ -11,18 +11,21 @@ constexpr int kTcRows = 128;         // rows per tile (TMEM lanes)
 constexpr int kTcChunk = 64;         // k per chunk: 4 MMAs of K = 16, 32 TMEM columns
 constexpr int kTcG = 4;              // chunks per group (256 k)
 
+// All work counts of a tensor-memory launch fit in 31 bits (the host plans only
+// launches whose units * grid < 2^31), so the schedule uses 32-bit integer
+// arithmetic: 64-bit division is a long software sequence on the GPU.
 struct TcSchedule {
     const LutLaunch *L;
     const LutPlan *P;
     // work item -> (group, first row, rows, row tile)
-    CQ_DEV void item(int64_t w, int &g, int &row0, int &nrows, int &rt) const {
+    CQ_DEV void item(int w, int &g, int &row0, int &nrows, int &rt) const {
         const int TT = 8 * P->nt;
-        const int64_t tile = w / P->n_row_tiles;
-        rt = (int)(w - tile * P->n_row_tiles);
+        const int tile = w / P->n_row_tiles;
+        rt = w - tile * P->n_row_tiles;
         if (L->uniform_rows > 0) {
             const int tpg = (L->uniform_rows + TT - 1) / TT;
-            g = (int)(tile / tpg);
-            row0 = g * L->uniform_rows + (int)(tile - (int64_t)g * tpg) * TT;
+            g = tile / tpg;
+            row0 = g * L->uniform_rows + (tile - g * tpg) * TT;
             nrows = min(TT, (g + 1) * L->uniform_rows - row0);
         } else {
             if (tile >= L->grp_tiles[L->G]) {
@@ -31,7 +34,7 @@ struct TcSchedule {
                 return;
             }
             g = L->tile_grp[tile];
-            row0 = L->grp_rows[g] + (int)(tile - L->grp_tiles[g]) * TT;
+            row0 = L->grp_rows[g] + (tile - L->grp_tiles[g]) * TT;
             nrows = min(TT, L->grp_rows[g + 1] - row0);
         }
     }
@@ -64,18 +67,19 @@ struct TcSchedule {
 // tile count.  Every role of the CTA walks the same sequence.
 struct TcWalk {
     const LutPlan *P;
-    int64_t w;        // work item of the current segment
+    int w;            // work item of the current segment
     int c0, gn;       // first chunk (item-relative) and chunk count of the group
     int c_begin, c_end;
     int slot;         // partial-sum slot the segment writes
-    int64_t nxt, lim;
+    int nxt, lim;
     bool valid;
 
-    CQ_DEV void init(const LutPlan &Pl, int64_t n_pieces) {
+    CQ_DEV void init(const LutPlan &Pl, int n_pieces) {
         P = &Pl;
         if (Pl.streamk) {
-            nxt = (int64_t)blockIdx.x * Pl.units / Pl.grid;
-            lim = ((int64_t)blockIdx.x + 1) * Pl.units / Pl.grid;
+            const int U = (int)Pl.units;
+            nxt = (int)blockIdx.x * U / Pl.grid;
+            lim = ((int)blockIdx.x + 1) * U / Pl.grid;
         } else {
             nxt = blockIdx.x;
             lim = n_pieces;
@@ -88,14 +92,16 @@ struct TcWalk {
         const int C = P->chunks_total;
         if (P->streamk) {
             w = nxt / C;
-            c_begin = (int)(nxt - w * C);
-            const int64_t e = min(lim, (w + 1) * C);
-            c_end = (int)(e - w * C);
-            slot = (int)(blockIdx.x - lut_cta_of_unit(*P, w * C));
+            c_begin = nxt - w * C;
+            const int e = min(lim, (w + 1) * C);
+            c_end = e - w * C;
+            // first CTA of the item: the one whose range holds its unit w * C
+            const int first = ((w * C + 1) * P->grid - 1) / (int)P->units;
+            slot = (int)blockIdx.x - first;
             nxt = e;
         } else {
             w = nxt / P->splits;
-            const int sp = (int)(nxt - w * P->splits);
+            const int sp = nxt - w * P->splits;
             c_begin = sp * P->chunks_per_split;
             c_end = min(C, c_begin + P->chunks_per_split);
             slot = sp;
@@ -115,12 +121,11 @@ struct TcWalk {
 
 // Pieces of a fixed-split launch that hold rows (the routing decides how many
 // token tiles there are; the host only knows an upper bound).
-CQ_DEV int64_t tc_pieces(const LutLaunch &L, const LutPlan &P) {
+CQ_DEV int tc_pieces(const LutLaunch &L, const LutPlan &P) {
     if (P.streamk) return 0;
     const int TT = 8 * P.nt;
-    const int64_t tiles = L.uniform_rows > 0
-                              ? (int64_t)L.G * ((L.uniform_rows + TT - 1) / TT)
-                              : min((int64_t)L.grp_tiles[L.G], (int64_t)L.max_tiles);
+    const int tiles = L.uniform_rows > 0 ? L.G * ((L.uniform_rows + TT - 1) / TT)
+                                         : min(L.grp_tiles[L.G], L.max_tiles);
     return tiles * P.n_row_tiles * P.splits;
 }
 
