@@ -1,26 +1,35 @@
 """Benchmark of the B200 CodeQuant LUT MoE linear layer.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|all] [--impl ours|reference]
 
-Default workload: the Qwen3-4B-shaped dense SwiGLU FFN decode layer (hidden
-2560, intermediate 9728, gate/up 2560->9728, down 9728->2560) in all six
-published variants -- M in {1, 4, 16} tokens x {A4W4, A8W4}.  One step runs
-each variant twice (84 tokens), every call on its own copy of the weights,
-so a step streams 12 x 38 MB of packed indices + codebooks (> 2 x the 126 MB
-L2) and no call finds its weights in L2 from the previous step.
+Default: all five workloads in one run, each a "step" of layer calls on
+seeded synthetic inputs with those models' layer shapes:
+  linear_m1_k2048_n2048     one linear, M=1, K=N=2048, A4W4 (rotate+quantize,
+                            LUT GEMV); a step = 128 calls, each on its own
+                            weight copy (> 2 x the 126 MB L2)
+  qwen3_4b_ffn_decode       Qwen3-4B-shaped dense SwiGLU FFN (2560 / 9728),
+                            M in {1, 4, 16} x {A4W4, A8W4}, each on two weight
+                            copies: 12 layer calls, 84 tokens per step
+  qwen3_30b_a3b_moe_decode  128 experts, top-8, 64 tokens, A4W4
+  mixtral_8x7b_moe          8 experts (one biased), top-2, 256 tokens, A8W4
+  prefill_moe_e64_s2        64 routed + 2 shared experts, top-6, 4096 tokens
+The JSON line's headline (value, roofline, e2e, cpu_baseline) is the prefill
+MoE layer, the largest single-GPU configuration by work (567 GFLOP, 4096
+tokens); the other four are blocks under "workloads" with the same keys.
 
-Reported (one JSON line from rank 0):
+Per workload:
   value       tokens/s of the whole job (sum over ranks / max time), device
-              timed with CUDA events, inputs resident in HBM; the step is
-              replayed from a CUDA graph (the decode serving path)
+              timed with CUDA events, inputs resident in HBM, the step
+              replayed from a CUDA graph
   e2e         the same metric through the C-ABI calls with host buffers: the
-              step's activations copied from pinned host memory and the
-              outputs copied back inside the timed region
-  roofline    the dominant LUT GEMM kernel, from its CUDA-event-timed launches:
-              the mma.sync decode kernel as algorithmic bytes against the
-              measured HBM copy peak, the tensor-memory kernel (groups of more
-              than 16 rows) as flops against the measured dense bf16 peak
-  cpu_baseline  the CPU oracle on the host cores, on a bounded token sample
+              step's activations (and router logits) copied from pinned host
+              memory and the outputs copied back inside the timed region
+  roofline    the dominant LUT GEMM kernel, from its CUDA-event-timed
+              launches: the decode kernels (mma.sync, tensor-memory decode)
+              as algorithmic bytes against the measured HBM copy peak, the
+              wide-token-tile tensor-memory kernel as flops against the
+              measured dense bf16 peak
+  cpu_baseline  (headline) the CPU oracle on the host cores, bounded sample
 Multi-GPU: replicas only (each rank runs the whole workload on its own GPU);
 the timing is the max over ranks.
 """
@@ -66,8 +75,11 @@ def workload_shapes(name):
     raise SystemExit(f"unknown workload {name}")
 
 
-WORKLOADS = ["qwen3_4b_ffn_decode", "qwen3_30b_a3b_moe_decode", "mixtral_8x7b_moe",
+LINEAR = "linear_m1_k2048_n2048"
+LINEAR_COPIES = 128            # 128 x 2.2 MB of weights per step (> 2 x L2)
+WORKLOADS = [LINEAR, "qwen3_4b_ffn_decode", "qwen3_30b_a3b_moe_decode", "mixtral_8x7b_moe",
              "prefill_moe_e64_s2"]
+HEADLINE = "prefill_moe_e64_s2"
 
 
 def load_peaks():
@@ -456,56 +468,95 @@ def timed(fn, steps, dist, world):
     return max_over_ranks(e0.elapsed_time(e1), dist, world)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="qwen3_4b_ffn_decode", choices=WORKLOADS)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-graph", action="store_true", help="time eager calls, not a CUDA graph")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
-    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
-    ap.add_argument("--no-bf16", action="store_true", help="skip the torch bf16 context leg")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
-    if args.impl == "reference":
-        return run_reference(args)
+class LinearCall:
+    """One linear call of the single-linear workload (rotate+quantize, then the
+    LUT GEMV), every tensor resident, plus pinned host copies for e2e."""
 
+    def __init__(self, cq, shape, x, w, cb, dev):
+        import torch
+        self.cq, self.s = cq, shape
+        self.x = torch.from_numpy(x).to(dev)
+        self.w, self.cb = w, cb
+        self.q = torch.empty((shape.M, shape.K // 2 if shape.act_bits == 4 else shape.K),
+                             dtype=torch.uint8 if shape.act_bits == 4 else torch.int8, device=dev)
+        self.sx = torch.empty((shape.M,), dtype=torch.float32, device=dev)
+        self.y = torch.empty((shape.M, shape.N), dtype=torch.float32, device=dev)
+        nb = cq.cq_lut_gemm_workspace_size(shape.M, shape.N, shape.K, shape.act_bits)
+        self.ws = torch.empty((max(nb, 1),), dtype=torch.uint8, device=dev)
+        self.x_h = torch.from_numpy(x).pin_memory()
+        self.y_h = torch.empty((shape.M, shape.N), dtype=torch.float32).pin_memory()
+        self.h2d, self.d2h = self.x_h.numel() * 2, self.y_h.numel() * 4
+
+    def run(self):
+        s = self.s
+        self.cq.cq_rotate_quantize(self.x, s.had_block, s.act_bits, q_out=self.q, s_out=self.sx)
+        self.cq.cq_lut_gemm(self.q, self.sx, s.K, s.act_bits, self.w, self.cb, y=self.y,
+                            workspace=self.ws)
+
+    def run_e2e(self):
+        self.x.copy_(self.x_h, non_blocking=True)
+        self.run()
+        self.y_h.copy_(self.y, non_blocking=True)
+
+
+def lut_timed_launches(cq, step, steps):
+    """Every LUT GEMM launch of `steps` eager steps, CUDA-event timed on its
+    stream.  A spin kernel ahead of every step keeps the GPU busy while the
+    host queues the step, so consecutive kernels run back to back and no
+    launch's events include time the GPU spent waiting for the host."""
     import torch
-    import torch.distributed as dist
+    t_host = time.perf_counter()
+    step()
+    torch.cuda.synchronize()
+    t_host = time.perf_counter() - t_host
+    spin_cycles = int(min(50e-3, 3 * t_host + 1e-3) * 2.0e9)
+    cq.cq_timing_read_launches()  # drop anything recorded before
+    cq.cq_timing_enable(True)
+    for _ in range(steps):
+        torch.cuda._sleep(spin_cycles)
+        step()
+    torch.cuda.synchronize()
+    cq.cq_timing_enable(False)
+    return cq.cq_timing_read_launches()
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    import lut_clustered_weight_b200 as cq
-
-    peak_gbs, peak_tf, peak_kind = load_peaks()
-    stream = torch.cuda.Stream(device=dev)
-    torch.cuda.set_stream(stream)
-
-    shapes, inputs = workload_inputs(args.workload)
-    layers = [DeviceLayer(cq, inputs[s.name], dev) for s in shapes]
-    tokens_per_step = sum(s.T for s in shapes)
+def measure(cq, name, args, dev, stream, dist, world, peaks):
+    """One workload: the step resident (graph replay), the LUT kernel launch by
+    launch, and the step end to end from host buffers.  Returns its block."""
+    import torch
+    import synth
+    peak_gbs, peak_tf, peak_kind = peaks
+    cpu_in = None
+    if name == LINEAR:
+        s = synth.CFG0
+        x, w_idx, cb = synth.linear_inputs(s)
+        w0 = torch.from_numpy(w_idx).to(dev)
+        c0 = torch.from_numpy(cb).to(dev)
+        calls = [LinearCall(cq, s, synth.activations(s.M, s.K, seed=0, name=f"{s.name}.x{i}"),
+                            w0.clone(), c0.clone(), dev) for i in range(LINEAR_COPIES)]
+        del w0, c0
+        units_per_step = LINEAR_COPIES * s.M
+        launch_alg = [(lut_alg_bytes(s.M, s.N, s.K, s.act_bits), 2 * s.M * s.N * s.K)]
+        launch_alg *= LINEAR_COPIES
+        alg_bytes_step = sum(b for b, _ in launch_alg) + LINEAR_COPIES * 2 * s.M * s.K
+        alg_flops_step = sum(f for _, f in launch_alg)
+        cfg = {"workload": name, "calls_per_step": LINEAR_COPIES, "M": s.M, "K": s.K, "N": s.N,
+               "had_block": s.had_block, "act_bits": s.act_bits,
+               "weights": "one k-means weight set, a device copy per call"}
+    else:
+        shapes, cpu_in = workload_inputs(name)
+        calls = [DeviceLayer(cq, cpu_in[sh.name], dev) for sh in shapes]
+        units_per_step = sum(sh.T for sh in shapes)
+        counts = [L.counts(dev) for L in calls]
+        launch_alg = [a for L, c in zip(calls, counts) for a in lut_launches(L.s, c)]
+        alg_bytes_step = sum(layer_alg(L.s, c)[0] for L, c in zip(calls, counts))
+        alg_flops_step = sum(layer_alg(L.s, c)[1] for L, c in zip(calls, counts))
+        cfg = {"workload": name, "layers_per_step": [sh.name for sh in shapes]}
 
     def step():
-        for L in layers:
-            L.run()
+        for c in calls:
+            c.run()
 
-    # byte / flop accounting (routing counts of the synthetic inputs)
-    counts = [L.counts(dev) for L in layers]
-    launch_alg = [a for L, c in zip(layers, counts) for a in lut_launches(L.s, c)]
-    alg_bytes_step = sum(layer_alg(L.s, c)[0] for L, c in zip(layers, counts))
-    alg_flops_step = sum(layer_alg(L.s, c)[1] for L, c in zip(layers, counts))
-
-    # ---- warm-up (eager), launch count of one step
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -525,65 +576,113 @@ def main():
         run = step
     for _ in range(args.warmup):
         run()
+    local = torch.cuda.current_device()
     with ClockSampler(local) as clk:
         ms = timed(run, args.steps, dist, world)
     clocks = clk.summary()
     ms_step = ms / args.steps
-    value = job_throughput(tokens_per_step, args.steps, world, ms)
+    value = job_throughput(units_per_step, args.steps, world, ms)
 
-    # ---- the LUT GEMM kernel, CUDA-event timed launch by launch (eager steps).
-    # A spin kernel ahead of every step keeps the GPU busy while the host
-    # queues the step, so consecutive kernels run back to back as in the
-    # graph and no launch's events include time the GPU spent waiting for
-    # the host.
-    t_host = time.perf_counter()
-    step()
-    torch.cuda.synchronize()
-    t_host = time.perf_counter() - t_host
-    spin_cycles = int(min(50e-3, 3 * t_host + 1e-3) * 2.0e9)
-    cq.cq_timing_read_launches()  # drop anything recorded before
-    cq.cq_timing_enable(True)
-    for _ in range(args.steps):
-        torch.cuda._sleep(spin_cycles)
-        step()
-    torch.cuda.synchronize()
-    cq.cq_timing_enable(False)
-    timed_launches = cq.cq_timing_read_launches()
+    # ---- the LUT GEMM kernel, launch by launch
+    timed_launches = lut_timed_launches(cq, step, args.steps)
     assert len(timed_launches) == args.steps * len(launch_alg), (len(timed_launches), len(launch_alg))
     roofline, kern_src = lut_roofline(launch_alg, timed_launches, args.steps, ms_step,
                                       peak_gbs, peak_tf, peak_kind)
     roofline["traffic"] = profile_traffic(ROOT / "lut_clustered_weight_b200" / "csrc" / kern_src,
-                                          ROOT / "profiles" / f"{roofline['kernel']}_{args.workload}.md")
+                                          ROOT / "profiles" / f"{roofline['kernel']}_{name}.md")
 
     # ---- e2e: host buffers through the C-ABI, copies inside the timed region
     def step_e2e():
-        for L in layers:
-            L.run_e2e()
+        for c in calls:
+            c.run_e2e()
     for _ in range(args.warmup):
         step_e2e()
     ms_e2e = timed(step_e2e, args.steps, dist, world)
-    e2e = {"value": job_throughput(tokens_per_step, args.steps, world, ms_e2e), "unit": "tokens/s",
-           "h2d_bytes_per_step": sum(L.h2d for L in layers),
-           "d2h_bytes_per_step": sum(L.d2h for L in layers),
-           "ms_per_step": ms_e2e / args.steps}
+    e2e = {"value": job_throughput(units_per_step, args.steps, world, ms_e2e), "unit": "tokens/s",
+           "h2d_bytes_per_step": sum(c.h2d for c in calls),
+           "d2h_bytes_per_step": sum(c.d2h for c in calls), "ms_per_step": ms_e2e / args.steps}
 
-    # ---- context: the same dense FFN step in bf16 with torch (F.linear, dense
-    # weights, own weight copy per call, CUDA graph) -- the pages compare
-    # their decode kernel against BF16
-    bf16 = None
-    if all(s.E == 0 for s in shapes) and not args.no_bf16:
+    cfg.update({"tokens_per_step": units_per_step, "cuda_graph": use_graph,
+                "l2": "no flush: each step streams "
+                      f"{alg_bytes_step / 1e6:.0f} MB of distinct weights (> 126 MB L2)",
+                "parallelism": f"replicas x{world}"})
+    block = {"value": value, "unit": "tokens/s", "ms_per_step": ms_step, "config": cfg,
+             "effective_gbs": alg_bytes_step / (ms_step / 1e3) / 1e9,
+             "alg_bytes_per_step": alg_bytes_step, "alg_flops_per_step": alg_flops_step,
+             "roofline": roofline, "e2e": e2e,
+             "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
+
+    # ---- context: the same dense FFN step in bf16 with torch (the pages
+    # compare their decode kernel against BF16)
+    if name != LINEAR and all(sh.E == 0 for sh in shapes) and not args.no_bf16:
         bf16 = bf16_dense_context(shapes, dev, stream, args.steps, args.warmup, dist, world)
         bf16["speedup_of_value"] = value / bf16["value"]
+        block["bf16_context"] = bf16
+    if use_graph:
+        del graph
+    del calls
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return block, cpu_in
 
-    # ---- CPU oracle baseline (rank 0, one GPU only)
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="all", choices=["all"] + WORKLOADS)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-graph", action="store_true", help="time eager calls, not a CUDA graph")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    ap.add_argument("--no-bf16", action="store_true", help="skip the torch bf16 context leg")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    headline = HEADLINE if args.workload == "all" else args.workload
+    if args.impl == "reference":
+        if headline == LINEAR:
+            raise SystemExit("the reference arm times the layer workloads")
+        args.workload = headline
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    import lut_clustered_weight_b200 as cq
+
+    peaks = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+
+    names = WORKLOADS if args.workload == "all" else [args.workload]
+    blocks, head_inputs = {}, None
+    for name in names:
+        blocks[name], cpu_in = measure(cq, name, args, dev, stream, dist, world, peaks)
+        if name == headline:
+            head_inputs = cpu_in
+    head = blocks.pop(headline)
+
+    # ---- CPU oracle baseline of the headline workload (rank 0, one GPU only)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu and headline != LINEAR:
         import oracle
-        n, dt, desc = cpu_oracle_sample(shapes, inputs, args.cpu_seconds)
+        shapes = workload_shapes(headline)
+        n, dt, desc = cpu_oracle_sample(shapes, head_inputs, args.cpu_seconds)
         cpu = {"value": n / dt, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
                "sample": desc}
         oracle.set_threads(1)
-        n1, dt1, desc1 = cpu_oracle_sample(shapes, inputs, args.cpu_seconds / 3)
+        n1, dt1, desc1 = cpu_oracle_sample(shapes, head_inputs, args.cpu_seconds / 3)
         oracle.set_threads(oracle_threads())
         cpu["single_thread"] = {"value": n1 / dt1, "unit": "tokens/s", "cores": 1,
                                 "sample": desc1}
@@ -592,24 +691,22 @@ def main():
         dist.barrier()
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f16", "data": "synthetic",
-            "config": {"workload": args.workload,
-                       "layers_per_step": [s.name for s in shapes],
-                       "tokens_per_step": tokens_per_step, "cuda_graph": use_graph,
-                       "l2": "no flush: each step streams "
-                             f"{alg_bytes_step / 1e6:.0f} MB of distinct weights (> 126 MB L2)",
-                       "parallelism": f"replicas x{world}"},
-            "effective_gbs": alg_bytes_step / (ms_step / 1e3) / 1e9,
-            "alg_bytes_per_step": alg_bytes_step, "alg_flops_per_step": alg_flops_step,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "bf16_context": bf16,
-            "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+            "dtype": "f16", "data": "synthetic", "config": head["config"],
+            "effective_gbs": head["effective_gbs"],
+            "alg_bytes_per_step": head["alg_bytes_per_step"],
+            "alg_flops_per_step": head["alg_flops_per_step"],
+            "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+            "workloads": blocks,
             "dtype_note": "int4/int8 codes and 4-bit indices; looked-up weights as fp16 "
-                          "into mma.sync (decode) or tcgen05 kind::f16 (more than 16 "
-                          "rows per group) with fp32 accumulation; rotation exact in fp64",
+                          "into mma.sync or tcgen05 kind::f16 (tensor memory A operand) with "
+                          "fp32 accumulation; rotation exact in fp64",
         }
+        if "bf16_context" in head:
+            line["bf16_context"] = head["bf16_context"]
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -236,10 +236,25 @@ class MoEInputs:
 
 
 def _expert_stack(n: int, N: int, K: int, seed: int, prefix: str):
+    """Weights of n experts.  Every expert draws from its own named stream, so
+    generating them on a thread pool (numpy's bulk draws and torch's CPU ops
+    release the interpreter lock) gives exactly the serial result."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
     idx = np.empty((n, N, K // 2), dtype=np.uint8)
     cb = np.empty((n, N, 16), dtype=np.float16)
-    for e in range(n):
+
+    def one(e):
         idx[e], cb[e] = lut_weights(N, K, seed=seed, name=f"{prefix}.{e}")
+
+    workers = max(1, min(n, (os.cpu_count() or 1), 16))
+    if workers == 1:
+        for e in range(n):
+            one(e)
+    else:
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            list(ex.map(one, range(n)))
     return idx, cb
 
 
