@@ -67,6 +67,7 @@ def lib():
         _lib.orc_rotate.argtypes = [P, I64, I64, I64, P]
         _lib.orc_quantize.argtypes = [P, I64, I64, I64, I32, P, P]
         _lib.orc_rotate_quantize.argtypes = [P, I64, I64, I64, I32, P, P]
+        _lib.orc_scale_permute.argtypes = [P, I64, I64, P, P, P]
         _lib.orc_unpack_int4.argtypes = [P, I64, I64, P]
         _lib.orc_pack_int4.argtypes = [P, I64, I64, P]
         _lib.orc_unpack_idx.argtypes = [P, I64, I64, P]
@@ -75,6 +76,7 @@ def lib():
         _lib.orc_swiglu.argtypes = [P, P, I64, P]
         _lib.orc_combine.argtypes = [P, P, I64, I64, I64, P, I64, P]
         for f in ("orc_hadamard_matrix", "orc_rotate", "orc_quantize", "orc_rotate_quantize",
+                  "orc_scale_permute",
                   "orc_lut_gemm", "orc_route"):
             getattr(_lib, f).restype = I32
     return _lib
@@ -141,8 +143,26 @@ def quantize(x_rot: np.ndarray, b: int, bits: int):
     return q, s
 
 
-def rotate_quantize(x: np.ndarray, b: int, bits: int):
-    """fp16 [M, K] -> (q int8 [M, K] unpacked, s fp32 [M])."""
+def scale_permute(x: np.ndarray, scale=None, perm=None) -> np.ndarray:
+    """fp16 [M, K] -> fp16 [M, K]: out[m, j] = fp16(x[m, perm[j]] * scale[perm[j]])
+    (the identity / 1 where perm / scale is None); ValueError unless perm is a
+    permutation of 0..K-1."""
+    x = _c(x, np.float16)
+    M, K = x.shape
+    sc = None if scale is None else _c(scale, np.float16).reshape(K)
+    pm = None if perm is None else _c(perm, np.int32).reshape(K)
+    out = np.empty((M, K), dtype=np.float16)
+    _check(lib().orc_scale_permute(_p(x.view(np.uint16)), M, K,
+                                   None if sc is None else _p(sc.view(np.uint16)), _p(pm),
+                                   _p(out.view(np.uint16))), "scale_permute")
+    return out
+
+
+def rotate_quantize(x: np.ndarray, b: int, bits: int, scale=None, perm=None):
+    """fp16 [M, K] -> (q int8 [M, K] unpacked, s fp32 [M]); with a smoothing
+    scale and/or channel permutation applied first (scale_permute)."""
+    if scale is not None or perm is not None:
+        x = scale_permute(x, scale, perm)
     x = _c(x, np.float16)
     M, K = x.shape
     q = np.empty((M, K), dtype=np.int8)

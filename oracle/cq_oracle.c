@@ -210,6 +210,45 @@ int orc_quantize(const double *xr, int64_t M, int64_t K, int64_t b, int bits,
     return ORC_OK;
 }
 
+/*
+ * Online smoothing scale and channel grouping ahead of the rotation.
+ * CodeQuant2 page, Figure 1: rotation and scaling are fused into the model
+ * (Table 5's base setting uses SmoothQuant scaling); CodeQuant podcast page,
+ * "Summary": the channels are reordered before clustering so that outliers
+ * are spread over different groups.  Both are applied to the layer input:
+ *   out[m, j] = rne16( x[m, p(j)] * s(p(j)) )
+ * with p = perm (the identity if perm is NULL) and s = scale (1 if NULL).
+ * The product of two fp16 numbers is exact in fp64 (11 + 11 significant
+ * bits), so out is the fp16 rounding, ties to even, of the exact product.
+ * x, scale, out: fp16 bits.  Returns ORC_EINVAL unless perm is a permutation
+ * of 0 .. K-1.
+ */
+int orc_scale_permute(const uint16_t *x, int64_t M, int64_t K, const uint16_t *scale,
+                      const int32_t *perm, uint16_t *out)
+{
+    if (perm) {
+        unsigned char *seen = (unsigned char *)calloc((size_t)K, 1);
+        if (!seen)
+            return ORC_EINVAL;
+        for (int64_t j = 0; j < K; j++) {
+            if (perm[j] < 0 || perm[j] >= K || seen[perm[j]]) {
+                free(seen);
+                return ORC_EINVAL;
+            }
+            seen[perm[j]] = 1;
+        }
+        free(seen);
+    }
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t j = 0; j < K; j++) {
+            const int64_t c = perm ? perm[j] : j;
+            const double v = orc_f16_to_f64(x[m * K + c]);
+            const double sc = scale ? orc_f16_to_f64(scale[c]) : 1.0;
+            out[m * K + j] = orc_f64_to_f16(v * sc);
+        }
+    return ORC_OK;
+}
+
 /* rotate then quantize; x fp16 bits [M, K]. */
 int orc_rotate_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t b, int bits,
                         int8_t *q, float *s)

@@ -414,3 +414,118 @@ def test_planted_mistakes_are_caught():
     assert np.allclose(y, ref, rtol=1e-12)
     assert not np.allclose(bad_drop, ref, rtol=1e-6)
     assert not np.allclose(y_swap, ref, rtol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# online smoothing scale and channel grouping ahead of the rotation
+
+
+def _f16_nearest_fraction(v: Fraction) -> float:
+    """The fp16 value nearest to the exact rational v, ties to even (written
+    from the format: 11 significant bits, exponent >= -14, subnormal quantum
+    2^-24), independent of the oracle's encoder and of numpy."""
+    if v == 0:
+        return 0.0
+    a = abs(v)
+    e = max(math.floor(math.log2(a)), -14)
+    while Fraction(2) ** e > a:          # guard the float log2
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    e = max(e, -14)
+    quantum = Fraction(2) ** (e - 10)
+    n = a / quantum
+    lo = math.floor(n)
+    r = n - lo
+    n = lo + 1 if (r > Fraction(1, 2) or (r == Fraction(1, 2) and lo % 2 == 1)) else lo
+    out = float(n * quantum)
+    return -out if v < 0 else out
+
+
+def test_scale_rounds_the_exact_product_to_nearest_even():
+    g = np.random.default_rng(41)
+    x = (g.standard_normal((3, 64)) * np.array([1, 1e-4, 300.0])[:, None]).astype(np.float16)
+    s = (g.random(64) * 4 + 0.01).astype(np.float16)
+    out = oracle.scale_permute(x, scale=s)
+    # numpy: the fp64 product of two fp16 values is exact; astype rounds to nearest even
+    ref = (x.astype(np.float64) * s.astype(np.float64)).astype(np.float16)
+    np.testing.assert_array_equal(out.view(np.uint16), ref.view(np.uint16))
+    # exact rationals on a sample, including subnormal results
+    for (m, k) in [(0, 0), (1, 5), (1, 17), (2, 63), (0, 31)]:
+        exact = Fraction(float(x[m, k])) * Fraction(float(s[k]))
+        assert float(out[m, k]) == _f16_nearest_fraction(exact)
+
+
+def test_scale_ties_go_to_even():
+    # exact products: 2050 * 0.5 = 1025 and 2054 * 0.25 = 513.5 are fp16 numbers
+    x2 = np.array([[2050.0, 2054.0]], dtype=np.float16)
+    out = oracle.scale_permute(x2, scale=np.array([0.5, 0.25], dtype=np.float16))
+    assert float(out[0, 0]) == 1025.0 and float(out[0, 1]) == 513.5
+    # 1025 * 1.5 = 1537.5 and 1027 * 1.5 = 1540.5 lie halfway between fp16
+    # neighbours (spacing 1 in [1024, 2048)): ties go to the even one
+    h = np.array([[1025.0, 1027.0]], dtype=np.float16)
+    out = oracle.scale_permute(h, scale=np.array([1.5, 1.5], dtype=np.float16))
+    assert float(out[0, 0]) == 1538.0 and float(out[0, 1]) == 1540.0
+
+
+def test_permutation_gathers_channels():
+    g = np.random.default_rng(43)
+    x = g.standard_normal((4, 32)).astype(np.float16)
+    perm = g.permutation(32).astype(np.int32)
+    out = oracle.scale_permute(x, perm=perm)
+    np.testing.assert_array_equal(out, x[:, perm])          # out[:, j] = x[:, perm[j]]
+    assert not np.array_equal(out, x[:, np.argsort(perm)])  # not the scatter
+    s = (g.random(32) + 0.5).astype(np.float16)
+    both = oracle.scale_permute(x, scale=s, perm=perm)
+    ref = (x.astype(np.float64) * s.astype(np.float64)).astype(np.float16)[:, perm]
+    np.testing.assert_array_equal(both.view(np.uint16), ref.view(np.uint16))
+
+
+def test_permutation_must_be_a_permutation():
+    x = np.zeros((1, 8), dtype=np.float16)
+    for bad in ([0, 1, 2, 3, 4, 5, 6, 6], [0, 1, 2, 3, 4, 5, 6, 8], [-1, 1, 2, 3, 4, 5, 6, 7]):
+        with pytest.raises(ValueError):
+            oracle.scale_permute(x, perm=np.array(bad, dtype=np.int32))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_power_of_two_scale_keeps_codes_and_scales_s(bits):
+    g = np.random.default_rng(47)
+    x = g.standard_normal((5, 256)).astype(np.float16)
+    q0, s0 = oracle.rotate_quantize(x, 64, bits)
+    q1, s1 = oracle.rotate_quantize(x, 64, bits, scale=np.full(256, 0.25, np.float16))
+    np.testing.assert_array_equal(q0, q1)
+    np.testing.assert_array_equal(s1, s0 * np.float32(0.25))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_block_permutation_permutes_the_rotated_blocks(bits):
+    """Moving whole rotation blocks permutes the rotated blocks; the absmax is
+    over the whole row, so codes move with them and the scale is unchanged."""
+    g = np.random.default_rng(53)
+    b, nb = 32, 6
+    x = g.standard_normal((3, b * nb)).astype(np.float16)
+    order = g.permutation(nb)
+    perm = np.concatenate([np.arange(o * b, o * b + b) for o in order]).astype(np.int32)
+    q0, s0 = oracle.rotate_quantize(x, b, bits)
+    q1, s1 = oracle.rotate_quantize(x, b, bits, perm=perm)
+    np.testing.assert_array_equal(q1, q0[:, perm])
+    np.testing.assert_array_equal(s1, s0)
+
+
+def test_permuted_input_and_weights_give_the_same_product():
+    """With b = 1 (no mixing) the codes move with the channels, so permuting
+    the activations and the weights' columns alike leaves y unchanged."""
+    g = np.random.default_rng(59)
+    K, N = 64, 16
+    x = g.standard_normal((3, K)).astype(np.float16)
+    perm = g.permutation(K).astype(np.int32)
+    q, s = oracle.rotate_quantize(x, 1, 4)
+    qp, sp = oracle.rotate_quantize(x, 1, 4, perm=perm)
+    np.testing.assert_array_equal(qp, q[:, perm])
+    idx = g.integers(0, 16, (N, K)).astype(np.uint8)
+    cb = (g.standard_normal((N, 16)) * 0.02).astype(np.float16)
+    pack = lambda v: (v[:, 0::2] | (v[:, 1::2] << 4)).astype(np.uint8)
+    y, _, _ = oracle.lut_gemm(q, s, pack(idx), cb)
+    yp, _, _ = oracle.lut_gemm(qp, sp, pack(idx[:, perm]), cb)
+    np.testing.assert_allclose(yp, y, rtol=1e-12, atol=1e-15)
