@@ -100,6 +100,29 @@ CQ_API cq_status cq_rotate_quantize(const void *x, int64_t M, int64_t K, int32_t
                              int32_t act_bits, void *q_out, float *s_out, cq_stream_t stream);
 
 /*
+ * cq_rotate_quantize_ex -- cq_rotate_quantize with the online smoothing scale
+ * and the channel grouping applied to x first:
+ *   x'[m, j] = fp16( x[m, perm[j]] * scale[perm[j]] )   (round to nearest even
+ *              of the exact product), then x' is rotated and quantized.
+ * Passages: CodeQuant2 Figure 1 (rotation and scaling fused into the model)
+ * and Table 5 (SmoothQuant scaling); CodeQuant podcast transcript, "Summary"
+ * (the channels are reordered before clustering so that outliers spread over
+ * different groups -- here, over different rotation blocks).
+ *
+ * scale   fp16 [K] per-channel multiplier (the reciprocals of the smoothing
+ *         factors folded into the weights), or NULL for 1
+ * perm    int32 [K], the order in which the weights' K columns are packed: a
+ *         permutation of 0..K-1, or NULL for the identity.  A value outside
+ *         [0, K) is clamped into range (nothing is read outside the row) and
+ *         the result is then unspecified.
+ * The scaled values must be finite (|x * scale| < 65520).  Other arguments,
+ * requirements and errors as cq_rotate_quantize.
+ */
+CQ_API cq_status cq_rotate_quantize_ex(const void *x, int64_t M, int64_t K, int32_t had_block,
+                                       int32_t act_bits, const void *scale, const int32_t *perm,
+                                       void *q_out, float *s_out, cq_stream_t stream);
+
+/*
  * cq_lut_gemm -- LUT (codebook) product of quantized activations with
  * 4-bit-index weights.
  *
@@ -171,6 +194,7 @@ CQ_API cq_status cq_lut_gemm_noalloc(const void *q, const float *s_x, int64_t M,
  * MoE (or dense SwiGLU) FFN layer.
  *
  *   xq, s_x = rotate_quantize(x, had_block_h)              once per token
+ *             (after the optional smoothing scale / channel order of w)
  *   routing: per token the top_k largest router logits (descending, ties to
  *            the lower expert id); weights = softmax over the selected logits
  *            (renormalize = 1) or over all E logits (renormalize = 0)
@@ -216,6 +240,11 @@ typedef struct {
     const void *sh_gate_cb;      /* fp16 [n_shared, I_shared, 16] */
     const void *sh_up_cb;        /* fp16 [n_shared, I_shared, 16] */
     const void *sh_down_cb;      /* fp16 [n_shared, H, 16] */
+    /* online smoothing scale and channel order of the layer input x, as in
+     * cq_rotate_quantize_ex (NULL: none); the gate/up weights' H columns are
+     * packed in the order x_perm gives */
+    const void *x_scale;         /* fp16 [H] or NULL */
+    const int32_t *x_perm;       /* int32 [H] or NULL */
 } cq_moe_weights;
 
 /* Optional copies of intermediate results (any field may be NULL).

@@ -13,6 +13,8 @@ from pathlib import Path
 
 import torch
 
+from .packing import outlier_grouping_perm, permute_weight_columns  # noqa: F401
+
 _PKG = Path(__file__).resolve().parent
 LIB_PATH = _PKG / "libcq_b200.so"
 
@@ -20,7 +22,7 @@ LIB_PATH = _PKG / "libcq_b200.so"
 EXPORTS = ("cq_status_string", "cq_version", "cq_rotate_quantize", "cq_lut_gemm_workspace_size",
            "cq_lut_gemm", "cq_moe_ffn_workspace_size", "cq_moe_ffn", "cq_launch_count",
            "cq_timing_enable", "cq_timing_read", "cq_lut_gemm_noalloc", "cq_device_error",
-           "cq_timing_read_launches", "cq_selftest_wait_timeout")
+           "cq_timing_read_launches", "cq_selftest_wait_timeout", "cq_rotate_quantize_ex")
 
 CQ_OK, CQ_ERR_INVALID_ARGUMENT, CQ_ERR_UNSUPPORTED, CQ_ERR_WORKSPACE, CQ_ERR_CUDA = range(5)
 
@@ -49,7 +51,7 @@ class MoEDesc(ctypes.Structure):
 class MoEWeights(ctypes.Structure):
     _fields_ = [(n, _P) for n in ("gate_idx", "up_idx", "down_idx", "gate_cb", "up_cb", "down_cb",
                                   "sh_gate_idx", "sh_up_idx", "sh_down_idx", "sh_gate_cb",
-                                  "sh_up_cb", "sh_down_cb")]
+                                  "sh_up_cb", "sh_down_cb", "x_scale", "x_perm")]
 
 
 MOE_DEBUG_FIELDS = ("topk_ids", "topk_w", "counts", "offsets", "perm", "x_codes", "x_scales",
@@ -66,6 +68,8 @@ lib.cq_version.argtypes = []
 lib.cq_version.restype = ctypes.c_char_p
 lib.cq_rotate_quantize.argtypes = [_P, _I64, _I64, _I32, _I32, _P, _P, _P]
 lib.cq_rotate_quantize.restype = ctypes.c_int
+lib.cq_rotate_quantize_ex.argtypes = [_P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P]
+lib.cq_rotate_quantize_ex.restype = ctypes.c_int
 lib.cq_lut_gemm_workspace_size.argtypes = [_I64, _I64, _I64, _I32]
 lib.cq_lut_gemm_workspace_size.restype = _SZ
 lib.cq_lut_gemm.argtypes = [_P, _P, _I64, _I64, _I32, _P, _P, _I64, _P, _P, _P, _SZ, _P]
@@ -174,15 +178,22 @@ def _empty_codes(M, K, bits, device):
 
 
 def cq_rotate_quantize(x: torch.Tensor, had_block: int, act_bits: int, q_out=None, s_out=None,
-                       stream=None):
-    """x fp16 [M, K] (CUDA) -> (codes, scales fp32 [M]); see include/cq.h."""
+                       stream=None, scale=None, perm=None):
+    """x fp16 [M, K] (CUDA) -> (codes, scales fp32 [M]); see include/cq.h.
+    scale (fp16 [K]) / perm (int32 [K]): the online smoothing scale and
+    channel order (cq_rotate_quantize_ex)."""
     M, K = x.shape
     if q_out is None:
         q_out = _empty_codes(M, K, act_bits, x.device)
     if s_out is None:
         s_out = torch.empty((M,), dtype=torch.float32, device=x.device)
-    _check(lib.cq_rotate_quantize(_ptr(x), M, K, had_block, act_bits, _ptr(q_out), _ptr(s_out),
-                                  _stream(stream)), "cq_rotate_quantize")
+    if scale is None and perm is None:
+        _check(lib.cq_rotate_quantize(_ptr(x), M, K, had_block, act_bits, _ptr(q_out),
+                                      _ptr(s_out), _stream(stream)), "cq_rotate_quantize")
+    else:
+        _check(lib.cq_rotate_quantize_ex(_ptr(x), M, K, had_block, act_bits, _ptr(scale),
+                                         _ptr(perm), _ptr(q_out), _ptr(s_out), _stream(stream)),
+               "cq_rotate_quantize_ex")
     return q_out, s_out
 
 

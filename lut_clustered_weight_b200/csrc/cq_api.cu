@@ -287,6 +287,24 @@ cq_status cq_rotate_quantize(const void *x, int64_t M, int64_t K, int32_t had_bl
                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
+cq_status cq_rotate_quantize_ex(const void *x, int64_t M, int64_t K, int32_t had_block,
+                                int32_t act_bits, const void *scale, const int32_t *perm,
+                                void *q_out, float *s_out, cq_stream_t stream) {
+    if (M < 0 || K <= 0) return CQ_ERR_INVALID_ARGUMENT;
+    if (act_bits != 4 && act_bits != 8) return CQ_ERR_INVALID_ARGUMENT;
+    if (!is_pow2(had_block) || K % had_block) return CQ_ERR_INVALID_ARGUMENT;
+    if (M > 0 && (!x || !q_out || !s_out)) return CQ_ERR_INVALID_ARGUMENT;
+    if (!aligned16(x) || !aligned16(q_out) || !aligned16(s_out) || !aligned16(scale) ||
+        !aligned16(perm))
+        return CQ_ERR_INVALID_ARGUMENT;
+    if (had_block > 8192 || K % 8 || K > kMaxK || M > INT32_MAX) return CQ_ERR_UNSUPPORTED;
+    if (M == 0) return CQ_OK;
+    return cuda_status(launch_rotate_quantize(x, K, M, (int)K, ilog2(had_block), act_bits, q_out,
+                                              code_bytes(K, act_bits), s_out,
+                                              reinterpret_cast<cudaStream_t>(stream), scale,
+                                              perm));
+}
+
 size_t cq_lut_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t act_bits) {
     (void)act_bits;
     if (M <= 0 || N <= 0 || K <= 0) return 0;
@@ -329,7 +347,8 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
     if (cs != CQ_OK) return cs;
     if (!w || (T > 0 && (!x || !out))) return CQ_ERR_INVALID_ARGUMENT;
     if ((d->E > 0) != (router_logits != nullptr)) return CQ_ERR_INVALID_ARGUMENT;
-    if (!aligned16(x) || !aligned16(router_logits) || !aligned16(out) || !aligned16(workspace))
+    if (!aligned16(x) || !aligned16(router_logits) || !aligned16(out) || !aligned16(workspace) ||
+        !aligned16(w->x_scale) || !aligned16(w->x_perm))
         return CQ_ERR_INVALID_ARGUMENT;
     if (d->E > 0) {
         const void *ps[] = {w->gate_idx, w->up_idx, w->down_idx, w->gate_cb, w->up_cb, w->down_cb};
@@ -375,7 +394,7 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
     const int64_t ldx = code_bytes(m.H, m.bits), ldh = code_bytes(m.Imax, m.bits);
 
     cudaError_t e = launch_rotate_quantize(x, m.H, T, (int)m.H, ilog2(d->had_block_h), m.bits, xq,
-                                           ldx, sx, st);
+                                           ldx, sx, st, w->x_scale, w->x_perm);
     if (e == cudaSuccess && m.E > 0)
         e = launch_route(router_logits, (int)T, (int)m.E, (int)m.k, d->renormalize, m.tile_rows,
                          ids, tw, counts, offsets, perm, inv, tiles, tgrp, m.max_tiles_r, st);

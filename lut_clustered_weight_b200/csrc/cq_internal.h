@@ -12,10 +12,13 @@ namespace cq {
 // ---------------------------------------------------------------- rotate + quantize
 constexpr int kMaxK = 16384;
 
-// x fp16 rows with stride ldx (elements); one CTA per row.
+// x fp16 rows with stride ldx (elements); one CTA per row.  scale (fp16 [K])
+// and perm (int32 [K]) are optional: row element j is fp16(x[perm[j]] *
+// scale[perm[j]]) before the rotation.
 cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K, int log2b,
                                    int bits, void *q, int64_t ldq_bytes, float *s,
-                                   cudaStream_t st);
+                                   cudaStream_t st, const void *scale = nullptr,
+                                   const int32_t *perm = nullptr);
 
 // ---------------------------------------------------------------- LUT GEMM
 // Token-row -> code-row mapping used by the grouped GEMM.

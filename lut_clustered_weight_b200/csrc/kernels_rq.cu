@@ -74,11 +74,42 @@ CQ_DEV void cluster_pos(int &cs, int &rank) {
     }
 }
 
+// Loads elements [e0, e0 + n) of one x row into buf as fp64: plainly, or
+// (scale / perm non-NULL) as fp16(x[perm[j]] * scale[perm[j]]) -- the online
+// smoothing scale and channel grouping.  fp16 x fp16 is exact in fp32 and
+// __float2half_rn rounds it to nearest even.  A permutation value outside
+// [0, K) is clamped into range, so no load can leave the row.
+CQ_DEV void load_x_part(double *buf, const __half *__restrict__ xr, int e0, int n, int K,
+                        const __half *__restrict__ scale, const int32_t *__restrict__ perm,
+                        int tid, int nthreads) {
+    if (!scale && !perm) {
+        for (int i = tid; i < n / 8; i += nthreads) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(xr + e0 + 8 * i);
+            const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const float2 f = __half22float2(h[j]);
+                buf[8 * i + 2 * j] = (double)f.x;
+                buf[8 * i + 2 * j + 1] = (double)f.y;
+            }
+        }
+        return;
+    }
+    for (int i = tid; i < n; i += nthreads) {
+        const int j = e0 + i;
+        const int c = perm ? (int)min((unsigned)perm[j], (unsigned)(K - 1)) : j;
+        float v = __half2float(xr[c]);
+        if (scale) v = __half2float(__float2half_rn(v * __half2float(scale[c])));
+        buf[i] = (double)v;
+    }
+}
+
 // ------------------------------------------------------------------ x rows
 template <bool CLUSTER>
 __global__ void __launch_bounds__(kRqThreads)
 k_rq_x(const __half *__restrict__ x, int64_t ldx, int K, int log2b, int bits,
-       uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s) {
+       uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s,
+       const __half *__restrict__ scale, const int32_t *__restrict__ perm) {
     extern __shared__ __align__(16) double buf[];
     int cs, rank;
     griddep_wait();
@@ -86,17 +117,7 @@ k_rq_x(const __half *__restrict__ x, int64_t ldx, int K, int log2b, int bits,
     cluster_pos<CLUSTER>(cs, rank);
     const int64_t m = blockIdx.x / cs;
     const RowPart part = row_part(K, log2b, rank, cs);
-    const __half *xr = x + m * ldx + part.e0;
-    for (int i = threadIdx.x; i < part.n / 8; i += kRqThreads) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(xr + 8 * i);
-        const __half2 *h = reinterpret_cast<const __half2 *>(&v);
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const float2 f = __half22float2(h[j]);
-            buf[8 * i + 2 * j] = (double)f.x;
-            buf[8 * i + 2 * j + 1] = (double)f.y;
-        }
-    }
+    load_x_part(buf, x + m * ldx, part.e0, part.n, K, scale, perm, threadIdx.x, kRqThreads);
     __syncthreads();
     rq_finish<CLUSTER>(buf, part, log2b, bits, q + m * ldq, s + m);
 }
@@ -167,7 +188,8 @@ constexpr int kWarpRows = 4;
 
 __global__ void __launch_bounds__(kWarpRows * 32)
 k_rq_x_warp(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log2b, int bits,
-            uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s) {
+            uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s,
+            const __half *__restrict__ scale, const int32_t *__restrict__ perm) {
     extern __shared__ __align__(16) double wbuf[];
     griddep_wait();
     griddep_launch();
@@ -175,17 +197,7 @@ k_rq_x_warp(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log
     const int64_t m = (int64_t)blockIdx.x * kWarpRows + w;
     if (m >= M) return;
     double *buf = wbuf + (size_t)w * K;
-    const __half *xr = x + m * ldx;
-    for (int i = lane; i < K / 8; i += 32) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(xr + 8 * i);
-        const __half2 *h = reinterpret_cast<const __half2 *>(&v);
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const float2 f = __half22float2(h[j]);
-            buf[8 * i + 2 * j] = (double)f.x;
-            buf[8 * i + 2 * j + 1] = (double)f.y;
-        }
-    }
+    load_x_part(buf, x + m * ldx, 0, K, K, scale, perm, lane, 32);
     __syncwarp();
     const double A = warp_fwht_absmax(buf, K, log2b);
     warp_quantize_row(buf, K, log2b, bits, A, q + m * ldq, s + m);
@@ -271,20 +283,23 @@ static cudaError_t launch_clustered(Kern kern, int64_t rows, int cs, size_t smem
 }
 
 cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K, int log2b,
-                                   int bits, void *q, int64_t ldq, float *s, cudaStream_t st) {
+                                   int bits, void *q, int64_t ldq, float *s, cudaStream_t st,
+                                   const void *scale, const int32_t *perm) {
+    const __half *sc = reinterpret_cast<const __half *>(scale);
     if (M == 0) return cudaSuccess;
     if (use_warp_rows(M, K, log2b)) {
         const size_t smem = (size_t)kWarpRows * K * sizeof(double);
         count_launch();
         return launch_pdl(k_rq_x_warp, dim3((unsigned)((M + kWarpRows - 1) / kWarpRows)),
                           dim3(kWarpRows * 32), smem, st, 1, reinterpret_cast<const __half *>(x),
-                          ldx, M, K, log2b, bits, reinterpret_cast<uint8_t *>(q), ldq, s);
+                          ldx, M, K, log2b, bits, reinterpret_cast<uint8_t *>(q), ldq, s, sc,
+                          perm);
     }
     const int cs = cluster_size(M, K, log2b);
     auto kern = cs == 1 ? k_rq_x<false> : k_rq_x<true>;
     return launch_clustered(kern, M, cs, part_smem(K, log2b, cs), st,
                             reinterpret_cast<const __half *>(x), ldx, K, log2b, bits,
-                            reinterpret_cast<uint8_t *>(q), ldq, s);
+                            reinterpret_cast<uint8_t *>(q), ldq, s, sc, perm);
 }
 
 cudaError_t launch_swiglu_rq(const SwigluArgs &a, int64_t rows, cudaStream_t st) {

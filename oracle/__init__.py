@@ -296,7 +296,8 @@ def moe_ffn(inp, shape=None):
     method quantizes).  ``inp`` is a synth.MoEInputs.  Returns dict with
     out fp64 [T, H] and the intermediate routing tables."""
     s = shape or inp.shape
-    xq, sx = rotate_quantize(inp.x, s.had_block_h, s.act_bits)
+    xq, sx = rotate_quantize(inp.x, s.had_block_h, s.act_bits,
+                             scale=inp.extra.get("x_scale"), perm=inp.extra.get("x_perm"))
     T, H = s.T, s.H
     out = {}
     y_shared = None

@@ -46,6 +46,9 @@ def upload_weights(inp: synth.MoEInputs, dev):
         a = getattr(inp, n)
         if a is not None:
             w[n] = torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    for n in ("x_scale", "x_perm"):   # online smoothing scale / channel order of x
+        if inp.extra.get(n) is not None:
+            w[n] = torch.from_numpy(np.ascontiguousarray(inp.extra[n])).to(dev)
     return w
 
 
@@ -112,7 +115,9 @@ def check_moe(inp: synth.MoEInputs, g: dict, *, sample_rows=None, sample_tokens=
     bits = s.act_bits
     stats = {}
     # -- x codes and scales (bit-exact)
-    xq_ref, sx_ref = oracle.rotate_quantize(inp.x, s.had_block_h, bits)
+    xq_ref, sx_ref = oracle.rotate_quantize(inp.x, s.had_block_h, bits,
+                                            scale=inp.extra.get("x_scale"),
+                                            perm=inp.extra.get("x_perm"))
     xq = oracle.unpack_codes(g["x_codes"], s.H, bits)
     assert np.array_equal(xq, xq_ref), "x codes differ"
     assert np.array_equal(g["x_scales"].view(np.uint32), sx_ref.view(np.uint32)), "x scales differ"

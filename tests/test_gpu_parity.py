@@ -79,6 +79,45 @@ def test_rotate_quantize_exact_ties(cq):
         assert s.item() == sr[0]
 
 
+RQ_SP_CASES = [
+    # (M, K, b, bits, scale, perm): one CTA / cluster per row, and the
+    # warp-per-row kernel (many rows, b <= 256)
+    (3, 2560, 512, 4, True, True),
+    (2, 2048, 2048, 8, True, False),
+    (5, 9728, 256, 4, False, True),
+    (700, 1408, 128, 8, True, True),
+    (600, 2048, 256, 4, False, True),
+]
+
+
+@pytest.mark.parametrize("M,K,b,bits,use_scale,use_perm", RQ_SP_CASES)
+def test_rotate_quantize_scale_perm_bit_exact(cq, M, K, b, bits, use_scale, use_perm):
+    """Online smoothing scale and channel grouping ahead of the rotation."""
+    g = np.random.default_rng(M + K)
+    x = synth.activations(M, K, seed=2, name=f"rqsp{M}.{K}")
+    scale = (g.random(K) * 1.5 + 0.05).astype(np.float16) if use_scale else None
+    perm = g.permutation(K).astype(np.int32) if use_perm else None
+    dev = lambda a: None if a is None else torch.from_numpy(a).to(DEV)
+    q, s = cq.cq_rotate_quantize(dev(x), b, bits, scale=dev(scale), perm=dev(perm))
+    torch.cuda.synchronize()
+    qr, sr = oracle.rotate_quantize(x, b, bits, scale=scale, perm=perm)
+    assert np.array_equal(oracle.unpack_codes(q.cpu().numpy(), K, bits), qr)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), sr.view(np.uint32))
+
+
+def test_moe_with_smoothing_scale_and_channel_order(cq):
+    """The layer input's smoothing scale / channel order reach the x codes."""
+    shape = synth.MoEShape("moe_scaled_perm", H=256, I=192, E=8, top_k=2, n_shared=1, T=24,
+                           act_bits=4, had_block_h=64, had_block_i=64)
+    inp = synth.moe_inputs(shape, seed=3)
+    g = np.random.default_rng(5)
+    inp.extra["x_scale"] = (g.random(256) + 0.25).astype(np.float16)
+    inp.extra["x_perm"] = g.permutation(256).astype(np.int32)
+    res = run_moe(inp)
+    st = check_moe(inp, res, e2e=True)
+    assert st["e2e_rel_l2"] < 5e-2, st
+
+
 # ---------------------------------------------------------------------------
 # LUT GEMM
 
