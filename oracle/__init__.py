@@ -71,12 +71,14 @@ def lib():
         _lib.orc_unpack_int4.argtypes = [P, I64, I64, P]
         _lib.orc_pack_int4.argtypes = [P, I64, I64, P]
         _lib.orc_unpack_idx.argtypes = [P, I64, I64, P]
+        _lib.orc_unpack_idx_bits.argtypes = [P, I64, I64, I32, P]
+        _lib.orc_lut_gemm_nc.argtypes = [P, P, I64, I64, P, P, I32, I64, P, P]
         _lib.orc_lut_gemm.argtypes = [P, P, I64, I64, P, P, I64, P, P, P]
         _lib.orc_route.argtypes = [P, I64, I64, I64, I32, P, P, P, P, P]
         _lib.orc_swiglu.argtypes = [P, P, I64, P]
         _lib.orc_combine.argtypes = [P, P, I64, I64, I64, P, I64, P]
         for f in ("orc_hadamard_matrix", "orc_rotate", "orc_quantize", "orc_rotate_quantize",
-                  "orc_scale_permute",
+                  "orc_scale_permute", "orc_lut_gemm_nc",
                   "orc_lut_gemm", "orc_route"):
             getattr(_lib, f).restype = I32
     return _lib
@@ -228,6 +230,35 @@ def lut_gemm(q: np.ndarray, s: np.ndarray, w_idx: np.ndarray, codebook: np.ndarr
     _check(lib().orc_lut_gemm(_p(q), _p(s), M, K, _p(idx), _p(cb.view(np.uint16)), N,
                               _p(y), _p(mag), _p(S)), "lut_gemm")
     return y, mag, S
+
+
+def unpack_idx_bits(w_idx: np.ndarray, K: int, idx_bits: int) -> np.ndarray:
+    """b-bit packed indices uint8 [N, K*b/8] (least significant bit first)
+    -> uint8 [N, K]."""
+    w = _c(w_idx, np.uint8)
+    N = w.shape[0]
+    idx = np.empty((N, K), dtype=np.uint8)
+    lib().orc_unpack_idx_bits(_p(w), N, K, int(idx_bits), _p(idx))
+    return idx
+
+
+def lut_gemm_bits(q: np.ndarray, s: np.ndarray, w_idx: np.ndarray, idx_bits: int,
+                  codebook: np.ndarray):
+    """The LUT product with 2^idx_bits centroids per row (adaptive codebook
+    size): q int8 [M, K]; w_idx b-bit packed [N, K*b/8]; codebook fp16
+    [N, 2^b].  Returns (y fp64 [M, N], mag fp64 [M, N])."""
+    q = _c(q, np.int8)
+    s = _c(s, np.float32)
+    M, K = q.shape
+    idx = unpack_idx_bits(w_idx, K, idx_bits)
+    N = idx.shape[0]
+    nc = 1 << idx_bits
+    cb = _c(codebook, np.float16).reshape(N, nc)
+    y = np.empty((M, N), dtype=np.float64)
+    mag = np.empty((M, N), dtype=np.float64)
+    _check(lib().orc_lut_gemm_nc(_p(q), _p(s), M, K, _p(idx), _p(cb.view(np.uint16)), nc, N,
+                                 _p(y), _p(mag)), "lut_gemm_bits")
+    return y, mag
 
 
 def lut_tolerance(mag: np.ndarray) -> np.ndarray:

@@ -296,6 +296,29 @@ void orc_unpack_idx(const uint8_t *p, int64_t N, int64_t K, uint8_t *idx)
         }
 }
 
+/*
+ * Adaptive codebook size (CodeQuant2 page, abstract: codebook sizes adapted
+ * to each layer's quantization difficulty; Figure 3: adaptive cluster
+ * allocation): a layer's rows use 2^b centroids, b in {3, 4, 5}, and its
+ * indices are b-bit fields, least significant bit first: index k of row n
+ * occupies bits [b*k, b*k + b) of the row's byte string (bit i of byte j is
+ * bit 8j + i).  b = 4 is the nibble format above.
+ * p: uint8 [N, K*b/8]; idx: uint8 [N, K].
+ */
+void orc_unpack_idx_bits(const uint8_t *p, int64_t N, int64_t K, int b, uint8_t *idx)
+{
+    const int64_t rowbytes = K * b / 8;
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) {
+            int v = 0;
+            for (int i = 0; i < b; i++) {
+                const int64_t bit = k * b + i;
+                v |= ((p[n * rowbytes + bit / 8] >> (bit % 8)) & 1) << i;
+            }
+            idx[n * K + k] = (uint8_t)v;
+        }
+}
+
 /* ------------------------------------------------------------------------ */
 /* LUT product                                                               */
 
@@ -330,6 +353,38 @@ int orc_lut_gemm(const int8_t *q, const float *s, int64_t M, int64_t K,
             if (S)
                 for (int c = 0; c < 16; c++)
                     S[(m * N + n) * 16 + c] = (int32_t)sums[c];
+        }
+    }
+    return ORC_OK;
+}
+
+/*
+ * The LUT product with per-row codebooks of nc centroids (nc = 2^b):
+ *   y[m,n]   = s[m] * sum_k C[n, idx[n,k]] * q[m,k]      (fp64)
+ *   mag[m,n] = |s[m]| * sum_k |C[n, idx[n,k]] * q[m,k]|
+ * q: int8 [M, K]; s: fp32 [M]; idx: uint8 [N, K] (0..nc-1); cb: fp16 bits [N, nc].
+ */
+int orc_lut_gemm_nc(const int8_t *q, const float *s, int64_t M, int64_t K,
+                    const uint8_t *idx, const uint16_t *cb, int nc, int64_t N,
+                    double *y, double *mag)
+{
+    if (nc < 1 || nc > 256)
+        return ORC_EINVAL;
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t n = 0; n < N; n++) {
+        double C[256];
+        for (int c = 0; c < nc; c++)
+            C[c] = orc_f16_to_f64(cb[n * nc + c]);
+        for (int64_t m = 0; m < M; m++) {
+            double acc = 0.0, am = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                const double w = C[idx[n * K + k] % nc];
+                const double t = w * (double)q[m * K + k];
+                acc += t;
+                am += fabs(t);
+            }
+            y[m * N + n] = (double)s[m] * acc;
+            mag[m * N + n] = fabs((double)s[m]) * am;
         }
     }
     return ORC_OK;

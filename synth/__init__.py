@@ -134,10 +134,23 @@ def pack_nibbles(v: np.ndarray) -> np.ndarray:
     return (v[..., 0::2] & 0xF) | ((v[..., 1::2] & 0xF) << 4)
 
 
-def lut_weights(N: int, K: int, *, seed: int, name: str) -> tuple[np.ndarray, np.ndarray]:
-    """(w_idx uint8 [N, K/2] packed, codebook fp16 [N, 16]) for one linear."""
-    idx, cb = kmeans_codebook(raw_weights(N, K, seed=seed, name=name))
-    return pack_nibbles(idx), cb
+def pack_bits(v: np.ndarray, bits: int) -> np.ndarray:
+    """uint8 [..., K] values below 2^bits -> uint8 [..., K*bits/8]: element k
+    in bits [bits*k, bits*k + bits), least significant bit first (bits = 4 is
+    pack_nibbles)."""
+    v = np.asarray(v, dtype=np.uint8)
+    planes = ((v[..., :, None] >> np.arange(bits, dtype=np.uint8)) & 1).astype(np.uint8)
+    flat = planes.reshape(v.shape[:-1] + (v.shape[-1] * bits,))
+    return np.packbits(flat, axis=-1, bitorder="little")
+
+
+def lut_weights(N: int, K: int, *, seed: int, name: str,
+                idx_bits: int = 4) -> tuple[np.ndarray, np.ndarray]:
+    """(w_idx packed uint8 [N, K*b/8], codebook fp16 [N, 2^b]) for one linear
+    with 2^idx_bits centroids per row (16 by default)."""
+    idx, cb = kmeans_codebook(raw_weights(N, K, seed=seed, name=name),
+                              n_centroids=1 << idx_bits)
+    return (pack_nibbles(idx) if idx_bits == 4 else pack_bits(idx, idx_bits)), cb
 
 
 # ---------------------------------------------------------------------------

@@ -529,3 +529,90 @@ def test_permuted_input_and_weights_give_the_same_product():
     y, _, _ = oracle.lut_gemm(q, s, pack(idx), cb)
     yp, _, _ = oracle.lut_gemm(qp, sp, pack(idx[:, perm]), cb)
     np.testing.assert_allclose(yp, y, rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# adaptive codebook size: 8 / 16 / 32 centroids, 3 / 4 / 5-bit indices
+
+
+def _np_unpack_bits(p, K, b):
+    """Independent reading of the b-bit format: index k = bits [b*k, b*k+b),
+    least significant first, via numpy's little-endian bit unpacking."""
+    bits = np.unpackbits(np.asarray(p, dtype=np.uint8), axis=-1, bitorder="little")
+    bits = bits[..., : K * b].reshape(p.shape[:-1] + (K, b)).astype(np.int64)
+    return (bits << np.arange(b)).sum(axis=-1).astype(np.uint8)
+
+
+@pytest.mark.parametrize("b", [3, 4, 5])
+def test_bit_packed_indices_unpack(b):
+    import synth
+    g = np.random.default_rng(60 + b)
+    idx = g.integers(0, 2 ** b, (7, 96)).astype(np.uint8)
+    p = synth.pack_bits(idx, b)
+    assert p.shape == (7, 96 * b // 8)
+    np.testing.assert_array_equal(_np_unpack_bits(p, 96, b), idx)
+    np.testing.assert_array_equal(oracle.unpack_idx_bits(p, 96, b), idx)
+    if b == 4:  # the 4-bit case is the nibble format (element 2j in the low nibble)
+        np.testing.assert_array_equal(p, (idx[:, 0::2] | (idx[:, 1::2] << 4)).astype(np.uint8))
+
+
+@pytest.mark.parametrize("b", [3, 5])
+def test_lut_gemm_bits_dense_dequant_matmul(b):
+    import synth
+    g = np.random.default_rng(70 + b)
+    M, K, N = 4, 96, 6
+    q = g.integers(-7, 8, (M, K)).astype(np.int8)
+    s = (g.random(M) * 0.1 + 0.01).astype(np.float32)
+    idx = g.integers(0, 2 ** b, (N, K)).astype(np.uint8)
+    cb = (g.standard_normal((N, 2 ** b)) * 0.05).astype(np.float16)
+    y, mag = oracle.lut_gemm_bits(q, s, synth.pack_bits(idx, b), b, cb)
+    W = np.take_along_axis(cb.astype(np.float64), idx.astype(np.int64), axis=1)
+    np.testing.assert_allclose(y, s.astype(np.float64)[:, None] * (q.astype(np.float64) @ W.T),
+                               rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(mag, np.abs(s.astype(np.float64))[:, None] *
+                               (np.abs(q.astype(np.float64)) @ np.abs(W).T), rtol=1e-12)
+
+
+@pytest.mark.parametrize("b", [3, 5])
+def test_lut_gemm_bits_all_index_pairs_exact(b):
+    """Every pair of indices at the first two positions (a row of K = 8, so
+    that it fills whole bytes; the other codes are zero), against exact
+    rationals."""
+    import synth
+    nc = 2 ** b
+    g = np.random.default_rng(80 + b)
+    cb = (g.standard_normal((1, nc)) * 0.3).astype(np.float16)
+    q = np.array([[3, -5, 0, 0, 0, 0, 0, 0]], dtype=np.int8)
+    s = np.array([0.125], dtype=np.float32)
+    fill = g.integers(0, nc, 6)
+    pairs = np.array([(i, j, *fill) for i in range(nc) for j in range(nc)], dtype=np.uint8)
+    cbs = np.repeat(cb, len(pairs), axis=0)
+    y, _ = oracle.lut_gemm_bits(q, s, synth.pack_bits(pairs, b), b, cbs)
+    for r, (i, j) in enumerate(pairs[:, :2]):
+        exact = Fraction(0.125) * (Fraction(float(cb[0, i])) * 3 + Fraction(float(cb[0, j])) * -5)
+        assert y[0, r] == float(exact)
+
+
+def test_lut_gemm_bits_4_agrees_with_the_16_centroid_routine():
+    g = np.random.default_rng(90)
+    q, s, idx, w_idx, cb = _rand_lut(g, 3, 64, 5)
+    y16, mag16, _ = oracle.lut_gemm(q, s, w_idx, cb)
+    y4, mag4 = oracle.lut_gemm_bits(q, s, w_idx, 4, cb)
+    np.testing.assert_array_equal(y4, y16)
+    np.testing.assert_array_equal(mag4, mag16)
+
+
+@pytest.mark.parametrize("b", [3, 5])
+def test_lut_gemm_bits_uniform_grid_is_an_integer_gemm(b):
+    import synth
+    nc = 2 ** b
+    g = np.random.default_rng(95 + b)
+    M, K, N = 3, 64, 4
+    q = g.integers(-127, 128, (M, K)).astype(np.int8)
+    s = np.ones(M, dtype=np.float32)
+    idx = g.integers(0, nc, (N, K)).astype(np.uint8)
+    delta = 2.0 ** -6
+    cb = np.tile(((np.arange(nc) - nc // 2) * delta).astype(np.float16), (N, 1))
+    y, _ = oracle.lut_gemm_bits(q, s, synth.pack_bits(idx, b), b, cb)
+    ref = (q.astype(np.int64) @ (idx.astype(np.int64) - nc // 2).T) * delta
+    np.testing.assert_array_equal(y, ref)
