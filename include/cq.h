@@ -155,6 +155,32 @@ CQ_API cq_status cq_lut_gemm(const void *q, const float *s_x, int64_t M, int64_t
                       cq_stream_t stream);
 
 /*
+ * cq_lut_gemm_ex -- cq_lut_gemm with a per-layer codebook size: 2^idx_bits
+ * centroids per output row, idx_bits in {3, 4, 5} (8, 16 or 32 centroids).
+ * Passages: CodeQuant2 abstract (codebook sizes adapted to each layer's
+ * quantization difficulty) and Figure 3 (adaptive cluster allocation).
+ *
+ *   y[m,n] = s_x[m] * sum_k C[n, I[n,k]] * q[m,k],   I[n,k] < 2^idx_bits
+ *
+ * w_idx      uint8 [N, K*idx_bits/8]: index k of row n occupies bits
+ *            [idx_bits*k, idx_bits*k + idx_bits) of the row's byte string,
+ *            least significant bit first (bit i of byte j is bit 8j + i).
+ *            idx_bits = 4 is cq_lut_gemm's nibble format.
+ * codebook   fp16 [N, 2^idx_bits]
+ * idx_bits = 4 runs exactly cq_lut_gemm (same kernels, same results); 3 and 5
+ * run a dedicated mma.sync kernel.  The error bound, the other arguments and
+ * the requirements (K % 32 == 0, N % 64 == 0) are those of cq_lut_gemm; the
+ * workspace is sized by cq_lut_gemm_ex_workspace_size.  Other idx_bits:
+ * CQ_ERR_UNSUPPORTED.
+ */
+CQ_API size_t cq_lut_gemm_ex_workspace_size(int64_t M, int64_t N, int64_t K, int32_t act_bits,
+                                            int32_t idx_bits);
+CQ_API cq_status cq_lut_gemm_ex(const void *q, const float *s_x, int64_t M, int64_t K,
+                                int32_t act_bits, const uint8_t *w_idx, int32_t idx_bits,
+                                const void *codebook, int64_t N, float *y, void *workspace,
+                                size_t workspace_bytes, cq_stream_t stream);
+
+/*
  * cq_lut_gemm_noalloc -- cq_lut_gemm for callers that cannot allocate device
  * memory.  The pages have no counterpart: this is a deployment variant.
  *
@@ -304,7 +330,8 @@ CQ_API cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *ro
 enum cq_kernel_kind {
     CQ_KERNEL_LUT_MMA = 0, /* mma.sync kernel, register / shared lookup tables */
     CQ_KERNEL_LUT_TC = 1,  /* tcgen05 kernel for wide token tiles (> 32 rows per group) */
-    CQ_KERNEL_LUT_TS = 2   /* tcgen05 decode kernel (<= 32 rows per group): pair tables */
+    CQ_KERNEL_LUT_TS = 2,  /* tcgen05 decode kernel (<= 32 rows per group): pair tables */
+    CQ_KERNEL_LUT_VB = 3   /* mma.sync kernel for 3- / 5-bit indices (cq_lut_gemm_ex) */
 };
 CQ_API int64_t cq_launch_count(void);
 

@@ -22,7 +22,8 @@ LIB_PATH = _PKG / "libcq_b200.so"
 EXPORTS = ("cq_status_string", "cq_version", "cq_rotate_quantize", "cq_lut_gemm_workspace_size",
            "cq_lut_gemm", "cq_moe_ffn_workspace_size", "cq_moe_ffn", "cq_launch_count",
            "cq_timing_enable", "cq_timing_read", "cq_lut_gemm_noalloc", "cq_device_error",
-           "cq_timing_read_launches", "cq_selftest_wait_timeout", "cq_rotate_quantize_ex")
+           "cq_timing_read_launches", "cq_selftest_wait_timeout", "cq_rotate_quantize_ex",
+           "cq_lut_gemm_ex_workspace_size", "cq_lut_gemm_ex")
 
 CQ_OK, CQ_ERR_INVALID_ARGUMENT, CQ_ERR_UNSUPPORTED, CQ_ERR_WORKSPACE, CQ_ERR_CUDA = range(5)
 
@@ -74,6 +75,10 @@ lib.cq_lut_gemm_workspace_size.argtypes = [_I64, _I64, _I64, _I32]
 lib.cq_lut_gemm_workspace_size.restype = _SZ
 lib.cq_lut_gemm.argtypes = [_P, _P, _I64, _I64, _I32, _P, _P, _I64, _P, _P, _P, _SZ, _P]
 lib.cq_lut_gemm.restype = ctypes.c_int
+lib.cq_lut_gemm_ex_workspace_size.argtypes = [_I64, _I64, _I64, _I32, _I32]
+lib.cq_lut_gemm_ex_workspace_size.restype = _SZ
+lib.cq_lut_gemm_ex.argtypes = [_P, _P, _I64, _I64, _I32, _P, _I32, _P, _I64, _P, _P, _SZ, _P]
+lib.cq_lut_gemm_ex.restype = ctypes.c_int
 lib.cq_moe_ffn_workspace_size.argtypes = [ctypes.POINTER(MoEDesc), _I64]
 lib.cq_moe_ffn_workspace_size.restype = _SZ
 lib.cq_moe_ffn.argtypes = [ctypes.POINTER(MoEDesc), _P, _P, _I64, ctypes.POINTER(MoEWeights), _P,
@@ -123,7 +128,7 @@ def cq_selftest_wait_timeout(stream=None) -> None:
     _check(lib.cq_selftest_wait_timeout(_stream(stream)), "cq_selftest_wait_timeout")
 
 
-KERNEL_KINDS = {0: "k_lut_mma", 1: "k_lut_tc", 2: "k_lut_ts"}   # cq_kernel_kind
+KERNEL_KINDS = {0: "k_lut_mma", 1: "k_lut_tc", 2: "k_lut_ts", 3: "k_lut_vb"}   # cq_kernel_kind
 
 
 def cq_timing_read_launches(cap: int = 1 << 16) -> list[tuple[str, float]]:
@@ -223,6 +228,25 @@ def cq_lut_gemm(q: torch.Tensor, s_x: torch.Tensor, K: int, act_bits: int, w_idx
                            _ptr(y), _ptr(centroid_sums if want_S else None), _ptr(workspace), wb,
                            _stream(stream)), "cq_lut_gemm")
     return (y, centroid_sums) if want_S else y
+
+
+def cq_lut_gemm_ex(q: torch.Tensor, s_x: torch.Tensor, K: int, act_bits: int, w_idx: torch.Tensor,
+                   idx_bits: int, codebook: torch.Tensor, y=None, workspace=None, stream=None):
+    """cq_lut_gemm with 2^idx_bits centroids per row (idx_bits 3, 4, 5); w_idx
+    uint8 [N, K*idx_bits/8], codebook fp16 [N, 2^idx_bits]; see include/cq.h."""
+    M = s_x.shape[0]
+    N = w_idx.shape[0]
+    dev = w_idx.device
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    nb = int(lib.cq_lut_gemm_ex_workspace_size(M, N, K, act_bits, idx_bits))
+    if workspace is None and nb:
+        workspace = torch.empty((nb,), dtype=torch.uint8, device=dev)
+    wb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.cq_lut_gemm_ex(_ptr(q), _ptr(s_x), M, K, act_bits, _ptr(w_idx), idx_bits,
+                              _ptr(codebook), N, _ptr(y), _ptr(workspace), wb, _stream(stream)),
+           "cq_lut_gemm_ex")
+    return y
 
 
 NOALLOC_SCRATCH_BYTES = 4 << 20

@@ -335,6 +335,58 @@ cq_status cq_lut_gemm(const void *q, const float *s_x, int64_t M, int64_t K, int
     return cuda_status(e);
 }
 
+size_t cq_lut_gemm_ex_workspace_size(int64_t M, int64_t N, int64_t K, int32_t act_bits,
+                                     int32_t idx_bits) {
+    if (idx_bits == 4) return cq_lut_gemm_workspace_size(M, N, K, act_bits);
+    if ((idx_bits != 3 && idx_bits != 5) || M <= 0 || N <= 0 || K <= 0 || N % 64 || K % 32 ||
+        K > (int64_t(1) << 30) || N > (int64_t(1) << 30) || M > (int64_t(1) << 30))
+        return 0;
+    const LutPlan P = plan_lut_vb((int)M, (int)N, (int)K, idx_bits);
+    return align256((size_t)P.splits * M * N * sizeof(float));
+}
+
+cq_status cq_lut_gemm_ex(const void *q, const float *s_x, int64_t M, int64_t K, int32_t act_bits,
+                         const uint8_t *w_idx, int32_t idx_bits, const void *codebook, int64_t N,
+                         float *y, void *workspace, size_t workspace_bytes, cq_stream_t stream) {
+    if (idx_bits == 4)
+        return cq_lut_gemm(q, s_x, M, K, act_bits, w_idx, codebook, N, y, nullptr, workspace,
+                           workspace_bytes, stream);
+    if (idx_bits != 3 && idx_bits != 5) return CQ_ERR_UNSUPPORTED;
+    if (M < 0 || K <= 0 || N <= 0) return CQ_ERR_INVALID_ARGUMENT;
+    if (act_bits != 4 && act_bits != 8) return CQ_ERR_INVALID_ARGUMENT;
+    if (K % 2) return CQ_ERR_INVALID_ARGUMENT;
+    if (!w_idx || !codebook || !y || (M > 0 && (!q || !s_x))) return CQ_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(s_x) || !aligned16(w_idx) || !aligned16(codebook) ||
+        !aligned16(y) || !aligned16(workspace))
+        return CQ_ERR_INVALID_ARGUMENT;
+    if (K % 32 || N % 64 || K > (int64_t(1) << 30) || N > (int64_t(1) << 30) ||
+        M > (int64_t(1) << 30))
+        return CQ_ERR_UNSUPPORTED;
+    if (M == 0) return CQ_OK;
+    const LutPlan P = plan_lut_vb((int)M, (int)N, (int)K, idx_bits);
+    const size_t ws = align256((size_t)P.splits * M * N * sizeof(float));
+    if (!workspace || workspace_bytes < ws) return CQ_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    LutLaunch L{};
+    L.codes = reinterpret_cast<const uint8_t *>(q);
+    L.ld_codes = code_bytes(K, act_bits);
+    L.scales = s_x;
+    L.act_bits = act_bits;
+    L.K = (int)K;
+    L.map_mode = kMapIdentity;
+    L.G = 1;
+    L.uniform_rows = (int)M;
+    L.idx0 = w_idx;
+    L.cb0 = codebook;
+    L.N = (int)N;
+    L.out = reinterpret_cast<float *>(workspace);
+    L.out_split_stride = M * N;
+    L.out_row_stride = N;
+    cudaError_t e = launch_lut_vb(L, P, idx_bits, st);
+    if (e == cudaSuccess) e = launch_reduce_plain(L.out, P, M, N, s_x, y, st);
+    return cuda_status(e);
+}
+
 size_t cq_moe_ffn_workspace_size(const cq_moe_desc *d, int64_t T) {
     if (check_moe_desc(d, T) != CQ_OK) return 0;
     return plan_moe(d, T).total;

@@ -33,6 +33,13 @@ CQ_DEV uint4 ldg_stream(const void *p) {
     return v;
 }
 
+// 32-bit shared-memory load at a shared-window address.
+CQ_DEV uint32_t lds32(uint32_t saddr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(saddr));
+    return v;
+}
+
 CQ_DEV float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

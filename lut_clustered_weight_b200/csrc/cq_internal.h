@@ -186,6 +186,11 @@ int read_device_error();
 enum LutPath : int { kPathAuto = 0, kPathMma = 1, kPathTc = 2, kPathTs = 3 };
 LutPath lut_path();
 
+// LUT GEMM with 3- or 5-bit indices (8 or 32 centroids per row), uniform
+// token rows (identity map): plan and launch; partial sums as launch_lut.
+LutPlan plan_lut_vb(int M, int N, int K, int idx_bits);
+cudaError_t launch_lut_vb(const LutLaunch &L, const LutPlan &P, int idx_bits, cudaStream_t st);
+
 // y[m, n] = s[m] * sum_{s < n(m, n)} part[s][m][n]
 cudaError_t launch_reduce_plain(const float *part, const LutPlan &P, int64_t M, int64_t N,
                                 const float *s, float *y, cudaStream_t st);

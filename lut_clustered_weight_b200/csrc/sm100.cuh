@@ -78,12 +78,6 @@ CQ_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t max_sleep_ns = 25
     return false;
 }
 
-// 32-bit shared-memory load at a shared-window address.
-CQ_DEV uint32_t lds32(uint32_t saddr) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(saddr));
-    return v;
-}
 
 // ---------------------------------------------------------------- cp.async (per thread)
 // 16-byte async copy; src_bytes = 0 writes zeros (nothing is read).
