@@ -520,6 +520,57 @@ def lut_timed_launches(cq, step, steps):
     return cq.cq_timing_read_launches()
 
 
+def lut_alg_bytes_bits(M, N, K, bits, idx_bits):
+    """Algorithmic bytes of one LUT product with 2^idx_bits centroids per row."""
+    return N * K * idx_bits // 8 + 2 * (1 << idx_bits) * N + M * K * bits // 8 + 4 * M + 4 * M * N
+
+
+def measure_codebook_sizes(cq, args, dev, peaks, copies=3):
+    """GB/s of the LUT GEMM per codebook size (8 / 16 / 32 centroids per row)
+    on the Qwen3-4B-shaped FFN linears (gate||up 2560 -> 19456 and down
+    9728 -> 2560) at M = 1 and 16, A4: every launch CUDA-event timed, each
+    call on its own weight copy (copies x the shapes > the 126 MB L2).  The
+    kernels' work does not depend on the values: indices are uniform random,
+    codebooks sorted N(0, 0.02^2) draws."""
+    import torch
+    peak_gbs = peaks[0]
+    g = np.random.default_rng(0)
+    out = {}
+    for b in (3, 4, 5):
+        calls = []
+        for (M, K, N) in [(1, 2560, 19456), (1, 9728, 2560), (16, 2560, 19456), (16, 9728, 2560)]:
+            q = torch.from_numpy(g.integers(0, 256, (M, K // 2), dtype=np.uint8)).to(dev)
+            sx = torch.full((M,), 1e-2, dtype=torch.float32, device=dev)
+            for _ in range(copies):
+                w = torch.from_numpy(g.integers(0, 256, (N, K * b // 8), dtype=np.uint8)).to(dev)
+                cbk = torch.from_numpy(np.sort(g.standard_normal((N, 1 << b)) * 0.02, axis=1)
+                                       .astype(np.float16)).to(dev)
+                y = torch.empty((M, N), dtype=torch.float32, device=dev)
+                nb = cq.cq_lut_gemm_ex_workspace_size(M, N, K, 4, b)
+                ws = torch.empty((max(nb, 1),), dtype=torch.uint8, device=dev)
+                calls.append((q, sx, K, w, cbk, y, ws, lut_alg_bytes_bits(M, N, K, 4, b)))
+
+        def step():
+            for (q, sx, K, w, cbk, y, ws, _) in calls:
+                cq.cq_lut_gemm_ex(q, sx, K, 4, w, b, cbk, y=y, workspace=ws)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        launches = lut_timed_launches(cq, step, args.steps)
+        assert len(launches) == args.steps * len(calls)
+        ms = sum(m for _, m in launches)
+        nbytes = args.steps * sum(c[-1] for c in calls)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[str(1 << b)] = {"idx_bits": b, "kernel": sorted({k for k, _ in launches}),
+                            "achieved": gbs, "unit": "GB/s", "peak": peak_gbs,
+                            "frac": gbs / peak_gbs, "launches_timed": len(launches),
+                            "avg_launch_us": 1e3 * ms / len(launches),
+                            "alg_bytes_per_step": nbytes // args.steps}
+        del calls
+        torch.cuda.empty_cache()
+    return out
+
+
 def measure(cq, name, args, dev, stream, dist, world, peaks):
     """One workload: the step resident (graph replay), the LUT kernel launch by
     launch, and the step end to end from host buffers.  Returns its block."""
@@ -618,6 +669,8 @@ def measure(cq, name, args, dev, stream, dist, world, peaks):
         bf16 = bf16_dense_context(shapes, dev, stream, args.steps, args.warmup, dist, world)
         bf16["speedup_of_value"] = value / bf16["value"]
         block["bf16_context"] = bf16
+    if name == LINEAR and not args.no_codebook_sizes:
+        block["codebook_sizes"] = measure_codebook_sizes(cq, args, dev, peaks)
     if use_graph:
         del graph
     del calls
@@ -638,6 +691,8 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--no-bf16", action="store_true", help="skip the torch bf16 context leg")
+    ap.add_argument("--no-codebook-sizes", action="store_true",
+                    help="skip the GB/s-per-codebook-size leg (8 / 16 / 32 centroids)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     headline = HEADLINE if args.workload == "all" else args.workload
@@ -705,8 +760,9 @@ def main():
                           "into mma.sync or tcgen05 kind::f16 (tensor memory A operand) with "
                           "fp32 accumulation; rotation exact in fp64",
         }
-        if "bf16_context" in head:
-            line["bf16_context"] = head["bf16_context"]
+        for extra in ("bf16_context", "codebook_sizes"):
+            if extra in head:
+                line[extra] = head[extra]
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

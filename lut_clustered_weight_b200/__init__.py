@@ -230,6 +230,10 @@ def cq_lut_gemm(q: torch.Tensor, s_x: torch.Tensor, K: int, act_bits: int, w_idx
     return (y, centroid_sums) if want_S else y
 
 
+def cq_lut_gemm_ex_workspace_size(M: int, N: int, K: int, act_bits: int, idx_bits: int) -> int:
+    return int(lib.cq_lut_gemm_ex_workspace_size(M, N, K, act_bits, idx_bits))
+
+
 def cq_lut_gemm_ex(q: torch.Tensor, s_x: torch.Tensor, K: int, act_bits: int, w_idx: torch.Tensor,
                    idx_bits: int, codebook: torch.Tensor, y=None, workspace=None, stream=None):
     """cq_lut_gemm with 2^idx_bits centroids per row (idx_bits 3, 4, 5); w_idx
