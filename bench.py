@@ -571,6 +571,124 @@ def measure_codebook_sizes(cq, args, dev, peaks, copies=3):
     return out
 
 
+def decoder_layer_vs_bf16(cq, args, dev, stream, dist, world, ctx=1024, n_layers=4):
+    """Decode step of n_layers Qwen3-4B-shaped decoder layers (hidden 2560, 32
+    query / 8 key-value heads of 128, intermediate 9728, a KV cache of ctx
+    tokens per sequence, M sequences decoding one token each), once with the
+    linears as this library's LUT layers (QKV and O through
+    cq_rotate_quantize + cq_lut_gemm, the SwiGLU FFN through cq_moe_ffn, A4W4)
+    and once all in bf16 (torch F.linear).  RMSNorm, rotary embedding and
+    attention (torch scaled_dot_product_attention) are the same torch code in
+    both, in fp16 / bf16.  Weights are random (the work does not depend on
+    their values); each of the n_layers layers has its own, so a step streams
+    more than the L2.  Both steps are replayed from CUDA graphs."""
+    import torch
+    import torch.nn.functional as F
+    H, I, nq, nkv, hd = 2560, 9728, 32, 8, 128
+    g = torch.Generator(device=dev).manual_seed(0)
+
+    def rnd_idx(n, k):
+        return torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device=dev, generator=g)
+
+    def rnd_cb(n):
+        return (torch.randn((n, 16), device=dev, generator=g) * 0.02).sort(dim=1)[0].half()
+
+    def rms(x, w):
+        xf = x.float()
+        return (xf * torch.rsqrt(xf.pow(2).mean(-1, keepdim=True) + 1e-6) * w).to(x.dtype)
+
+    pos = torch.arange(hd // 2, device=dev, dtype=torch.float32)
+    ang = ctx * (1e6 ** (-2 * pos / hd))
+    cos, sin = torch.cos(ang), torch.sin(ang)
+
+    def rope(t):
+        a, b = t.float()[..., : hd // 2], t.float()[..., hd // 2:]
+        return torch.cat([a * cos - b * sin, a * sin + b * cos], -1).to(t.dtype)
+
+    def attention(qkv, kc, vc, M, dt):
+        q = rope(qkv[:, : nq * hd].to(dt).view(M, nq, 1, hd))
+        k = rope(qkv[:, nq * hd:(nq + nkv) * hd].to(dt).view(M, nkv, 1, hd))
+        v = qkv[:, (nq + nkv) * hd:].to(dt).view(M, nkv, 1, hd)
+        kc[:, :, ctx:ctx + 1] = k
+        vc[:, :, ctx:ctx + 1] = v
+        o = F.scaled_dot_product_attention(q, kc, vc, enable_gqa=True)
+        return o.reshape(M, nq * hd)
+
+    out = {}
+    for M in (1, 16):
+        lut_layers, bf_layers = [], []
+        for _ in range(n_layers):
+            nqkv = (nq + 2 * nkv) * hd
+            w = {"sh_gate_idx": rnd_idx(I, H)[None], "sh_up_idx": rnd_idx(I, H)[None],
+                 "sh_down_idx": rnd_idx(H, I)[None], "sh_gate_cb": rnd_cb(I)[None],
+                 "sh_up_cb": rnd_cb(I)[None], "sh_down_cb": rnd_cb(H)[None]}
+            cfg = cq.MoEConfig(H=H, I=I, E=0, top_k=0, n_shared=1, I_shared=I, act_bits=4,
+                               had_block_h=512, had_block_i=256, had_block_i_shared=256)
+            lut_layers.append(dict(
+                wqkv=rnd_idx(nqkv, H), cqkv=rnd_cb(nqkv), wo=rnd_idx(H, nq * hd), co=rnd_cb(H),
+                ffn=cq.MoELayer(cfg, M, w, dev), w=w,
+                kc=torch.randn((M, nkv, ctx + 1, hd), device=dev, generator=g).half(),
+                vc=torch.randn((M, nkv, ctx + 1, hd), device=dev, generator=g).half(),
+                n1=torch.ones(H, device=dev), n2=torch.ones(H, device=dev),
+                y=torch.empty((M, H), dtype=torch.float32, device=dev)))
+            bf_layers.append(dict(
+                wqkv=(torch.randn((nqkv, H), device=dev, generator=g) * 0.02).bfloat16(),
+                wo=(torch.randn((H, nq * hd), device=dev, generator=g) * 0.02).bfloat16(),
+                wgu=(torch.randn((2 * I, H), device=dev, generator=g) * 0.02).bfloat16(),
+                wd=(torch.randn((H, I), device=dev, generator=g) * 0.02).bfloat16(),
+                kc=torch.randn((M, nkv, ctx + 1, hd), device=dev, generator=g).bfloat16(),
+                vc=torch.randn((M, nkv, ctx + 1, hd), device=dev, generator=g).bfloat16(),
+                n1=torch.ones(H, device=dev), n2=torch.ones(H, device=dev)))
+        x_lut = torch.randn((M, H), device=dev, generator=g).half()
+        x_bf = x_lut.bfloat16()
+
+        def lut_step():
+            x = x_lut
+            for L in lut_layers:
+                qc, sq = cq.cq_rotate_quantize(rms(x, L["n1"]), 512, 4)
+                qkv = cq.cq_lut_gemm(qc, sq, H, 4, L["wqkv"], L["cqkv"])
+                a = attention(qkv, L["kc"], L["vc"], M, torch.float16)
+                oc, so = cq.cq_rotate_quantize(a.contiguous(), 4096, 4)
+                x1 = x + cq.cq_lut_gemm(oc, so, nq * hd, 4, L["wo"], L["co"]).half()
+                L["ffn"](rms(x1, L["n2"]).contiguous(), None, L["y"])
+                x = x1 + L["y"].half()
+            return x
+
+        def bf_step():
+            x = x_bf
+            for L in bf_layers:
+                qkv = F.linear(rms(x, L["n1"]), L["wqkv"])
+                a = attention(qkv, L["kc"], L["vc"], M, torch.bfloat16)
+                x1 = x + F.linear(a, L["wo"])
+                gu = F.linear(rms(x1, L["n2"]), L["wgu"])
+                x = x1 + F.linear(F.silu(gu[:, :I]) * gu[:, I:], L["wd"])
+            return x
+
+        res = {}
+        for nm, fn in (("lut", lut_step), ("bf16", bf_step)):
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                fn()
+            for _ in range(args.warmup):
+                graph.replay()
+            ms = timed(graph.replay, args.steps, dist, world)
+            res[nm] = {"tokens_per_s": job_throughput(M, args.steps, world, ms),
+                       "ms_per_step": ms / args.steps}
+            del graph
+        out[f"M{M}"] = {**res, "speedup_vs_bf16": res["lut"]["tokens_per_s"] /
+                        res["bf16"]["tokens_per_s"]}
+        del lut_layers, bf_layers
+        torch.cuda.empty_cache()
+    out["config"] = {"model": "Qwen3-4B-shaped decoder layers (random weights)",
+                     "layers_per_step": n_layers, "kv_context": ctx, "heads": [nq, nkv, hd],
+                     "lut": "A4W4, QKV / O / FFN through the C ABI; attention torch fp16",
+                     "bf16": "torch F.linear, attention torch bf16"}
+    return out
+
+
 def measure(cq, name, args, dev, stream, dist, world, peaks):
     """One workload: the step resident (graph replay), the LUT kernel launch by
     launch, and the step end to end from host buffers.  Returns its block."""
@@ -669,6 +787,8 @@ def measure(cq, name, args, dev, stream, dist, world, peaks):
         bf16 = bf16_dense_context(shapes, dev, stream, args.steps, args.warmup, dist, world)
         bf16["speedup_of_value"] = value / bf16["value"]
         block["bf16_context"] = bf16
+    if name == "qwen3_4b_ffn_decode" and not args.no_bf16:
+        block["decoder_layer_vs_bf16"] = decoder_layer_vs_bf16(cq, args, dev, stream, dist, world)
     if name == LINEAR and not args.no_codebook_sizes:
         block["codebook_sizes"] = measure_codebook_sizes(cq, args, dev, peaks)
     if use_graph:
@@ -760,7 +880,7 @@ def main():
                           "into mma.sync or tcgen05 kind::f16 (tensor memory A operand) with "
                           "fp32 accumulation; rotation exact in fp64",
         }
-        for extra in ("bf16_context", "codebook_sizes"):
+        for extra in ("bf16_context", "codebook_sizes", "decoder_layer_vs_bf16"):
             if extra in head:
                 line[extra] = head[extra]
         print(json.dumps(line), flush=True)
