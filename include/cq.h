@@ -188,25 +188,25 @@ CQ_API cq_status cq_lut_gemm_ex(const void *q, const float *s_x, int64_t M, int6
  * custom-op hosts whose framework owns all device memory and exposes no
  * allocator, and serving processes that forbid cudaMalloc after start-up
  * because it synchronizes the device and fragments a pre-sized pool.  This
- * entry point computes the same product as cq_lut_gemm with the mma.sync LUT
- * kernel (the one cq_lut_gemm uses for M <= 16, with the same split of the
- * contraction, so for M <= 16 the results are identical; for larger M the
- * two agree within the stated error bound), but keeps its split-K partial
- * sums in a fixed array of CQ_NOALLOC_SCRATCH_BYTES bytes compiled into the
- * library.  It calls no cudaMalloc / cudaFree and no allocating library
- * routine.
+ * entry point runs exactly cq_lut_gemm's plan and kernels (so its results are
+ * bitwise identical to cq_lut_gemm's for every shape it accepts), but keeps
+ * the scratch -- the split-K partial sums and, on the tensor-memory kernels,
+ * the fp16 copy of the codes -- in a fixed array of CQ_NOALLOC_SCRATCH_BYTES
+ * bytes compiled into the library.  It calls no cudaMalloc / cudaFree and no
+ * allocating library routine.
  *   - The array occupies CQ_NOALLOC_SCRATCH_BYTES of memory on every GPU that
  *     loads the library, until the process exits.
  *   - The first call on a device looks up the array's device address (once
- *     per device, under a lock); make that first call before any stream
- *     capture.
+ *     per device, under a lock) and keeps it; make that first call before any
+ *     stream capture.  The kept address does not survive cudaDeviceReset: do
+ *     not call this entry point again after resetting the device.
  *   - All calls share the array and it keeps the last call's contents; each
- *     call overwrites every partial sum it reads, so nothing needs clearing.
+ *     call overwrites every scratch value it reads, so nothing needs clearing.
  *     Calls whose work overlaps on the GPU (other streams, other threads)
  *     race on the array and must be serialized by the caller.
- *   - A problem whose partial sums need more than CQ_NOALLOC_SCRATCH_BYTES
- *     (splits * M * N * 4 bytes, where the split count is chosen as for
- *     cq_lut_gemm) returns CQ_ERR_UNSUPPORTED and enqueues nothing.
+ *   - A problem whose scratch needs more than CQ_NOALLOC_SCRATCH_BYTES (as
+ *     cq_lut_gemm_workspace_size reports) returns CQ_ERR_UNSUPPORTED and
+ *     enqueues nothing.
  * Arguments, layouts and the other checks are those of cq_lut_gemm (without
  * centroid_sums and workspace).
  */

@@ -1,13 +1,13 @@
 """cq_lut_gemm_noalloc: the LUT GEMM for callers that cannot allocate device
 memory (framework plugins that are handed only inputs and outputs, serving
-processes that forbid cudaMalloc after start-up).  Its split-K scratch is a
-fixed array inside the library, so these checks call it through the C ABI
-with caller-owned inputs/outputs only and compare it with cq_lut_gemm, twice
-in a row (the second call reuses the array the first one left behind).
+processes that forbid cudaMalloc after start-up).  Its scratch is a fixed
+array inside the library, so these checks call it through the C ABI with
+caller-owned inputs/outputs only, twice in a row (the second call reuses the
+array the first one left behind), and compare it with the oracle at the
+stated tolerance and with cq_lut_gemm bit for bit (the two run the same plan
+and kernels).
 
 This file is named to be collected last."""
-import ctypes
-
 import numpy as np
 import pytest
 import torch
@@ -18,10 +18,12 @@ import synth
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    # (M, K, N, bits): all need split-K partials (several CTAs per row tile)
+    # (M, K, N, bits): all need split-K scratch; M > 16 runs a tensor-memory kernel
     (4, 9728, 128, 4),
     (16, 9728, 256, 8),
     (1, 14336, 64, 4),
+    (40, 9728, 128, 4),
+    (24, 2560, 256, 8),
 ]
 
 
@@ -35,7 +37,7 @@ def _inputs(M, K, N, bits, seed):
 
 
 @pytest.mark.parametrize("M,K,N,bits", CASES)
-def test_noalloc_matches_workspace_entry_point(M, K, N, bits):
+def test_noalloc_matches_oracle_and_workspace_entry_point(M, K, N, bits):
     import lut_clustered_weight_b200 as cq
     assert torch.cuda.is_available()
     dev = "cuda"
@@ -46,8 +48,8 @@ def test_noalloc_matches_workspace_entry_point(M, K, N, bits):
     sd = torch.from_numpy(s).to(dev)
     wd = torch.from_numpy(w_idx).to(dev)
     cd = torch.from_numpy(cb).to(dev)
-    y_ref = cq.cq_lut_gemm(qd, sd, K, bits, wd, cd)
-    _, mag, _ = oracle.lut_gemm(q, s, w_idx, cb)
+    y_ws = cq.cq_lut_gemm(qd, sd, K, bits, wd, cd).cpu().numpy()
+    yr, mag, _ = oracle.lut_gemm(q, s, w_idx, cb)
     tol = oracle.lut_tolerance(mag)
     stream = torch.cuda.current_stream().cuda_stream
     for _ in range(2):
@@ -56,8 +58,9 @@ def test_noalloc_matches_workspace_entry_point(M, K, N, bits):
                                         wd.data_ptr(), cd.data_ptr(), N, y.data_ptr(), stream)
         assert rc == cq.CQ_OK, cq.status_string(rc)
         torch.cuda.synchronize()
-        err = np.abs(y.cpu().numpy().astype(np.float64) - y_ref.cpu().numpy())
-        assert np.all(err <= tol)
+        yn = y.cpu().numpy()
+        assert np.all(np.abs(yn.astype(np.float64) - yr) <= tol)
+        assert np.array_equal(yn.view(np.uint32), y_ws.view(np.uint32))
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
