@@ -90,6 +90,11 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(tab_ready + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool tr0 = tid == 0;  // trace: expand warp 0
+    if (tr0) {
+        TS_TRACE(0);
+        TS_TRACE_ANCHOR();
+    }
     constexpr uint32_t kTmemCols = 512;  // A ring 256 + accumulators kAcc x NTOK (<= 256)
     const TcSchedule S{&L, &P};
 
@@ -182,6 +187,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 const bool first = mw.seg_first(), last = mw.seg_last();
                 if (first && items > 0) ok = mbar_wait(d_empty, (uint32_t)(items - 1) & 1u);
                 ok = ok && mbar_wait(&a_full[gs], (uint32_t)(gi / kTcA) & 1u);
+                TS_TRACE(1100 + 2 * gi);
                 if (!ok) break;
                 tc_fence_after();
                 for (int i = 0; i < mw.gn; i++, jc++) {
@@ -208,6 +214,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 }
                 if (!ok) break;
                 tc_commit(&a_empty[gs]);
+                TS_TRACE(1101 + 2 * gi);
                 if (last) {
                     tc_commit(d_full);
                     items++;
@@ -273,6 +280,20 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
         bool ok = true;
         TcWalk cw;
         cw.init(P, n_pieces);
+        // the codebook of the coming segment is loaded one segment ahead, so a
+        // new work item does not wait for its codebook's HBM round trip
+        auto codebook = [&](const TcWalk &wk, uint4 &a, uint4 &b) {
+            if (!wk.valid) return;
+            int gg, r0, nr, rtt, cc;
+            const uint8_t *ip;
+            const __half *cp;
+            S.item(wk.w, gg, r0, nr, rtt);
+            S.row_ptrs(max(gg, 0), rtt, t, ip, cp, cc);
+            a = ldg_stream(cp);
+            b = ldg_stream(cp + 8);
+        };
+        uint4 cbn0 = make_uint4(0, 0, 0, 0), cbn1 = cbn0;
+        codebook(cw, cbn0, cbn1);
         for (int gi = 0; cw.valid; gi++, cw.next()) {
             const int gs = gi % kTcA;
             if (cw.seg_first()) {
@@ -280,6 +301,13 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 const __half *cbp;
                 S.item(cw.w, g, row0, nrows, rt);
                 S.row_ptrs(max(g, 0), rt, t, idxp, cbp, col);
+                const uint4 c0v = cbn0, c1v = cbn1;
+                {
+                    TcWalk nx = cw;
+                    nx.c0 = nx.c_end;
+                    nx.next();
+                    codebook(nx, cbn0, cbn1);
+                }
                 if (L.h_out) {  // loads in flight during the segment; used by its epilogue
 #pragma unroll
                     for (int i = 0; i < kScl; i++) {
@@ -288,14 +316,14 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                     }
                 }
                 // the one-time LUT precompute for this row
-                const uint4 c0v = *reinterpret_cast<const uint4 *>(cbp);
-                const uint4 c1v = *reinterpret_cast<const uint4 *>(cbp + 8);
                 const uint32_t cu[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
                 if (PAIR) {
                     // the two warps of the quarter build half of the table each
-#pragma unroll 1
-                    for (int hh = 8 * h; hh < 8 * h + 8; hh++) {
-                        const uint32_t hv = (uint32_t)__half_as_ushort(cbp[hh]);
+#pragma unroll
+                    for (int i = 0; i < 8; i++) {
+                        const int hh = 8 * h + i;  // high nibble of the entries
+                        const uint32_t wv = h ? cu[4 + (i >> 1)] : cu[i >> 1];
+                        const uint32_t hv = (i & 1) ? (wv >> 16) : (wv & 0xFFFFu);
 #pragma unroll
                         for (int l = 0; l < 16; l++)
                             tab[(hh * 16 + l) * kTcRows] =
@@ -314,6 +342,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 }
             }
             cp_async_wait_group<kTcWStages - 2>();
+            if (tr0) TS_TRACE(2 + 6 * gi);
             uint32_t wd[16];
             {
                 const uint4 *src = wring + (size_t)(gi % kTcWStages) * 4 * kTcExpand + tid;
@@ -327,6 +356,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 }
             }
             issue_group();
+            if (tr0) TS_TRACE(3 + 6 * gi);
             if (2 * h < cw.gn) {
                 // 128 weights -> 64 fp16 pairs (k = 2b, 2b + 1 in column b)
                 uint32_t v[64];
@@ -349,6 +379,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                         v[4 * qq + 3] = h4[3];
                     }
                 }
+                if (tr0) TS_TRACE(4 + 6 * gi - 0);  // looked up (slot shared with the wait below)
                 if (gi >= kTcA) {
                     ok = mbar_wait(&a_empty[gs], (uint32_t)(gi / kTcA - 1) & 1u);
                     if (!ok) break;
@@ -368,9 +399,11 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[gs]);
+            if (tr0) TS_TRACE(5 + 6 * gi);
             if (cw.seg_last()) {
                 // segment done: this warp's half of the NTOK fp32 columns -> partials
                 ok = mbar_wait(d_full, (uint32_t)items & 1u);
+                if (tr0) TS_TRACE(6 + 6 * gi);
                 if (!ok) break;
                 tc_fence_after();
                 float *out = L.out + (int64_t)cw.slot * L.out_split_stride;
@@ -442,6 +475,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(d_empty);
+                if (tr0) TS_TRACE(7 + 6 * gi);
                 items++;
             }
         }
@@ -452,6 +486,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     __syncthreads();
     tc_fence_after();
     if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
+    if (tr0) TS_TRACE(1999);
 }
 
 // ---------------------------------------------------------------- host side
