@@ -499,11 +499,12 @@ class LinearCall:
         self.y_h.copy_(self.y, non_blocking=True)
 
 
-def lut_timed_launches(cq, step, steps):
-    """Every LUT GEMM launch of `steps` eager steps, CUDA-event timed on its
-    stream.  A spin kernel ahead of every step keeps the GPU busy while the
-    host queues the step, so consecutive kernels run back to back and no
-    launch's events include time the GPU spent waiting for the host."""
+def lut_timed_launches(cq, step, steps, every_kernel=False):
+    """Every LUT GEMM launch (every launch of the library with every_kernel)
+    of `steps` eager steps, CUDA-event timed on its stream.  A spin kernel
+    ahead of every step keeps the GPU busy while the host queues the step, so
+    consecutive kernels run back to back and no launch's events include time
+    the GPU spent waiting for the host."""
     import torch
     t_host = time.perf_counter()
     step()
@@ -511,13 +512,30 @@ def lut_timed_launches(cq, step, steps):
     t_host = time.perf_counter() - t_host
     spin_cycles = int(min(50e-3, 3 * t_host + 1e-3) * 2.0e9)
     cq.cq_timing_read_launches()  # drop anything recorded before
-    cq.cq_timing_enable(True)
+    cq.cq_timing_enable(True, every_kernel=every_kernel)
     for _ in range(steps):
         torch.cuda._sleep(spin_cycles)
         step()
     torch.cuda.synchronize()
     cq.cq_timing_enable(False)
     return cq.cq_timing_read_launches()
+
+
+def kernel_breakdown(launches, steps):
+    """Device time per step of each kernel kind, every launch of the library
+    event-timed (eager steps; the events cost a few microseconds per launch
+    and stop consecutive kernels from overlapping, so the sum exceeds the
+    graph-replayed step time)."""
+    per = {}
+    for k, ms in launches:
+        e = per.setdefault(k, [0, 0.0])
+        e[0] += 1
+        e[1] += ms
+    total = sum(v[1] for v in per.values()) or 1.0
+    out = {k: {"launches_per_step": v[0] / steps, "us_per_step": 1e3 * v[1] / steps,
+               "share": v[1] / total} for k, v in sorted(per.items(), key=lambda kv: -kv[1][1])}
+    return {"kernels": out, "us_per_step_sum": 1e3 * total / steps,
+            "method": "CUDA events around every launch of the library, eager steps"}
 
 
 def lut_alg_bytes_bits(M, N, K, bits, idx_bits):
@@ -759,6 +777,8 @@ def measure(cq, name, args, dev, stream, dist, world, peaks):
                                       peak_gbs, peak_tf, peak_kind)
     roofline["traffic"] = profile_traffic(ROOT / "lut_clustered_weight_b200" / "csrc" / kern_src,
                                           ROOT / "profiles" / f"{roofline['kernel']}_{name}.md")
+    breakdown = kernel_breakdown(lut_timed_launches(cq, step, args.steps, every_kernel=True),
+                                 args.steps)
 
     # ---- e2e: host buffers through the C-ABI, copies inside the timed region
     def step_e2e():
@@ -778,7 +798,7 @@ def measure(cq, name, args, dev, stream, dist, world, peaks):
     block = {"value": value, "unit": "tokens/s", "ms_per_step": ms_step, "config": cfg,
              "effective_gbs": alg_bytes_step / (ms_step / 1e3) / 1e9,
              "alg_bytes_per_step": alg_bytes_step, "alg_flops_per_step": alg_flops_step,
-             "roofline": roofline, "e2e": e2e,
+             "roofline": roofline, "kernel_breakdown": breakdown, "e2e": e2e,
              "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
 
     # ---- context: the same dense FFN step in bf16 with torch (the pages
@@ -880,7 +900,7 @@ def main():
                           "into mma.sync or tcgen05 kind::f16 (tensor memory A operand) with "
                           "fp32 accumulation; rotation exact in fp64",
         }
-        for extra in ("bf16_context", "codebook_sizes", "decoder_layer_vs_bf16"):
+        for extra in ("kernel_breakdown", "bf16_context", "codebook_sizes", "decoder_layer_vs_bf16"):
             if extra in head:
                 line[extra] = head[extra]
         print(json.dumps(line), flush=True)

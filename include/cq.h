@@ -311,15 +311,17 @@ CQ_API cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *ro
  *
  * cq_launch_count   number of kernels this library has launched since it was
  *                   loaded (process-wide).
- * cq_timing_enable  on != 0: every LUT GEMM kernel launch is bracketed by two
- *                   CUDA events on its stream; on = 0 stops recording.
+ * cq_timing_enable  on = 1: every LUT GEMM kernel launch is bracketed by two
+ *                   CUDA events on its stream; on = 2: every launch of the
+ *                   library (LUT GEMMs, rotate-quantize, routing, combine,
+ *                   code conversion, reductions); on = 0 stops recording.
  * cq_timing_read    waits for the recorded events, returns the number of timed
  *                   launches and their summed device time in ms, and clears
  *                   the record.  Returns CQ_ERR_CUDA if an event failed.
  * cq_timing_read_launches
  *                   the same record launch by launch, in launch order: for the
  *                   first min(*n, cap) launches, kinds[i] (CQ_KERNEL_*: which
- *                   LUT GEMM kernel ran) and ms[i] (device time; -1 if its
+ *                   kernel ran) and ms[i] (device time; -1 if its
  *                   events failed, and the call then returns CQ_ERR_CUDA).
  *                   *n = number of recorded launches.  Host arrays of cap
  *                   entries, owned by the caller (NULL allowed when cap = 0).
@@ -331,7 +333,14 @@ enum cq_kernel_kind {
     CQ_KERNEL_LUT_MMA = 0, /* mma.sync kernel, register / shared lookup tables */
     CQ_KERNEL_LUT_TC = 1,  /* tcgen05 kernel for wide token tiles (> 32 rows per group) */
     CQ_KERNEL_LUT_TS = 2,  /* tcgen05 decode kernel (<= 32 rows per group): pair tables */
-    CQ_KERNEL_LUT_VB = 3   /* mma.sync kernel for 3- / 5-bit indices (cq_lut_gemm_ex) */
+    CQ_KERNEL_LUT_VB = 3,  /* mma.sync kernel for 3- / 5-bit indices (cq_lut_gemm_ex) */
+    /* recorded with cq_timing_enable(2) only */
+    CQ_KERNEL_ROTATE_QUANTIZE = 4, /* rotation + quantization of x or h (SwiGLU fused) */
+    CQ_KERNEL_CODES_F16 = 5,       /* activation codes -> fp16 B operand rows */
+    CQ_KERNEL_ROUTE = 6,           /* router top-k and expert grouping (two kernels) */
+    CQ_KERNEL_COMBINE = 7,         /* weighted sum of expert outputs */
+    CQ_KERNEL_REDUCE = 8,          /* split-K partial sums -> y */
+    CQ_KERNEL_CENTROID_SUMS = 9    /* per-centroid integer sums */
 };
 CQ_API int64_t cq_launch_count(void);
 

@@ -110,8 +110,10 @@ def cq_device_error() -> int:
     return int(lib.cq_device_error())
 
 
-def cq_timing_enable(on: bool = True) -> None:
-    _check(lib.cq_timing_enable(1 if on else 0), "cq_timing_enable")
+def cq_timing_enable(on: bool | int = True, every_kernel: bool = False) -> None:
+    """Time LUT GEMM launches (on), or every launch of the library
+    (every_kernel as well); on = False stops recording."""
+    _check(lib.cq_timing_enable((2 if every_kernel else 1) if on else 0), "cq_timing_enable")
 
 
 def cq_timing_read() -> tuple[int, float]:
@@ -128,12 +130,15 @@ def cq_selftest_wait_timeout(stream=None) -> None:
     _check(lib.cq_selftest_wait_timeout(_stream(stream)), "cq_selftest_wait_timeout")
 
 
-KERNEL_KINDS = {0: "k_lut_mma", 1: "k_lut_tc", 2: "k_lut_ts", 3: "k_lut_vb"}   # cq_kernel_kind
+KERNEL_KINDS = {0: "k_lut_mma", 1: "k_lut_tc", 2: "k_lut_ts", 3: "k_lut_vb",   # cq_kernel_kind
+                4: "rotate_quantize", 5: "codes_to_f16", 6: "route", 7: "combine", 8: "reduce",
+                9: "centroid_sums"}
+LUT_KERNELS = frozenset(v for v in KERNEL_KINDS.values() if v.startswith("k_lut"))
 
 
 def cq_timing_read_launches(cap: int = 1 << 16) -> list[tuple[str, float]]:
-    """[(kernel, device ms)] of every timed LUT GEMM launch, in launch order;
-    clears the record."""
+    """[(kernel, device ms)] of every timed launch, in launch order; clears
+    the record."""
     kinds = (ctypes.c_int32 * cap)()
     ms = (ctypes.c_float * cap)()
     n = _I64(0)

@@ -203,8 +203,22 @@ int sm_count();
 
 // ---------------------------------------------------------------- measurement aids
 void count_launch(int n = 1);
-bool timing_on();
+bool timing_on();       // LUT GEMM launches are timed
+bool timing_on_all();   // every launch is timed
 void timing_begin(cudaStream_t st, int kind);  // kind: CQ_KERNEL_*
 void timing_end(cudaStream_t st);
+// Brackets the launches of its scope with timing events when every launch is timed.
+struct TimedScope {
+    cudaStream_t st;
+    bool on;
+    TimedScope(cudaStream_t s, int kind) : st(s), on(timing_on_all()) {
+        if (on) timing_begin(st, kind);
+    }
+    ~TimedScope() {
+        if (on) timing_end(st);
+    }
+    TimedScope(const TimedScope &) = delete;
+    TimedScope &operator=(const TimedScope &) = delete;
+};
 
 }  // namespace cq

@@ -414,6 +414,7 @@ cudaError_t launch_reduce_plain(const float *part, const LutPlan &P, int64_t M, 
                                 const float *s, float *y, cudaStream_t st) {
     const int64_t n = M * N;
     if (n == 0) return cudaSuccess;
+    TimedScope ts(st, CQ_KERNEL_REDUCE);
     count_launch();
     dim3 grid((unsigned)((N + 255) / 256), (unsigned)M);
     return launch_pdl(k_reduce_plain, grid, dim3(256), 0, st, 1, part, P, M, N, s, y);
@@ -452,6 +453,7 @@ cudaError_t launch_centroid_sums(const void *q, int64_t M, int64_t K, int bits,
                                  const uint8_t *w_idx, int64_t N, int32_t *S, cudaStream_t st) {
     const int64_t n = M * N;
     if (n == 0) return cudaSuccess;
+    TimedScope ts(st, CQ_KERNEL_CENTROID_SUMS);
     count_launch();
     return launch_pdl(k_centroid_sums, dim3((unsigned)((n + 127) / 128)), dim3(128), 0, st, 1,
                       reinterpret_cast<const uint8_t *>(q), M, K, bits, w_idx, N, S);

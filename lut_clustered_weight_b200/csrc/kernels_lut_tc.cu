@@ -49,11 +49,18 @@
 
 namespace cq {
 
-constexpr int kTcExpandWarps = 8;    // 2 per TMEM lane quarter: low / high half of a group
+// Expand warps per TMEM lane quarter; each takes kTcG / kTcWq chunks of every
+// group.  Four warps per quarter (one 64-k chunk each) keep four expand warps
+// on every SM sub-partition, so one warp's index loads and tensor-memory
+// stores overlap the others' lookups.
+constexpr int kTcWq = 4;
+constexpr int kTcCpw = kTcG / kTcWq;              // chunks per expand warp and group
+constexpr int kTcPieces = 2 * kTcCpw;             // 16-byte index pieces per thread and group
+constexpr int kTcExpandWarps = 4 * kTcWq;
 constexpr int kTcExpand = kTcExpandWarps * 32;
-constexpr int kWarpMma = 8;          // TMEM allocation + MMA issue (lane 0)
-constexpr int kWarpTma = 9;          // B tile loads (lane 0)
-constexpr int kTcThreads = 320;
+constexpr int kWarpMma = kTcExpandWarps;          // TMEM allocation + MMA issue (lane 0)
+constexpr int kWarpTma = kTcExpandWarps + 1;      // B tile loads (lane 0)
+constexpr int kTcThreads = kTcExpand + 64;
 constexpr int kTcA = 2;              // A ring depth in groups (TMEM columns [0, 256))
 // B ring (shared memory, NTOK x 128 B per chunk tile): kTcB stages of kBG
 // chunk tiles; a stage is freed by the commit of the MMAs that read it.
@@ -65,9 +72,15 @@ template <int NTOK> struct TcBG { static constexpr int n = NTOK <= 64 ? kTcG : 1
 // bound by the MMA latency, so tiles of few tokens spread the four K steps
 // of a chunk over four accumulators (summed in the epilogue).
 template <int NTOK> struct TcAcc { static constexpr int n = NTOK <= 32 ? 4 : 1; };
+// Tiles of up to 128 tokens keep two accumulator buffers (2 x 128 TMEM
+// columns beside the A ring): the MMAs of one work item run while the
+// previous item's accumulator is drained.
+template <int NTOK> struct TcDB { static constexpr bool on = NTOK <= 128; };
 constexpr int kTcWStages = 4;        // index-byte ring per thread, in groups (3 in flight)
 constexpr size_t kPairTableBytes = 256 * kTcRows * 4;  // 128 KB
 
+// 18 warps: five on two of the four SM sub-partitions, whose register files
+// hold 16K registers each, so at most 96 registers per thread.
 template <int NTOK, bool PAIR>
 __global__ void __launch_bounds__(kTcThreads, 1)
 k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPlan P, int b_row_mod) {
@@ -82,12 +95,17 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     uint8_t *bslots = sm;                                     // [kTcB][kBG][NTOK][128 B]
     uint8_t *tables = sm + kTcB * kBG * kBSlot;               // PAIR: [256][128 rows] x 4 B
     uint8_t *wring_raw = tables + (PAIR ? kPairTableBytes : 0);  // [stage][4][256 thr] x 16 B
-    uint64_t *bars = reinterpret_cast<uint64_t *>(wring_raw + kTcWStages * 4 * kTcExpand * 16);
-    uint64_t *a_full = bars, *a_empty = bars + kTcA;
-    uint64_t *b_full = bars + 2 * kTcA, *b_empty = b_full + kTcB;
-    uint64_t *d_full = b_empty + kTcB, *d_empty = d_full + 1, *fin = d_full + 2;
+    uint64_t *bars =
+        reinterpret_cast<uint64_t *>(wring_raw + kTcWStages * kTcPieces * kTcExpand * 16);
+    // A ring barriers per (slot, chunk): the expand warps of one chunk and the
+    // MMAs of that chunk hand a TMEM slot back and forth on their own, so the
+    // warps of a lane quarter do not run in lockstep
+    uint64_t *a_full = bars, *a_empty = bars + kTcA * kTcG;  // [kTcA][kTcG]
+    uint64_t *b_full = bars + 2 * kTcA * kTcG, *b_empty = b_full + kTcB;
+    uint64_t *d_full = b_empty + kTcB, *d_empty = d_full + 2, *fin = d_full + 4;  // d_*: [2]
     uint64_t *tab_ready = fin + 1;  // [4]: PAIR table of a lane quarter built
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(tab_ready + 4);
+    uint64_t *tab_free = tab_ready + 4;  // [4]: both warps of the quarter done with it
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(tab_free + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool tr0 = tid == 0;  // trace: expand warp 0
@@ -95,25 +113,32 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
         TS_TRACE(0);
         TS_TRACE_ANCHOR();
     }
-    constexpr uint32_t kTmemCols = 512;  // A ring 256 + accumulators kAcc x NTOK (<= 256)
+    constexpr bool kDB = TcDB<NTOK>::on;
+    constexpr uint32_t kTmemCols = 512;  // A ring 256 + (kDB ? 2 : 1) x kAcc x NTOK (<= 256)
+    static_assert(kTcA * 128 + (kDB ? 2 : 1) * kAcc * NTOK <= (int)kTmemCols, "TMEM columns");
     const TcSchedule S{&L, &P};
 
     if (warp == kWarpMma) {
         tmem_alloc(s_tmem, kTmemCols);
         tmem_relinquish();
         if (lane == 0) {
-            for (int s = 0; s < kTcA; s++) {
-                mbar_init(&a_full[s], kTcExpandWarps);
+            for (int s = 0; s < kTcA * kTcG; s++) {
+                mbar_init(&a_full[s], 4);  // the chunk's warp in each lane quarter
                 mbar_init(&a_empty[s], 1);
             }
             for (int s = 0; s < kTcB; s++) {
                 mbar_init(&b_full[s], 1);
                 mbar_init(&b_empty[s], 1);
             }
-            mbar_init(d_full, 1);
-            mbar_init(d_empty, kTcExpandWarps);
+            for (int bb = 0; bb < 2; bb++) {
+                mbar_init(&d_full[bb], 1);
+                mbar_init(&d_empty[bb], kTcExpandWarps);
+            }
             mbar_init(fin, 1);
-            for (int qq = 0; qq < 4; qq++) mbar_init(&tab_ready[qq], 2);
+            for (int qq = 0; qq < 4; qq++) {
+                mbar_init(&tab_ready[qq], kTcWq);
+                mbar_init(&tab_free[qq], kTcWq);
+            }
             fence_barrier_init();
             prefetch_tmap(&tmB);
         }
@@ -126,7 +151,10 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     griddep_launch();
     const uint32_t tmem = *s_tmem;
     const uint32_t tmem_a = tmem;                 // columns [0, 256): A ring (2 x 128)
-    const uint32_t tmem_d = tmem + kTcA * 128;    // columns [256, 256 + kAcc NTOK)
+    const uint32_t tmem_d = tmem + kTcA * 128;    // columns [256, 256 + (1|2) kAcc NTOK)
+    // accumulator buffer of work item j, and the phase of its j-th use
+    auto acc_buf = [&](int j) { return kDB ? (j & 1) : 0; };
+    auto acc_use = [&](int j) { return kDB ? (j >> 1) : j; };
 
     // ---- this CTA's groups and chunks (every thread walks the same sequence)
     const int n_pieces = tc_pieces(L, P);
@@ -177,7 +205,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     } else if (warp == kWarpMma) {
         // ====================== MMA issuer (one thread) ======================
         if (lane == 0 && nchunks > 0) {
-            constexpr uint32_t idesc = idesc_f16(kTcRows, NTOK);
+            uint32_t idesc = idesc_f16(kTcRows, NTOK);
             TcWalk mw;
             mw.init(P, n_pieces);
             int items = 0, consumed = 0, jc = 0;
@@ -185,12 +213,31 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
             for (int gi = 0; mw.valid && ok; gi++, mw.next()) {
                 const int gs = gi % kTcA;
                 const bool first = mw.seg_first(), last = mw.seg_last();
-                if (first && items > 0) ok = mbar_wait(d_empty, (uint32_t)(items - 1) & 1u);
-                ok = ok && mbar_wait(&a_full[gs], (uint32_t)(gi / kTcA) & 1u);
-                TS_TRACE(1100 + 2 * gi);
+                const int ab = acc_buf(items);
+                const uint32_t dbase = tmem_d + (uint32_t)(ab * kAcc * NTOK);
+                if (first) {
+                    // MMA width = the item's rows rounded up to 16: the last tile
+                    // of a token group costs what its rows need, not a full tile
+                    int g_, r0_, nr_, rt_;
+                    S.item(mw.w, g_, r0_, nr_, rt_);
+                    idesc = idesc_f16(kTcRows, min(NTOK, max(16, (nr_ + 15) & ~15)));
+                }
+                if (first && acc_use(items) > 0)
+                    ok = mbar_wait(&d_empty[ab], (uint32_t)(acc_use(items) - 1) & 1u);
                 if (!ok) break;
-                tc_fence_after();
-                for (int i = 0; i < mw.gn; i++, jc++) {
+                TS_TRACE(1100 + 2 * gi);
+                // every chunk barrier of the slot completes once per group (short
+                // groups included), so its phase is (gi / kTcA) & 1
+                for (int i = 0; i < kTcG; i++) {
+                    if (!mbar_wait(&a_full[gs * kTcG + i], (uint32_t)(gi / kTcA) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    if (i >= mw.gn) {
+                        tc_commit(&a_empty[gs * kTcG + i]);
+                        continue;
+                    }
+                    tc_fence_after();
                     const int js = kBG == 1 ? jc : gi;
                     const int sb = js % kTcB;
                     if (kBG == 1 || i == 0) {
@@ -206,17 +253,18 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
 #pragma unroll
                     for (int kk = 0; kk < kTcChunk / 16; kk++) {
                         const uint32_t dcol = (uint32_t)((kk % kAcc) * NTOK);
-                        tc_mma_ts(tmem_d + dcol, tmem_a + gs * 128 + i * 32 + kk * 8,
+                        tc_mma_ts(dbase + dcol, tmem_a + gs * 128 + i * 32 + kk * 8,
                                   bd + (uint64_t)(2 * kk), idesc,
                                   (fresh && kk < kAcc) ? 0u : 1u);
                     }
                     if (kBG == 1 || i == mw.gn - 1) tc_commit(&b_empty[sb]);
+                    tc_commit(&a_empty[gs * kTcG + i]);
+                    jc++;
                 }
                 if (!ok) break;
-                tc_commit(&a_empty[gs]);
                 TS_TRACE(1101 + 2 * gi);
                 if (last) {
-                    tc_commit(d_full);
+                    tc_commit(&d_full[ab]);
                     items++;
                 }
             }
@@ -230,8 +278,9 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
         }
     } else {
         // ====================== expand warps ======================
-        // warp e: TMEM lane quarter q = e % 4 (row t), half h = e / 4 of every
-        // group: chunks 2h and 2h + 1, i.e. 64 index bytes -> 64 TMEM columns
+        // warp e: TMEM lane quarter q = e % 4 (row t), part h = e / 4 of every
+        // group: chunks cpw h .. cpw h + cpw - 1 (cpw = kTcCpw), i.e. 32 cpw
+        // index bytes -> 32 cpw TMEM columns
         const int q = warp & 3, h = warp >> 2;
         const int t = q * 32 + lane;  // row within the tile = TMEM lane
         const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
@@ -253,12 +302,12 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                     S.row_ptrs(max(gg, 0), rtt, t, p_row, cbx, cc);
                     p_item = pw.w;
                 }
-                uint4 *dst = wring + (size_t)(gp % kTcWStages) * 4 * kTcExpand + tid;
+                uint4 *dst = wring + (size_t)(gp % kTcWStages) * kTcPieces * kTcExpand + tid;
 #pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    // piece i: k = c0*64 + 128h + 32i .. +32 (chunk 2h + i/2 of the group)
-                    const int k0 = pw.c0 * kTcChunk + 128 * h + 32 * i;
-                    const bool live = (2 * h + (i >> 1)) < pw.gn && k0 < L.K;
+                for (int i = 0; i < kTcPieces; i++) {
+                    // piece i: k = c0*64 + 64 cpw h + 32i .. +32 (chunk cpw h + i/2 of the group)
+                    const int k0 = pw.c0 * kTcChunk + kTcChunk * kTcCpw * h + 32 * i;
+                    const bool live = (kTcCpw * h + (i >> 1)) < pw.gn && k0 < L.K;
                     cp_async16_zfill(dst + i * kTcExpand, live ? p_row + k0 / 2 : p_row,
                                      live ? 16 : 0);
                 }
@@ -271,13 +320,116 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
 
         int g = 0, row0 = 0, nrows = 0, rt = 0, col = 0, items = 0;
         // epilogue: this warp's slice of the NTOK token columns
-        constexpr int kEpi = NTOK >= 32 ? NTOK / 2 : 16;
+        constexpr int kEpi = NTOK / kTcWq >= 16 ? NTOK / kTcWq : 16;
         constexpr int kScl = (kEpi + 31) / 32;
         const int cbeg = h * kEpi;
         float scl[kScl];  // fused SwiGLU: token scales of the slice, lane l holds c = cbeg + l + 32 i
 #pragma unroll
         for (int i = 0; i < kScl; i++) scl[i] = 0.0f;
         bool ok = true;
+        // this warp's chunks of A slot gs free again (the MMAs of group gi - kTcA done)
+        auto wait_slot = [&](int gs, int gi) -> bool {
+#pragma unroll
+            for (int j = 0; j < kTcCpw; j++)
+                if (!mbar_wait(&a_empty[gs * kTcG + kTcCpw * h + j], (uint32_t)(gi / kTcA - 1) & 1u))
+                    return false;
+            return true;
+        };
+        // ---- epilogue of a finished item (deferred: see the group loop)
+        // kLd 16-column loads in flight per wait; a slice covers 16 or 32
+        // columns, whose token scales sit in pd_scl[0] (lane l: column
+        // 32 j + l of the warp's range, j the slices' 32-column block)
+        constexpr int kLd = kAcc == 1 && kTcWq == 2 ? (kEpi >= 32 ? 2 : 1) : 1;
+        static_assert(16 * kLd <= 32, "one scale register per slice");
+        constexpr int kSlices = kEpi / (16 * kLd);
+        int pd_left = 0;  // slices of the pending item still to drain
+        int pd_item = 0, pd_row0 = 0, pd_nrows = 0, pd_col = 0, pd_slot = 0;
+        float pd_scl[kScl];
+#pragma unroll
+        for (int i = 0; i < kScl; i++) pd_scl[i] = 0.0f;
+        auto drain = [&](int n, int gi_tr) -> bool {
+            const int ab = acc_buf(pd_item);
+            const uint32_t dbase = tmem_d + (uint32_t)(ab * kAcc * NTOK);
+            for (; n > 0 && pd_left > 0; n--) {
+                const int it = kSlices - pd_left;
+                if (it == 0) {
+                    if (!mbar_wait(&d_full[ab], (uint32_t)acc_use(pd_item) & 1u)) return false;
+                    if (tr0) TS_TRACE(6 + 6 * gi_tr);
+                    tc_fence_after();
+                }
+                const float cur = pd_scl[0];
+                const int off = (it * 16 * kLd) & 31;  // first column of the slice in cur
+                if ((((it + 1) * 16 * kLd) & 31) == 0) {
+#pragma unroll
+                    for (int i = 0; i + 1 < kScl; i++) pd_scl[i] = pd_scl[i + 1];
+                }
+                const int c0 = cbeg + it * 16 * kLd;
+                if (cbeg < NTOK && c0 < pd_nrows) {  // columns past the rows: nothing to store
+                    // the kAcc accumulators summed one at a time (few live registers)
+                    float acc[kLd][16];
+#pragma unroll
+                    for (int a = 0; a < kAcc; a++) {
+                        uint32_t d[kLd][16];
+#pragma unroll
+                        for (int bb = 0; bb < kLd; bb++)
+                            tmem_ld16(dbase + lane_base + a * NTOK + c0 + 16 * bb, d[bb]);
+                        tmem_wait_ld();
+                        if (tr0) TS_TRACE(1400 + 8 * (pd_item % 60) + 2 * it);
+#pragma unroll
+                        for (int bb = 0; bb < kLd; bb++)
+#pragma unroll
+                            for (int qq = 0; qq < 16; qq++)
+                                acc[bb][qq] = a == 0 ? __uint_as_float(d[bb][qq])
+                                                     : acc[bb][qq] + __uint_as_float(d[bb][qq]);
+                    }
+                    if (L.h_out) {
+                        // SwiGLU.  Lanes 2j (gate) and 2j + 1 (up) hold the same output
+                        // column; the even lane finishes token c and the odd lane token
+                        // c + 1 after one exchange.  All values first (independent
+                        // chains, no branches), then the predicated stores.
+                        const int odd = lane & 1;
+                        __half hv[kLd * 8];
+#pragma unroll
+                        for (int bb = 0; bb < kLd; bb++)
+#pragma unroll
+                            for (int qq = 0; qq < 16; qq += 2) {
+                                const float a0 = acc[bb][qq], a1 = acc[bb][qq + 1];
+                                const float recv = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
+                                const float gv = odd ? recv : a0, uv = odd ? a1 : recv;
+                                const float sx =
+                                    __shfl_sync(0xffffffffu, cur, off + 16 * bb + qq + odd);
+                                hv[bb * 8 + qq / 2] = __float2half_rn(silu_mul(gv * sx, uv * sx));
+                            }
+#pragma unroll
+                        for (int j = 0; j < kLd * 8; j++) {
+                            const int c = c0 + 2 * j + odd;
+                            if (c < pd_nrows)
+                                L.h_out[(int64_t)(pd_row0 + c) * L.h_row_stride + (pd_col >> 1)] =
+                                    hv[j];
+                        }
+                    } else {
+                        float *out = L.out + (int64_t)pd_slot * L.out_split_stride;
+#pragma unroll
+                        for (int bb = 0; bb < kLd; bb++)
+#pragma unroll
+                            for (int qq = 0; qq < 16; qq++) {
+                                const int c = c0 + 16 * bb + qq;
+                                if (c < pd_nrows)
+                                    out[(int64_t)(pd_row0 + c) * L.out_row_stride + pd_col] =
+                                        acc[bb][qq];
+                            }
+                    }
+                }
+                if (tr0) TS_TRACE(1401 + 8 * (pd_item % 60) + 2 * it);
+                if (--pd_left == 0) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&d_empty[ab]);
+                    if (tr0) TS_TRACE(7 + 6 * gi_tr);
+                }
+            }
+            return true;
+        };
         TcWalk cw;
         cw.init(P, n_pieces);
         // the codebook of the coming segment is loaded one segment ahead, so a
@@ -318,12 +470,22 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 // the one-time LUT precompute for this row
                 const uint32_t cu[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
                 if (PAIR) {
-                    // the two warps of the quarter build half of the table each
+                    // the two warps of the quarter build half of the table each,
+                    // once both have finished looking up the previous item
+                    if (items > 0 && !mbar_wait(&tab_free[q], (uint32_t)(items - 1) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    // warp h: entries whose high nibble is in [16 h / kTcWq, 16 (h + 1) / kTcWq)
+                    constexpr int kHi = 16 / kTcWq;
 #pragma unroll
-                    for (int i = 0; i < 8; i++) {
-                        const int hh = 8 * h + i;  // high nibble of the entries
-                        const uint32_t wv = h ? cu[4 + (i >> 1)] : cu[i >> 1];
-                        const uint32_t hv = (i & 1) ? (wv >> 16) : (wv & 0xFFFFu);
+                    for (int i = 0; i < kHi; i++) {
+                        uint32_t wv = cu[i >> 1];  // centroid word of high nibble kHi h + i
+#pragma unroll
+                        for (int hq = 1; hq < kTcWq; hq++)
+                            if (h == hq) wv = cu[(kHi * hq + i) >> 1];
+                        const uint32_t hv = ((kHi * h + i) & 1) ? (wv >> 16) : (wv & 0xFFFFu);
+                        const int hh = kHi * h + i;
 #pragma unroll
                         for (int l = 0; l < 16; l++)
                             tab[(hh * 16 + l) * kTcRows] =
@@ -343,11 +505,11 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
             }
             cp_async_wait_group<kTcWStages - 2>();
             if (tr0) TS_TRACE(2 + 6 * gi);
-            uint32_t wd[16];
+            uint32_t wd[4 * kTcPieces];
             {
-                const uint4 *src = wring + (size_t)(gi % kTcWStages) * 4 * kTcExpand + tid;
+                const uint4 *src = wring + (size_t)(gi % kTcWStages) * kTcPieces * kTcExpand + tid;
 #pragma unroll
-                for (int i = 0; i < 4; i++) {
+                for (int i = 0; i < kTcPieces; i++) {
                     const uint4 v4 = src[i * kTcExpand];
                     wd[4 * i] = v4.x;
                     wd[4 * i + 1] = v4.y;
@@ -357,20 +519,21 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
             }
             issue_group();
             if (tr0) TS_TRACE(3 + 6 * gi);
-            if (2 * h < cw.gn) {
-                // 128 weights -> 64 fp16 pairs (k = 2b, 2b + 1 in column b)
-                uint32_t v[64];
+            if (kTcCpw * h < cw.gn) {
+                // 64 cpw weights -> 32 cpw fp16 pairs (k = 2b, 2b + 1 in column b)
+                constexpr int kB = 32 * kTcCpw;
+                uint32_t v[kB];
                 if (PAIR) {
-                    // 64 independent shared loads (32-bit shared addresses)
+                    // independent shared loads (32-bit shared addresses)
                     const uint32_t tab_s = smem_u32(tab);
 #pragma unroll
-                    for (int b = 0; b < 64; b++) {
+                    for (int b = 0; b < kB; b++) {
                         const uint32_t byte = prmt(wd[b >> 2], 0u, 0x4440u | (uint32_t)(b & 3));
                         v[b] = lds32(tab_s + byte * (kTcRows * 4));
                     }
                 } else {
 #pragma unroll
-                    for (int qq = 0; qq < 16; qq++) {
+                    for (int qq = 0; qq < kB / 4; qq++) {
                         uint32_t h4[4];
                         dequant8(wd[qq], lo, hi, h4);
                         v[4 * qq] = h4[0];
@@ -381,104 +544,57 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 }
                 if (tr0) TS_TRACE(4 + 6 * gi - 0);  // looked up (slot shared with the wait below)
                 if (gi >= kTcA) {
-                    ok = mbar_wait(&a_empty[gs], (uint32_t)(gi / kTcA - 1) & 1u);
+                    ok = wait_slot(gs, gi);
                     if (!ok) break;
                     tc_fence_after();
                 }
-                const uint32_t ta = tmem_a + lane_base + gs * 128 + h * 64;
+                const uint32_t ta = tmem_a + lane_base + gs * 128 + h * kB;
                 tmem_st32(ta, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
-                if (2 * h + 1 < cw.gn)
-                    tmem_st32(ta + 32, *reinterpret_cast<const uint32_t(*)[32]>(&v[32]));
+                if (kTcCpw == 2 && kTcCpw * h + 1 < cw.gn)
+                    tmem_st32(ta + 32, *reinterpret_cast<const uint32_t(*)[32]>(&v[kB - 32]));
                 tmem_wait_st();
             } else if (gi >= kTcA) {
                 // nothing to store (short group), but the slot must be free
                 // before this warp reports it filled
-                ok = mbar_wait(&a_empty[gs], (uint32_t)(gi / kTcA - 1) & 1u);
+                ok = wait_slot(gs, gi);
                 if (!ok) break;
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[gs]);
+            if (lane == 0) {
+#pragma unroll
+                for (int j = 0; j < kTcCpw; j++) mbar_arrive(&a_full[gs * kTcG + kTcCpw * h + j]);
+            }
             if (tr0) TS_TRACE(5 + 6 * gi);
+            // the previous item's accumulator: one slice after each group with
+            // two buffers (its drain overlaps this item's MMAs), all of it
+            // after the first group with one buffer
+            if (pd_left > 0 && !drain(kDB ? 1 : kSlices, gi)) {
+                ok = false;
+                break;
+            }
             if (cw.seg_last()) {
-                // segment done: this warp's half of the NTOK fp32 columns -> partials
-                ok = mbar_wait(d_full, (uint32_t)items & 1u);
-                if (tr0) TS_TRACE(6 + 6 * gi);
-                if (!ok) break;
-                tc_fence_after();
-                float *out = L.out + (int64_t)cw.slot * L.out_split_stride;
-                if (cbeg < NTOK) {
-                    // kLd 16-column loads in flight per wait; an iteration covers
-                    // at most 32 columns, whose token scales sit in scl[0]
-                    constexpr int kLd = kAcc == 1 ? (kEpi >= 32 ? 2 : 1) : 1;
-                    static_assert(16 * kLd <= 32, "one scale register per iteration");
-#pragma unroll 1
-                    for (int it = 0; it < kEpi / (16 * kLd); it++) {
-                        const int c0 = cbeg + it * 16 * kLd;
-                        const float cur = scl[0];
-#pragma unroll
-                        for (int i = 0; i + 1 < kScl; i++) scl[i] = scl[i + 1];
-                        uint32_t d[kAcc * kLd][16];
-#pragma unroll
-                        for (int a = 0; a < kAcc; a++)
-#pragma unroll
-                            for (int bb = 0; bb < kLd; bb++)
-                                tmem_ld16(tmem_d + lane_base + a * NTOK + c0 + 16 * bb, d[a * kLd + bb]);
-                        tmem_wait_ld();
-                        if (L.h_out) {
-                            // SwiGLU.  Lanes 2j (gate) and 2j + 1 (up) hold the same output
-                            // column; the even lane finishes token c and the odd lane token
-                            // c + 1 after one exchange.  All values first (independent
-                            // chains, no branches), then the predicated stores.
-                            const int odd = lane & 1;
-                            __half hv[kLd * 8];
-#pragma unroll
-                            for (int bb = 0; bb < kLd; bb++)
-#pragma unroll
-                                for (int qq = 0; qq < 16; qq += 2) {
-                                    float a0 = __uint_as_float(d[bb][qq]);
-                                    float a1 = __uint_as_float(d[bb][qq + 1]);
-#pragma unroll
-                                    for (int a = 1; a < kAcc; a++) {
-                                        a0 += __uint_as_float(d[a * kLd + bb][qq]);
-                                        a1 += __uint_as_float(d[a * kLd + bb][qq + 1]);
-                                    }
-                                    const float recv =
-                                        __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
-                                    const float gv = odd ? recv : a0, uv = odd ? a1 : recv;
-                                    const float sx =
-                                        __shfl_sync(0xffffffffu, cur, 16 * bb + qq + odd);
-                                    hv[bb * 8 + qq / 2] = __float2half_rn(silu_mul(gv * sx, uv * sx));
-                                }
-#pragma unroll
-                            for (int j = 0; j < kLd * 8; j++) {
-                                const int c = c0 + 2 * j + odd;
-                                if (c < nrows)
-                                    L.h_out[(int64_t)(row0 + c) * L.h_row_stride + (col >> 1)] = hv[j];
-                            }
-                        } else {
-#pragma unroll
-                            for (int bb = 0; bb < kLd; bb++)
-#pragma unroll
-                                for (int qq = 0; qq < 16; qq++) {
-                                    float a0 = __uint_as_float(d[bb][qq]);
-#pragma unroll
-                                    for (int a = 1; a < kAcc; a++)
-                                        a0 += __uint_as_float(d[a * kLd + bb][qq]);
-                                    const int c = c0 + 16 * bb + qq;
-                                    if (c < nrows)
-                                        out[(int64_t)(row0 + c) * L.out_row_stride + col] = a0;
-                                }
-                        }
-                    }
+                if (PAIR) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tab_free[q]);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(d_empty);
-                if (tr0) TS_TRACE(7 + 6 * gi);
+                // a short item may still have its predecessor pending
+                if (pd_left > 0 && !drain(kSlices, gi)) {
+                    ok = false;
+                    break;
+                }
+                pd_item = items;
+                pd_row0 = row0;
+                pd_nrows = nrows;
+                pd_col = col;
+                pd_slot = cw.slot;
+#pragma unroll
+                for (int i = 0; i < kScl; i++) pd_scl[i] = scl[i];
+                pd_left = kSlices;
                 items++;
             }
         }
+        if (ok && pd_left > 0) ok = drain(kSlices, 0);
         cp_async_wait_group<0>();
     }
     // ---- teardown: all MMAs and TMEM reads are complete before TMEM is freed
@@ -564,7 +680,7 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
     const bool pair = ntok <= 16;
     const int nb = ntok <= 64 ? 4 * kTcG : ntok <= 128 ? 8 : 4;  // chunk tiles in the B ring
     P.smem = 1024 + (size_t)nb * ntok * 128 + (pair ? kPairTableBytes : 0) +
-             (size_t)kTcWStages * 4 * kTcExpand * 16 + 512;
+             (size_t)kTcWStages * kTcPieces * kTcExpand * 16 + 512;
     P.tc = 1;
     return P;
 }
@@ -725,6 +841,7 @@ cudaError_t launch_codes_to_f16(const void *codes, int64_t ld_codes, int bits, i
                                 float *scales_out) {
     const int64_t n = rows * (K / 8);
     if (n == 0) return cudaSuccess;
+    TimedScope ts(st, CQ_KERNEL_CODES_F16);
     count_launch();
     return launch_pdl(k_codes_to_f16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, 1,
                       reinterpret_cast<const uint8_t *>(codes), ld_codes, bits, K, rows, map_mode,

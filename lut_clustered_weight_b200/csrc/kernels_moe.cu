@@ -163,6 +163,7 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
                          int32_t *ids, float *w, int32_t *counts, int32_t *offsets, int32_t *perm,
                          int32_t *inv_perm, int32_t *grp_tiles, int32_t *tile_grp,
                          int max_tiles, cudaStream_t st) {
+    TimedScope ts(st, CQ_KERNEL_ROUTE);
     count_launch(2);
     cudaError_t e = launch_pdl(k_topk, dim3((T + kTopkWarps - 1) / kTopkWarps),
                                dim3(kTopkWarps * 32), 0, st, 1, logits, T, E, k, renorm, ids, w);
@@ -245,6 +246,7 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
     if ((int64_t)a.T * a.H == 0) return cudaSuccess;
+    TimedScope ts(st, CQ_KERNEL_COMBINE);
     count_launch();
     return launch_pdl(k_combine, dim3((unsigned)a.T, (unsigned)((a.H + 1023) / 1024)), dim3(256), 0,
                       st, 1, a);

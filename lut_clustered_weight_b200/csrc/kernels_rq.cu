@@ -203,6 +203,178 @@ k_rq_x_warp(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log
     warp_quantize_row(buf, K, log2b, bits, A, q + m * ldq, s + m);
 }
 
+// ------------------------------------------------------------------ rows in registers
+// Thread j of a row holds positions [32 j, 32 j + 32) as fp64 registers.
+// Index bits 0-4 of the transform are butterflies inside the thread, bits
+// 5-9 pair threads j and j ^ 2^(bit - 5) of the same warp (a block's threads
+// are consecutive and aligned, since rows and blocks start at multiples of
+// min(b, 1024) / 32 threads), and bits 10 .. log2b - 1 pair threads of
+// different warps of the row through shared memory.  The row's absmax is
+// reduced through shared memory, then every
+// thread quantizes its 32 values and stores their codes as 16- or 32-byte
+// vectors.  Same exact fp64 arithmetic as the shared-memory kernels, so the
+// codes and scales are identical; no row buffer, so many rows per SM.
+constexpr int kRegThreads = 512;
+
+template <bool XWARP>  // blocks over 1024: levels across warps
+__global__ void __launch_bounds__(kRegThreads)
+k_rq_x_reg(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log2b, int bits,
+           uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s,
+           const __half *__restrict__ scale, const int32_t *__restrict__ perm, int rows_per_cta) {
+    // [threads]: max |v| of each thread's 32; then, for blocks over 1024, the
+    // exchange area [32][threads] (position i of thread t at i * threads + t)
+    extern __shared__ __align__(16) double tmax[];
+    griddep_wait();
+    griddep_launch();
+    const int K32 = K >> 5;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int r = tid / K32, j = tid - r * K32;  // row within the CTA, thread within the row
+    const int64_t m = (int64_t)blockIdx.x * rows_per_cta + r;
+    const bool live = r < rows_per_cta && m < M;
+    double v[32];
+    if (live) {
+        const __half *xr = x + m * ldx;
+        const int e0 = 32 * j;
+        if (!scale && !perm) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(xr + e0);
+            uint4 w[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) w[i] = src[i];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const __half2 *h = reinterpret_cast<const __half2 *>(&w[i]);
+#pragma unroll
+                for (int t = 0; t < 4; t++) {
+                    const float2 f = __half22float2(h[t]);
+                    v[8 * i + 2 * t] = (double)f.x;
+                    v[8 * i + 2 * t + 1] = (double)f.y;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                const int c = perm ? (int)min((unsigned)perm[e0 + i], (unsigned)(K - 1)) : e0 + i;
+                float f = __half2float(xr[c]);
+                if (scale) f = __half2float(__float2half_rn(f * __half2float(scale[c])));
+                v[i] = (double)f;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++) v[i] = 0.0;
+    }
+    // index bits 0-4: inside the thread
+#pragma unroll
+    for (int L = 0; L < 5; L++) {
+        if (L < log2b) {
+            const int h = 1 << L;
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                if ((i & h) == 0) {
+                    const double a = v[i], c = v[i + h];
+                    v[i] = a + c;
+                    v[i + h] = a - c;
+                }
+            }
+        }
+    }
+    // index bits 5-9: across the block's threads of one warp (lower thread
+    // keeps v + p, upper p - v: one correctly rounded fma with an exact +-1
+    // product)
+    for (int L = 5; L < min(log2b, 10); L++) {
+        const int bit = 1 << (L - 5);
+        const double sg = (j & bit) ? -1.0 : 1.0;
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            const double p = __shfl_xor_sync(0xffffffffu, v[i], bit);
+            v[i] = fma(sg, v[i], p);
+        }
+    }
+    // index bits 10..: threads j and j ^ 2^(bit - 5) sit in different warps
+    if (XWARP) {
+        const int T = blockDim.x;
+        double *xch = tmax + T;
+        for (int L = 10; L < log2b; L++) {
+            const int bit = 1 << (L - 5);
+#pragma unroll
+            for (int i = 0; i < 32; i++) xch[i * T + tid] = v[i];
+            __syncthreads();
+            const int pt = tid ^ bit;  // same row: rows start at multiples of b / 32 threads
+            const bool upper = j & bit;
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                const double p = xch[i * T + pt];
+                v[i] = upper ? p - v[i] : v[i] + p;
+            }
+            __syncthreads();
+        }
+    }
+    double mx = 0.0;
+#pragma unroll
+    for (int i = 0; i < 32; i++) mx = fmax(mx, fabs(v[i]));
+    tmax[tid] = mx;
+    __syncthreads();
+    if (!live) return;
+    double A = 0.0;
+    for (int i = 0; i < K32; i++) A = fmax(A, tmax[r * K32 + i]);
+    const int qmax = (1 << (bits - 1)) - 1;
+    const long long Ai = __double2ll_rn(A * 16777216.0);
+    const double R = Ai > 0 ? __ddiv_rn((double)qmax, A) : 0.0;
+    // codes packed as they are made (bits 4: 8 per word, bits 8: 4 per word)
+    const int per_word = bits == 4 ? 8 : 4, fbits = bits;
+    const uint32_t fmask = bits == 4 ? 15u : 255u;
+    uint32_t w[8];
+#pragma unroll
+    for (int t = 0; t < 8; t++) w[t] = 0;
+    uint32_t ties = 0;
+    if (Ai > 0) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            bool t;
+            const int c = quantize_round(v[i], R, t);
+            ties |= (uint32_t)t << i;
+            if (bits == 4)
+                w[i >> 3] |= ((uint32_t)c & 15u) << (4 * (i & 7));
+            else
+                w[i >> 2] |= ((uint32_t)c & 255u) << (8 * (i & 3));
+        }
+    }
+    if (ties) {
+        // rare: the exact rotated value again from the input (the block's
+        // signed sum, exact in fp64 in any order) and the exact rational decision
+        const __half *xr = x + m * ldx;
+        const int b = 1 << log2b;
+#pragma unroll 1
+        for (int i = 0; i < 32; i++) {
+            if (!((ties >> i) & 1u)) continue;
+            const int p = 32 * j + i, blk0 = p & ~(b - 1), pos = p - blk0;
+            double sum = 0.0;
+            for (int k = 0; k < b; k++) {
+                const int e = blk0 + k;
+                const int c = perm ? (int)min((unsigned)perm[e], (unsigned)(K - 1)) : e;
+                float f = __half2float(xr[c]);
+                if (scale) f = __half2float(__float2half_rn(f * __half2float(scale[c])));
+                sum += (__popc(pos & k) & 1) ? -(double)f : (double)f;
+            }
+            const uint32_t c = (uint32_t)quantize_tie(sum, Ai, qmax) & fmask;
+            const int wi = i / per_word, sh = fbits * (i % per_word);
+#pragma unroll
+            for (int t = 0; t < 8; t++)
+                if (t == wi) w[t] = (w[t] & ~(fmask << sh)) | (c << sh);
+        }
+    }
+    uint8_t *qrow = q + m * ldq;
+    if (bits == 4) {
+        *reinterpret_cast<uint4 *>(qrow + 16 * j) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+        uint4 *dst = reinterpret_cast<uint4 *>(qrow + 32 * j);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+    if (j == 0) s[m] = Ai > 0 ? quant_scale(A, log2b, qmax) : 0.0f;
+    (void)lane;
+}
+
 __global__ void __launch_bounds__(kWarpRows * 32) k_rq_swiglu_warp(const SwigluArgs a, int64_t R) {
     extern __shared__ __align__(16) double wbuf[];
     __shared__ int s_ns[kWarpRows][kMaxK / 64];
@@ -260,6 +432,16 @@ static bool use_warp_rows(int64_t rows, int K, int log2b) {
     return log2b <= 8 && K <= 4096 && rows >= 4LL * sm_count();
 }
 
+// The register kernel: blocks of at most 8192, whole rows of at most 512
+// threads, 16-byte aligned rows and code rows, and rows enough for the SMs.
+static bool use_reg_rows(int64_t rows, int K, int log2b, int bits, const void *x, int64_t ldx,
+                         const void *q, int64_t ldq) {
+    const bool aligned = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (ldx % 8 == 0) &&
+                         (reinterpret_cast<uintptr_t>(q) % 16 == 0) && (ldq % 16 == 0);
+    return log2b <= 13 && K % 32 == 0 && K / 32 <= kRegThreads && (bits == 4 || bits == 8) &&
+           aligned && rows >= 2LL * sm_count();
+}
+
 // ------------------------------------------------------------------ launchers
 static int cluster_size(int64_t rows, int K, int log2b) {
     const int ub = std::max(1 << log2b, 8);
@@ -287,6 +469,19 @@ cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K,
                                    const void *scale, const int32_t *perm) {
     const __half *sc = reinterpret_cast<const __half *>(scale);
     if (M == 0) return cudaSuccess;
+    TimedScope ts(st, CQ_KERNEL_ROTATE_QUANTIZE);
+    if (use_reg_rows(M, K, log2b, bits, x, ldx, q, ldq)) {
+        const int K32 = K / 32;
+        const int rows_per_cta = std::max(1, kRegThreads / K32);
+        const int threads = (rows_per_cta * K32 + 31) / 32 * 32;
+        const size_t smem = (size_t)threads * sizeof(double) * (log2b > 10 ? 33 : 1);
+        count_launch();
+        return launch_pdl(log2b > 10 ? k_rq_x_reg<true> : k_rq_x_reg<false>,
+                          dim3((unsigned)((M + rows_per_cta - 1) / rows_per_cta)),
+                          dim3(threads), smem, st, 1,
+                          reinterpret_cast<const __half *>(x), ldx, M, K, log2b, bits,
+                          reinterpret_cast<uint8_t *>(q), ldq, s, sc, perm, rows_per_cta);
+    }
     if (use_warp_rows(M, K, log2b)) {
         const size_t smem = (size_t)kWarpRows * K * sizeof(double);
         count_launch();
@@ -304,6 +499,7 @@ cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K,
 
 cudaError_t launch_swiglu_rq(const SwigluArgs &a, int64_t rows, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
+    TimedScope ts(st, CQ_KERNEL_ROTATE_QUANTIZE);
     const bool warp_r = a.R_routed == 0 || use_warp_rows(rows, a.I, a.log2b_i);
     const bool warp_s = a.R_shared == 0 || use_warp_rows(rows, a.I_shared, a.log2b_i_shared);
     if (warp_r && warp_s) {

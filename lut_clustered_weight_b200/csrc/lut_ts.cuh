@@ -141,7 +141,7 @@ k_lut_ts(const __grid_constant__ CUtensorMap tmI0, const __grid_constant__ CUten
     const bool routed = L.uniform_rows == 0;
     // index stream: the first stages go out before the CTA barrier (uniform
     // launches), the HBM latency of the weights overlaps the set-up
-    TcWalk tw;
+    TcWalk tw{};
     int tgi = 0;
     auto issue_index = [&]() {
         const int s = tgi % kTsI;

@@ -157,6 +157,29 @@ CQ_DEV int quantize_fast(double v, double R, long long Ai, int qmax) {
     return v < 0 ? -q : q;
 }
 
+// The exact decision of quantize_fast's near-tie branch, for the rare values
+// whose fp64 quotient lies within 1e-9 of a tie.
+CQ_DEV int quantize_tie(double v, long long Ai, int qmax) {
+    const int q = quantize_exact(fabs(v), Ai, qmax);
+    return v < 0 ? -q : q;
+}
+
+// Code of one rotated value, as quantize_fast, for callers that quantize many
+// values in registers: t = v * R rounded to the nearest integer (ties to even)
+// by adding and subtracting 1.5 * 2^52 -- the sum lies in [2^52, 2^53), where
+// the fp64 spacing is 1 -- and the integer read from the low word of the sum.
+// Sets *near_tie when |t - round(t)| > 0.5 - 1e-9: the caller then takes
+// quantize_tie instead (|t| <= 127, so outside that window the rounding of t
+// cannot change the decision).
+CQ_DEV int quantize_round(double v, double R, bool &near_tie) {
+    constexpr double kMagic = 6755399441055744.0;  // 1.5 * 2^52
+    const double t = v * R;
+    const double big = t + kMagic;
+    const double r = t - (big - kMagic);
+    near_tie = fabs(r) > 0.5 - 1e-9;
+    return __double2loint(big);
+}
+
 // Quantize buf[0, n) (rotated values of row positions [e0, e0 + n)) and
 // store the codes: bits 4 -> packed bytes (low nibble = even position),
 // bits 8 -> int8.  e0 and n are even.  A is the absmax of the whole row.

@@ -24,6 +24,7 @@ static std::vector<EventPair> g_pending, g_free;
 void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 bool timing_on() { return g_timing.load(std::memory_order_relaxed) != 0; }
+bool timing_on_all() { return g_timing.load(std::memory_order_relaxed) == 2; }
 
 // Record the opening event of a timed launch (closed by timing_end).
 void timing_begin(cudaStream_t st, int kind) {
@@ -64,7 +65,7 @@ CQ_API cq_status cq_selftest_wait_timeout(cq_stream_t stream) {
 }
 
 CQ_API cq_status cq_timing_enable(int32_t on) {
-    cq::g_timing.store(on ? 1 : 0);
+    cq::g_timing.store(on == 2 ? 2 : on ? 1 : 0);
     return CQ_OK;
 }
 

@@ -46,10 +46,20 @@ RQ_CASES = [
     (5, 24, 1, 8, 1),
     (33, 64, 4, 4, 0),
     (0, 256, 256, 4, 0),
-    # many short rows with blocks of at most 256: one warp per row
+    # many rows, blocks of at most 1024: a row in registers, 32 positions per
+    # thread (blocks of 1 to 1024: 0 to 5 levels across threads)
     (600, 1408, 128, 4, 8),
     (700, 4096, 256, 8, 4),
     (593, 64, 8, 4, 0),
+    (400, 2048, 1024, 4, 4),
+    (320, 1536, 512, 8, 2),
+    (301, 96, 32, 4, 0),
+    (310, 224, 1, 8, 1),
+    (333, 4096, 64, 4, 3),
+    # blocks over 1024: levels across warps through shared memory
+    (300, 2048, 2048, 4, 4),
+    (320, 4096, 4096, 8, 3),
+    (296, 8192, 8192, 4, 2),
 ]
 
 
@@ -79,6 +89,26 @@ def test_rotate_quantize_exact_ties(cq):
         assert s.item() == sr[0]
 
 
+@pytest.mark.parametrize("b", [32, 128, 1024, 2048])
+def test_rotate_quantize_exact_ties_many_rows(cq, b):
+    # x = (10.5, 3.5, 0, ...) per block: the Walsh-Hadamard outputs alternate
+    # 14 and 7, so A = 14 and every 7 lands exactly on a tie for int4 (7 * 7 /
+    # 14 = 3.5) -- with hundreds of rows, on the register-resident kernel
+    M, K = 320, 2048
+    x = np.zeros((M, K), dtype=np.float16)
+    x[:, 0::b] = 10.5
+    x[:, 1::b] = 3.5
+    x[1::2] *= -1                       # negative rows: ties on the other side
+    x[5, :] = 0                         # a zero row
+    x[7, 2::b] = 0.25                   # no longer exact ties on row 7
+    for bits in (4, 8):
+        q, s = cq.cq_rotate_quantize(torch.from_numpy(x).to(DEV), b, bits)
+        torch.cuda.synchronize()
+        qr, sr = oracle.rotate_quantize(x, b, bits)
+        assert np.array_equal(oracle.unpack_codes(q.cpu().numpy(), K, bits), qr)
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), sr.view(np.uint32))
+
+
 RQ_SP_CASES = [
     # (M, K, b, bits, scale, perm): one CTA / cluster per row, and the
     # warp-per-row kernel (many rows, b <= 256)
@@ -87,6 +117,7 @@ RQ_SP_CASES = [
     (5, 9728, 256, 4, False, True),
     (700, 1408, 128, 8, True, True),
     (600, 2048, 256, 4, False, True),
+    (400, 2048, 2048, 4, True, True),
 ]
 
 
