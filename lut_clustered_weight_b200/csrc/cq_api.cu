@@ -445,11 +445,25 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
     float *rsc = reinterpret_cast<float *>(ws + m.o_rs);
     const int64_t ldx = code_bytes(m.H, m.bits), ldh = code_bytes(m.Imax, m.bits);
 
-    cudaError_t e = launch_rotate_quantize(x, m.H, T, (int)m.H, ilog2(d->had_block_h), m.bits, xq,
-                                           ldx, sx, st, w->x_scale, w->x_perm);
-    if (e == cudaSuccess && m.E > 0)
+    // routing first: the x rotation then writes the tensor-core B rows of the
+    // routed slots itself (row inv[t * k + j] for token t's j-th expert)
+    cudaError_t e = cudaSuccess;
+    if (m.E > 0)
         e = launch_route(router_logits, (int)T, (int)m.E, (int)m.k, d->renormalize, m.tile_rows,
                          ids, tw, counts, offsets, perm, inv, tiles, tgrp, m.max_tiles_r, st);
+    RqF16 xf{};
+    if (m.E > 0 && m.k_r != kKernMma) {
+        xf.rows = reinterpret_cast<__half *>(ws + m.o_bx_r);
+        xf.map = inv;
+        xf.ncopy = (int)m.k;
+        xf.row_scales = m.fused ? rsc : nullptr;
+    }
+    if (m.ns > 0 && m.k_s != kKernMma) xf.ident = reinterpret_cast<__half *>(ws + m.o_bx_s);
+    const bool x16 = (xf.ncopy > 0 || xf.ident) &&
+                     rq_writes_f16(T, (int)m.H, ilog2(d->had_block_h), m.bits, x, m.H, xq, ldx);
+    if (e == cudaSuccess)
+        e = launch_rotate_quantize(x, m.H, T, (int)m.H, ilog2(d->had_block_h), m.bits, xq, ldx,
+                                   sx, st, w->x_scale, w->x_perm, x16 ? &xf : nullptr);
     // gate / up (dual) -> partial g, u
     if (e == cudaSuccess && m.E > 0) {
         LutLaunch L{};
@@ -467,8 +481,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         }
         if (m.k_r != kKernMma) {
             void *b = ws + m.o_bx_r;
-            e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, m.Rr, kMapPerm, perm, (int)m.k,
-                                    (int)T, b, st, m.fused ? sx : nullptr, rsc);
+            if (!x16)
+                e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, m.Rr, kMapPerm, perm, (int)m.k,
+                                        (int)T, b, st, m.fused ? sx : nullptr, rsc);
             if (e == cudaSuccess)
                 e = m.k_r == kKernTs ? launch_lut_ts(L, m.gu_r, b, m.Rr, 0, st)
                                      : launch_lut_tc(L, m.gu_r, b, m.Rr, 0, st);
@@ -491,8 +506,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         }
         if (m.k_s != kKernMma) {
             void *b = ws + m.o_bx_s;
-            e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, T, kMapIdentity, nullptr, 1,
-                                    (int)T, b, st);
+            if (!x16)
+                e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, T, kMapIdentity, nullptr, 1,
+                                        (int)T, b, st);
             if (e == cudaSuccess)
                 e = m.k_s == kKernTs ? launch_lut_ts(L, m.gu_s, b, T, (int)T, st)
                                      : launch_lut_tc(L, m.gu_s, b, T, (int)T, st);
@@ -501,15 +517,28 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         }
     }
     // SwiGLU + rotate + quantize of h
+    bool h16_r = false, h16_s = false;  // the down projections' B rows written by the rotation
     if (e == cudaSuccess && m.fused) {
         // h was written by the gate/up epilogues: rotate + quantize its rows
-        if (m.E > 0)
+        // ... and write the down projections' tensor-core B rows as they go
+        if (m.E > 0) {
+            RqF16 hf16{};
+            hf16.ident = reinterpret_cast<__half *>(ws + m.o_bh_r);
+            h16_r = m.k_r != kKernMma &&
+                    rq_writes_f16(m.Rr, (int)m.I, ilog2(d->had_block_i), m.bits, hf, m.Imax, hq, ldh);
             e = launch_rotate_quantize(hf, m.Imax, m.Rr, (int)m.I, ilog2(d->had_block_i), m.bits,
-                                       hq, ldh, sh, st);
-        if (e == cudaSuccess && m.ns > 0)
+                                       hq, ldh, sh, st, nullptr, nullptr, h16_r ? &hf16 : nullptr);
+        }
+        if (e == cudaSuccess && m.ns > 0) {
+            RqF16 hf16{};
+            hf16.ident = reinterpret_cast<__half *>(ws + m.o_bh_s);
+            h16_s = m.k_s != kKernMma &&
+                    rq_writes_f16(m.Rs, (int)m.Is, ilog2(d->had_block_i_shared), m.bits,
+                                  hf + m.Rr * m.Imax, m.Imax, hq + m.Rr * ldh, ldh);
             e = launch_rotate_quantize(hf + m.Rr * m.Imax, m.Imax, m.Rs, (int)m.Is,
                                        ilog2(d->had_block_i_shared), m.bits, hq + m.Rr * ldh, ldh,
-                                       sh + m.Rr, st);
+                                       sh + m.Rr, st, nullptr, nullptr, h16_s ? &hf16 : nullptr);
+        }
         if (e == cudaSuccess && dbg && dbg->h)
             e = cudaMemcpyAsync(dbg->h, hf, (size_t)m.R * m.Imax * 2, cudaMemcpyDeviceToDevice, st);
     } else if (e == cudaSuccess) {
@@ -536,8 +565,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.out = pdn_r; L.out_split_stride = m.Rr * m.H; L.out_row_stride = m.H;
         if (m.k_r != kKernMma) {
             void *b = ws + m.o_bh_r;
-            e = launch_codes_to_f16(hq, ldh, m.bits, (int)m.I, m.Rr, kMapIdentity, nullptr, 1, 1,
-                                    b, st);
+            if (!h16_r)
+                e = launch_codes_to_f16(hq, ldh, m.bits, (int)m.I, m.Rr, kMapIdentity, nullptr, 1,
+                                        1, b, st);
             if (e == cudaSuccess)
                 e = m.k_r == kKernTs ? launch_lut_ts(L, m.dn_r, b, m.Rr, 0, st)
                                      : launch_lut_tc(L, m.dn_r, b, m.Rr, 0, st);
@@ -555,8 +585,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.out = pdn_s; L.out_split_stride = m.Rs * m.H; L.out_row_stride = m.H;
         if (m.k_s != kKernMma) {
             void *b = ws + m.o_bh_s;
-            e = launch_codes_to_f16(hq + m.Rr * ldh, ldh, m.bits, (int)m.Is, m.Rs, kMapIdentity,
-                                    nullptr, 1, 1, b, st);
+            if (!h16_s)
+                e = launch_codes_to_f16(hq + m.Rr * ldh, ldh, m.bits, (int)m.Is, m.Rs,
+                                        kMapIdentity, nullptr, 1, 1, b, st);
             if (e == cudaSuccess)
                 e = m.k_s == kKernTs ? launch_lut_ts(L, m.dn_s, b, m.Rs, 0, st)
                                      : launch_lut_tc(L, m.dn_s, b, m.Rs, 0, st);

@@ -14,11 +14,28 @@ constexpr int kMaxK = 16384;
 
 // x fp16 rows with stride ldx (elements); one CTA per row.  scale (fp16 [K])
 // and perm (int32 [K]) are optional: row element j is fp16(x[perm[j]] *
-// scale[perm[j]]) before the rotation.
+// scale[perm[j]]) before the rotation.  f16 (optional): fp16 copies of the
+// codes as well (see RqF16); only when rq_writes_f16 holds for the same
+// arguments, else the call returns cudaErrorNotSupported.
+struct RqF16;
 cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K, int log2b,
                                    int bits, void *q, int64_t ldq_bytes, float *s,
                                    cudaStream_t st, const void *scale = nullptr,
-                                   const int32_t *perm = nullptr);
+                                   const int32_t *perm = nullptr, const RqF16 *f16 = nullptr);
+bool rq_writes_f16(int64_t M, int K, int log2b, int bits, const void *x, int64_t ldx,
+                   const void *q, int64_t ldq_bytes);
+// fp16 copies of the code rows (the B operand of the tensor-core GEMMs),
+// written by the rotate-quantize kernel itself: copy d (d < ncopy) of row m
+// goes to rows[map[m * ncopy + d]] (rows[m] when map is NULL), with the row's
+// scale at row_scales[that row] when row_scales is non-NULL; ident, when
+// non-NULL, receives one more copy at row m.  Rows of K halves.
+struct RqF16 {
+    __half *rows = nullptr;
+    const int32_t *map = nullptr;
+    int ncopy = 0;
+    float *row_scales = nullptr;
+    __half *ident = nullptr;
+};
 
 // ---------------------------------------------------------------- LUT GEMM
 // Token-row -> code-row mapping used by the grouped GEMM.

@@ -176,27 +176,38 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
 // ------------------------------------------------------------------ combine
 // out[t, n] = sum_j w[t,j] * s_h[p] * sum_split part[split][p][n]  (j in order)
 //           + sum_s s_h[ps] * sum_split part_s[split][ps][n]
-// grid (T, ceil(H / 1024)); each thread 4 consecutive columns.
-__global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
-    __shared__ int s_p[kMaxTopK];
-    __shared__ float s_c[kMaxTopK];   // w[t, j] (scale of row p applied separately)
-    __shared__ float s_sh[kMaxTopK];  // h scale of row p
-    __shared__ int s_ns[4][24];       // slot counts, shared expert x row tile of this block (<= 17)
+// One CTA per token and 4 * kCombThreads columns; each thread 4 consecutive
+// columns.  The token's routed and shared rows are one list of sources, and
+// the loads of eight sources go out together, so a token with up to eight
+// rows costs one memory round trip.
+constexpr int kCombThreads = 256;
+constexpr int kCombF = 8;  // sources in flight per round
+
+__global__ void __launch_bounds__(kCombThreads, 3) k_combine(CombineArgs a) {
+    __shared__ int64_t s_row[kMaxTopK + 4];  // source -> partial row (slot 0)
+    __shared__ float s_c[kMaxTopK];          // w[t, j] (scale of row p applied separately)
+    __shared__ float s_sh[kMaxTopK + 4];     // h scale of the source's row
+    __shared__ int s_ns[4][24];              // slot counts, shared expert x row tile of this block (<= 17)
     griddep_wait();
     griddep_launch();
     const int t = blockIdx.x;
-    const int n0 = blockIdx.y * 1024;
+    const int n0 = blockIdx.y * 4 * kCombThreads;
+    const int F = a.topk + a.n_shared;
     if (threadIdx.x < a.topk) {
         const int p = a.inv_perm[t * a.topk + threadIdx.x];
-        s_p[threadIdx.x] = p;
+        s_row[threadIdx.x] = p;
         s_c[threadIdx.x] = a.w[t * a.topk + threadIdx.x];
         s_sh[threadIdx.x] = a.h_scales[p];
+    } else if (threadIdx.x < F) {
+        const int64_t lp = (int64_t)(threadIdx.x - a.topk) * a.T + t;
+        s_row[threadIdx.x] = lp;
+        s_sh[threadIdx.x] = a.h_scales[a.R_routed + lp];
     }
     const int rpt = a.n_shared ? a.plan_s.rows_per_rt : 1;
     const int rt0 = n0 / rpt;
-    const int nrt = a.n_shared ? (min(n0 + 1023, a.H - 1)) / rpt - rt0 + 1 : 0;
-    if (threadIdx.x < a.n_shared * nrt) {
-        const int s = threadIdx.x / nrt, r = threadIdx.x - s * nrt;
+    const int nrt = a.n_shared ? (min(n0 + 4 * kCombThreads - 1, a.H - 1)) / rpt - rt0 + 1 : 0;
+    for (int i = threadIdx.x; i < a.n_shared * nrt; i += kCombThreads) {
+        const int s = i / nrt, r = i - s * nrt;
         s_ns[s][r] = lut_splits_at(a.plan_s, (int64_t)s * a.T + t, (rt0 + r) * rpt);
     }
     __syncthreads();
@@ -204,42 +215,52 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
     if (n >= a.H) return;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     const int64_t stride_r = a.R_routed * (int64_t)a.H / 4, stride_s = a.R_shared * (int64_t)a.H / 4;
-    // routed rows, four at a time (their split-K slot loads in flight together)
-    for (int j0 = 0; j0 < a.topk; j0 += 4) {
-        float4 y[4];
-        const float4 *pj[4];
-        int nsj[4];
+    const int rti = n / rpt - rt0;  // this thread's row tile among the block's
+    for (int f0 = 0; f0 < F; f0 += kCombF) {
+        // slot 0 of every source, all loads in flight together
+        float4 y[kCombF];
+        int nsmax = 0;
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
+        for (int u = 0; u < kCombF; u++) {
+            const int f = f0 + u;
             y[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            const int j = min(j0 + u, a.topk - 1);
-            pj[u] = reinterpret_cast<const float4 *>(a.part_r + (int64_t)s_p[j] * a.H + n);
-            nsj[u] = j0 + u < a.topk ? a.plan_r.splits : 0;
+            if (f < F) {
+                const bool routed = f < a.topk;
+                const int ns = routed ? a.plan_r.splits : s_ns[f - a.topk][rti];
+                nsmax = max(nsmax, ns);
+                if (ns > 0)
+                    y[u] = *reinterpret_cast<const float4 *>((routed ? a.part_r : a.part_s) +
+                                                             s_row[f] * a.H + n);
+            }
         }
-        sum_slots<4>(pj, nsj, stride_r, y);
+        // further split-K slots (a dense layer's decode-time down projection)
+        for (int s0 = 1; s0 < nsmax; s0++) {
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const int j = j0 + u;
-            if (j >= a.topk) break;
-            const float sc = s_sh[j];
-            y[u].x *= sc; y[u].y *= sc; y[u].z *= sc; y[u].w *= sc;
-            if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + (int64_t)s_p[j] * a.H + n) = y[u];
-            const float c = s_c[j];
-            acc.x += c * y[u].x; acc.y += c * y[u].y; acc.z += c * y[u].z; acc.w += c * y[u].w;
+            for (int u = 0; u < kCombF; u++) {
+                const int f = f0 + u;
+                if (f >= F) break;
+                const bool routed = f < a.topk;
+                if (s0 < (routed ? a.plan_r.splits : s_ns[f - a.topk][rti]))
+                    vadd(y[u], *reinterpret_cast<const float4 *>(
+                                   (routed ? a.part_r : a.part_s) + s_row[f] * a.H + n +
+                                   s0 * 4 * (routed ? stride_r : stride_s)));
+            }
         }
-    }
-    // shared experts (at most four), eight split-K slots per round: a dense
-    // layer's down projection is split over many CTAs at decode
-    for (int s = 0; s < a.n_shared; s++) {
-        const int64_t lp = (int64_t)s * a.T + t;
-        const float4 *ps[1] = {reinterpret_cast<const float4 *>(a.part_s + lp * a.H + n)};
-        const int nss[1] = {s_ns[s][n / rpt - rt0]};
-        float4 y[1] = {make_float4(0.f, 0.f, 0.f, 0.f)};
-        sum_slots<1, 8>(ps, nss, stride_s, y);
-        const float sc = a.h_scales[a.R_routed + lp];
-        y[0].x *= sc; y[0].y *= sc; y[0].z *= sc; y[0].w *= sc;
-        if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + (a.R_routed + lp) * a.H + n) = y[0];
-        acc.x += y[0].x; acc.y += y[0].y; acc.z += y[0].z; acc.w += y[0].w;
+#pragma unroll
+        for (int u = 0; u < kCombF; u++) {
+            const int f = f0 + u;
+            if (f >= F) break;
+            const float sc = s_sh[f];
+            y[u].x *= sc; y[u].y *= sc; y[u].z *= sc; y[u].w *= sc;
+            const int64_t dbg_row = f < a.topk ? s_row[f] : a.R_routed + s_row[f];
+            if (a.y_dbg) *reinterpret_cast<float4 *>(a.y_dbg + dbg_row * a.H + n) = y[u];
+            if (f < a.topk) {
+                const float c = s_c[f];
+                acc.x += c * y[u].x; acc.y += c * y[u].y; acc.z += c * y[u].z; acc.w += c * y[u].w;
+            } else {
+                acc.x += y[u].x; acc.y += y[u].y; acc.z += y[u].z; acc.w += y[u].w;
+            }
+        }
     }
     *reinterpret_cast<float4 *>(a.out + (int64_t)t * a.H + n) = acc;
 }
@@ -248,8 +269,9 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
     if ((int64_t)a.T * a.H == 0) return cudaSuccess;
     TimedScope ts(st, CQ_KERNEL_COMBINE);
     count_launch();
-    return launch_pdl(k_combine, dim3((unsigned)a.T, (unsigned)((a.H + 1023) / 1024)), dim3(256), 0,
-                      st, 1, a);
+    const int cols = 4 * kCombThreads;
+    return launch_pdl(k_combine, dim3((unsigned)a.T, (unsigned)((a.H + cols - 1) / cols)),
+                      dim3(kCombThreads), 0, st, 1, a);
 }
 
 }  // namespace cq

@@ -220,159 +220,203 @@ template <bool XWARP>  // blocks over 1024: levels across warps
 __global__ void __launch_bounds__(kRegThreads)
 k_rq_x_reg(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log2b, int bits,
            uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s,
-           const __half *__restrict__ scale, const int32_t *__restrict__ perm, int rows_per_cta) {
+           const __half *__restrict__ scale, const int32_t *__restrict__ perm, int rows_per_cta,
+           int n_groups, const RqF16 f16) {
     // [threads]: max |v| of each thread's 32; then, for blocks over 1024, the
     // exchange area [32][threads] (position i of thread t at i * threads + t)
     extern __shared__ __align__(16) double tmax[];
     griddep_wait();
     griddep_launch();
     const int K32 = K >> 5;
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int r = tid / K32, j = tid - r * K32;  // row within the CTA, thread within the row
-    const int64_t m = (int64_t)blockIdx.x * rows_per_cta + r;
-    const bool live = r < rows_per_cta && m < M;
-    double v[32];
-    if (live) {
-        const __half *xr = x + m * ldx;
-        const int e0 = 32 * j;
-        if (!scale && !perm) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(xr + e0);
-            uint4 w[4];
+    const int tid = threadIdx.x;
+    const int r = tid / K32, j = tid - r * K32;  // row within the group, thread within the row
+    const bool plain = !scale && !perm;
+    // persistent: row groups blockIdx.x, + gridDim.x, ...; the fp16 inputs of
+    // the next group are loaded while this one is rotated and quantized
+    uint4 nx[4];
+    auto fetch = [&](int grp) {
+        const int64_t mm = (int64_t)grp * rows_per_cta + r;
+        if (plain && grp < n_groups && r < rows_per_cta && mm < M) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + mm * ldx + 32 * j);
 #pragma unroll
-            for (int i = 0; i < 4; i++) w[i] = src[i];
+            for (int i = 0; i < 4; i++) nx[i] = __ldcs(src + i);
+        }
+    };
+    fetch(blockIdx.x);
+    for (int grp = blockIdx.x; grp < n_groups; grp += gridDim.x) {
+        const int64_t m = (int64_t)grp * rows_per_cta + r;
+        const bool live = r < rows_per_cta && m < M;
+        double v[32];
+        if (live) {
+            const __half *xr = x + m * ldx;
+            const int e0 = 32 * j;
+            if (plain) {
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const __half2 *h = reinterpret_cast<const __half2 *>(&w[i]);
+                for (int i = 0; i < 4; i++) {
+                    const __half2 *h = reinterpret_cast<const __half2 *>(&nx[i]);
 #pragma unroll
-                for (int t = 0; t < 4; t++) {
-                    const float2 f = __half22float2(h[t]);
-                    v[8 * i + 2 * t] = (double)f.x;
-                    v[8 * i + 2 * t + 1] = (double)f.y;
+                    for (int t = 0; t < 4; t++) {
+                        const float2 f = __half22float2(h[t]);
+                        v[8 * i + 2 * t] = (double)f.x;
+                        v[8 * i + 2 * t + 1] = (double)f.y;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    const int c = perm ? (int)min((unsigned)perm[e0 + i], (unsigned)(K - 1)) : e0 + i;
+                    float f = __half2float(xr[c]);
+                    if (scale) f = __half2float(__float2half_rn(f * __half2float(scale[c])));
+                    v[i] = (double)f;
                 }
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 32; i++) {
-                const int c = perm ? (int)min((unsigned)perm[e0 + i], (unsigned)(K - 1)) : e0 + i;
-                float f = __half2float(xr[c]);
-                if (scale) f = __half2float(__float2half_rn(f * __half2float(scale[c])));
-                v[i] = (double)f;
-            }
+            for (int i = 0; i < 32; i++) v[i] = 0.0;
         }
-    } else {
+        fetch(grp + gridDim.x);
+        // index bits 0-4: inside the thread
 #pragma unroll
-        for (int i = 0; i < 32; i++) v[i] = 0.0;
-    }
-    // index bits 0-4: inside the thread
+        for (int L = 0; L < 5; L++) {
+            if (L < log2b) {
+                const int h = 1 << L;
 #pragma unroll
-    for (int L = 0; L < 5; L++) {
-        if (L < log2b) {
-            const int h = 1 << L;
-#pragma unroll
-            for (int i = 0; i < 32; i++) {
-                if ((i & h) == 0) {
-                    const double a = v[i], c = v[i + h];
-                    v[i] = a + c;
-                    v[i + h] = a - c;
+                for (int i = 0; i < 32; i++) {
+                    if ((i & h) == 0) {
+                        const double a = v[i], c = v[i + h];
+                        v[i] = a + c;
+                        v[i + h] = a - c;
+                    }
                 }
             }
         }
-    }
-    // index bits 5-9: across the block's threads of one warp (lower thread
-    // keeps v + p, upper p - v: one correctly rounded fma with an exact +-1
-    // product)
-    for (int L = 5; L < min(log2b, 10); L++) {
-        const int bit = 1 << (L - 5);
-        const double sg = (j & bit) ? -1.0 : 1.0;
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
-            const double p = __shfl_xor_sync(0xffffffffu, v[i], bit);
-            v[i] = fma(sg, v[i], p);
-        }
-    }
-    // index bits 10..: threads j and j ^ 2^(bit - 5) sit in different warps
-    if (XWARP) {
-        const int T = blockDim.x;
-        double *xch = tmax + T;
-        for (int L = 10; L < log2b; L++) {
+        // index bits 5-9: across the block's threads of one warp (lower thread
+        // keeps v + p, upper p - v: one correctly rounded fma with an exact +-1
+        // product)
+        for (int L = 5; L < min(log2b, 10); L++) {
             const int bit = 1 << (L - 5);
-#pragma unroll
-            for (int i = 0; i < 32; i++) xch[i * T + tid] = v[i];
-            __syncthreads();
-            const int pt = tid ^ bit;  // same row: rows start at multiples of b / 32 threads
-            const bool upper = j & bit;
+            const double sg = (j & bit) ? -1.0 : 1.0;
 #pragma unroll
             for (int i = 0; i < 32; i++) {
-                const double p = xch[i * T + pt];
-                v[i] = upper ? p - v[i] : v[i] + p;
+                const double p = __shfl_xor_sync(0xffffffffu, v[i], bit);
+                v[i] = fma(sg, v[i], p);
             }
-            __syncthreads();
         }
-    }
-    double mx = 0.0;
+        // index bits 10..: threads j and j ^ 2^(bit - 5) sit in different warps
+        if (XWARP) {
+            const int T = blockDim.x;
+            double *xch = tmax + T;
+            for (int L = 10; L < log2b; L++) {
+                const int bit = 1 << (L - 5);
 #pragma unroll
-    for (int i = 0; i < 32; i++) mx = fmax(mx, fabs(v[i]));
-    tmax[tid] = mx;
-    __syncthreads();
-    if (!live) return;
-    double A = 0.0;
-    for (int i = 0; i < K32; i++) A = fmax(A, tmax[r * K32 + i]);
-    const int qmax = (1 << (bits - 1)) - 1;
-    const long long Ai = __double2ll_rn(A * 16777216.0);
-    const double R = Ai > 0 ? __ddiv_rn((double)qmax, A) : 0.0;
-    // codes packed as they are made (bits 4: 8 per word, bits 8: 4 per word)
-    const int per_word = bits == 4 ? 8 : 4, fbits = bits;
-    const uint32_t fmask = bits == 4 ? 15u : 255u;
-    uint32_t w[8];
+                for (int i = 0; i < 32; i++) xch[i * T + tid] = v[i];
+                __syncthreads();
+                const int pt = tid ^ bit;  // same row: rows start at multiples of b / 32 threads
+                const bool upper = j & bit;
 #pragma unroll
-    for (int t = 0; t < 8; t++) w[t] = 0;
-    uint32_t ties = 0;
-    if (Ai > 0) {
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
-            bool t;
-            const int c = quantize_round(v[i], R, t);
-            ties |= (uint32_t)t << i;
-            if (bits == 4)
-                w[i >> 3] |= ((uint32_t)c & 15u) << (4 * (i & 7));
-            else
-                w[i >> 2] |= ((uint32_t)c & 255u) << (8 * (i & 3));
+                for (int i = 0; i < 32; i++) {
+                    const double p = xch[i * T + pt];
+                    v[i] = upper ? p - v[i] : v[i] + p;
+                }
+                __syncthreads();
+            }
         }
-    }
-    if (ties) {
-        // rare: the exact rotated value again from the input (the block's
-        // signed sum, exact in fp64 in any order) and the exact rational decision
-        const __half *xr = x + m * ldx;
-        const int b = 1 << log2b;
+        double mx = 0.0;
+#pragma unroll
+        for (int i = 0; i < 32; i++) mx = fmax(mx, fabs(v[i]));
+        tmax[tid] = mx;
+        __syncthreads();
+        if (live) {
+            double A = 0.0;
+            for (int i = 0; i < K32; i++) A = fmax(A, tmax[r * K32 + i]);
+            const int qmax = (1 << (bits - 1)) - 1;
+            const long long Ai = __double2ll_rn(A * 16777216.0);
+            const double R = Ai > 0 ? __ddiv_rn((double)qmax, A) : 0.0;
+            // codes packed as they are made (bits 4: 8 per word, bits 8: 4 per word)
+            const int per_word = bits == 4 ? 8 : 4, fbits = bits;
+            const uint32_t fmask = bits == 4 ? 15u : 255u;
+            uint32_t w[8];
+#pragma unroll
+            for (int t = 0; t < 8; t++) w[t] = 0;
+            uint32_t ties = 0;
+            if (Ai > 0) {
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    bool t;
+                    const int c = quantize_round(v[i], R, t);
+                    ties |= (uint32_t)t << i;
+                    if (bits == 4)
+                        w[i >> 3] |= ((uint32_t)c & 15u) << (4 * (i & 7));
+                    else
+                        w[i >> 2] |= ((uint32_t)c & 255u) << (8 * (i & 3));
+                }
+            }
+            if (ties) {
+                // rare: the exact rotated value again from the input (the block's
+                // signed sum, exact in fp64 in any order) and the exact rational decision
+                const __half *xr = x + m * ldx;
+                const int b = 1 << log2b;
 #pragma unroll 1
-        for (int i = 0; i < 32; i++) {
-            if (!((ties >> i) & 1u)) continue;
-            const int p = 32 * j + i, blk0 = p & ~(b - 1), pos = p - blk0;
-            double sum = 0.0;
-            for (int k = 0; k < b; k++) {
-                const int e = blk0 + k;
-                const int c = perm ? (int)min((unsigned)perm[e], (unsigned)(K - 1)) : e;
-                float f = __half2float(xr[c]);
-                if (scale) f = __half2float(__float2half_rn(f * __half2float(scale[c])));
-                sum += (__popc(pos & k) & 1) ? -(double)f : (double)f;
-            }
-            const uint32_t c = (uint32_t)quantize_tie(sum, Ai, qmax) & fmask;
-            const int wi = i / per_word, sh = fbits * (i % per_word);
+                for (int i = 0; i < 32; i++) {
+                    if (!((ties >> i) & 1u)) continue;
+                    const int p = 32 * j + i, blk0 = p & ~(b - 1), pos = p - blk0;
+                    double sum = 0.0;
+                    for (int k = 0; k < b; k++) {
+                        const int e = blk0 + k;
+                        const int c = perm ? (int)min((unsigned)perm[e], (unsigned)(K - 1)) : e;
+                        float f = __half2float(xr[c]);
+                        if (scale) f = __half2float(__float2half_rn(f * __half2float(scale[c])));
+                        sum += (__popc(pos & k) & 1) ? -(double)f : (double)f;
+                    }
+                    const uint32_t c = (uint32_t)quantize_tie(sum, Ai, qmax) & fmask;
+                    const int wi = i / per_word, sh = fbits * (i % per_word);
 #pragma unroll
-            for (int t = 0; t < 8; t++)
-                if (t == wi) w[t] = (w[t] & ~(fmask << sh)) | (c << sh);
-        }
-    }
-    uint8_t *qrow = q + m * ldq;
-    if (bits == 4) {
-        *reinterpret_cast<uint4 *>(qrow + 16 * j) = make_uint4(w[0], w[1], w[2], w[3]);
-    } else {
-        uint4 *dst = reinterpret_cast<uint4 *>(qrow + 32 * j);
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    }
-    if (j == 0) s[m] = Ai > 0 ? quant_scale(A, log2b, qmax) : 0.0f;
-    (void)lane;
+                    for (int t = 0; t < 8; t++)
+                        if (t == wi) w[t] = (w[t] & ~(fmask << sh)) | (c << sh);
+                }
+            }
+            uint8_t *qrow = q + m * ldq;
+            if (bits == 4) {
+                *reinterpret_cast<uint4 *>(qrow + 16 * j) = make_uint4(w[0], w[1], w[2], w[3]);
+            } else {
+                uint4 *dst = reinterpret_cast<uint4 *>(qrow + 32 * j);
+                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+            const float sq = Ai > 0 ? quant_scale(A, log2b, qmax) : 0.0f;
+            if (j == 0) s[m] = sq;
+            if (f16.ncopy > 0 || f16.ident) {
+                // the 32 codes as fp16 (small integers: exact), 64 bytes per copy
+                uint32_t hw[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    int c0, c1;
+                    if (bits == 4) {
+                        c0 = (int)(w[i >> 3] << (28 - 4 * (i & 7))) >> 28;
+                        c1 = (int)(w[(i + 1) >> 3] << (28 - 4 * ((i + 1) & 7))) >> 28;
+                    } else {
+                        c0 = (int)(w[i >> 2] << (24 - 8 * (i & 3))) >> 24;
+                        c1 = (int)(w[(i + 1) >> 2] << (24 - 8 * ((i + 1) & 3))) >> 24;
+                    }
+                    const __half2 h2 = __halves2half2(__int2half_rn(c0), __int2half_rn(c1));
+                    hw[i >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+                auto put = [&](__half *row) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(row + 32 * j);
+#pragma unroll
+                    for (int t = 0; t < 4; t++)
+                        dst[t] = make_uint4(hw[4 * t], hw[4 * t + 1], hw[4 * t + 2], hw[4 * t + 3]);
+                };
+                for (int d = 0; d < f16.ncopy; d++) {
+                    const int64_t row = f16.map ? (int64_t)f16.map[m * f16.ncopy + d] : m;
+                    put(f16.rows + row * K);
+                    if (f16.row_scales && j == 0) f16.row_scales[row] = sq;
+                }
+                if (f16.ident) put(f16.ident + m * K);
+            }
+        }  // live
+        __syncthreads();  // tmax (and the exchange area) are reused by the next group
+    }  // row groups
 }
 
 __global__ void __launch_bounds__(kWarpRows * 32) k_rq_swiglu_warp(const SwigluArgs a, int64_t R) {
@@ -464,9 +508,14 @@ static cudaError_t launch_clustered(Kern kern, int64_t rows, int cs, size_t smem
     return launch_pdl(kern, dim3((unsigned)(rows * cs)), dim3(kRqThreads), smem, st, cs, args...);
 }
 
+bool rq_writes_f16(int64_t M, int K, int log2b, int bits, const void *x, int64_t ldx,
+                   const void *q, int64_t ldq) {
+    return use_reg_rows(M, K, log2b, bits, x, ldx, q, ldq);
+}
+
 cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K, int log2b,
                                    int bits, void *q, int64_t ldq, float *s, cudaStream_t st,
-                                   const void *scale, const int32_t *perm) {
+                                   const void *scale, const int32_t *perm, const RqF16 *f16) {
     const __half *sc = reinterpret_cast<const __half *>(scale);
     if (M == 0) return cudaSuccess;
     TimedScope ts(st, CQ_KERNEL_ROTATE_QUANTIZE);
@@ -475,13 +524,16 @@ cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K,
         const int rows_per_cta = std::max(1, kRegThreads / K32);
         const int threads = (rows_per_cta * K32 + 31) / 32 * 32;
         const size_t smem = (size_t)threads * sizeof(double) * (log2b > 10 ? 33 : 1);
+        const int64_t n_groups = (M + rows_per_cta - 1) / rows_per_cta;
+        const int grid = (int)std::min<int64_t>(n_groups, 2LL * sm_count());
         count_launch();
-        return launch_pdl(log2b > 10 ? k_rq_x_reg<true> : k_rq_x_reg<false>,
-                          dim3((unsigned)((M + rows_per_cta - 1) / rows_per_cta)),
+        return launch_pdl(log2b > 10 ? k_rq_x_reg<true> : k_rq_x_reg<false>, dim3((unsigned)grid),
                           dim3(threads), smem, st, 1,
                           reinterpret_cast<const __half *>(x), ldx, M, K, log2b, bits,
-                          reinterpret_cast<uint8_t *>(q), ldq, s, sc, perm, rows_per_cta);
+                          reinterpret_cast<uint8_t *>(q), ldq, s, sc, perm, rows_per_cta,
+                          (int)n_groups, f16 ? *f16 : RqF16{});
     }
+    if (f16 && (f16->ncopy > 0 || f16->ident)) return cudaErrorNotSupported;
     if (use_warp_rows(M, K, log2b)) {
         const size_t smem = (size_t)kWarpRows * K * sizeof(double);
         count_launch();
