@@ -233,17 +233,24 @@ __global__ void __launch_bounds__(kCombThreads, 3) k_combine(CombineArgs a) {
                                                              s_row[f] * a.H + n);
             }
         }
-        // further split-K slots (a dense layer's decode-time down projection)
-        for (int s0 = 1; s0 < nsmax; s0++) {
+        // further split-K slots (a dense layer's decode-time down projection),
+        // source by source with eight slot loads in flight, added in slot order
+        if (nsmax > 1) {
 #pragma unroll
             for (int u = 0; u < kCombF; u++) {
                 const int f = f0 + u;
                 if (f >= F) break;
                 const bool routed = f < a.topk;
-                if (s0 < (routed ? a.plan_r.splits : s_ns[f - a.topk][rti]))
-                    vadd(y[u], *reinterpret_cast<const float4 *>(
-                                   (routed ? a.part_r : a.part_s) + s_row[f] * a.H + n +
-                                   s0 * 4 * (routed ? stride_r : stride_s)));
+                const int ns = routed ? a.plan_r.splits : s_ns[f - a.topk][rti];
+                if (ns < 2) continue;
+                const int64_t st4 = routed ? stride_r : stride_s;
+                const float4 *p1[1] = {reinterpret_cast<const float4 *>(
+                                           (routed ? a.part_r : a.part_s) + s_row[f] * a.H + n) +
+                                       st4};
+                const int ns1[1] = {ns - 1};
+                float4 acc1[1] = {y[u]};
+                sum_slots<1, 8>(p1, ns1, st4, acc1);
+                y[u] = acc1[0];
             }
         }
 #pragma unroll
