@@ -78,6 +78,10 @@ template <int NTOK> struct TcAcc { static constexpr int n = NTOK <= 32 ? 4 : 1; 
 template <int NTOK> struct TcDB { static constexpr bool on = NTOK <= 128; };
 constexpr int kTcWStages = 4;        // index-byte ring per thread, in groups (3 in flight)
 constexpr size_t kPairTableBytes = 256 * kTcRows * 4;  // 128 KB
+// 256-token tiles with SwiGLU in the epilogue: h of one item is staged in
+// shared memory per expand-warp group (64 tokens x 64 columns, fp16) and
+// written as whole 128-byte rows
+template <int NTOK> struct TcHStage { static constexpr size_t bytes = NTOK == 256 ? kTcWq * 64 * 128 : 0; };
 
 // 18 warps: five on two of the four SM sub-partitions, whose register files
 // hold 16K registers each, so at most 96 registers per thread.
@@ -94,9 +98,9 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     constexpr int kAcc = TcAcc<NTOK>::n;
     uint8_t *bslots = sm;                                     // [kTcB][kBG][NTOK][128 B]
     uint8_t *tables = sm + kTcB * kBG * kBSlot;               // PAIR: [256][128 rows] x 4 B
-    uint8_t *wring_raw = tables + (PAIR ? kPairTableBytes : 0);  // [stage][4][256 thr] x 16 B
-    uint64_t *bars =
-        reinterpret_cast<uint64_t *>(wring_raw + kTcWStages * kTcPieces * kTcExpand * 16);
+    uint8_t *wring_raw = tables + (PAIR ? kPairTableBytes : 0);  // [stage][pieces][thr] x 16 B
+    uint8_t *hstage = wring_raw + kTcWStages * kTcPieces * kTcExpand * 16;  // [kTcWq][64][128 B]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(hstage + TcHStage<NTOK>::bytes);
     // A ring barriers per (slot, chunk): the expand warps of one chunk and the
     // MMAs of that chunk hand a TMEM slot back and forth on their own, so the
     // warps of a lane quarter do not run in lockstep
@@ -105,7 +109,8 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
     uint64_t *d_full = b_empty + kTcB, *d_empty = d_full + 2, *fin = d_full + 4;  // d_*: [2]
     uint64_t *tab_ready = fin + 1;  // [4]: PAIR table of a lane quarter built
     uint64_t *tab_free = tab_ready + 4;  // [4]: both warps of the quarter done with it
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(tab_free + 4);
+    uint64_t *hs_bar = tab_free + 4;     // [kTcWq]: staged h of a token range (4 warps)
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(hs_bar + kTcWq);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool tr0 = tid == 0;  // trace: expand warp 0
@@ -139,6 +144,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                 mbar_init(&tab_ready[qq], kTcWq);
                 mbar_init(&tab_free[qq], kTcWq);
             }
+            for (int hh = 0; hh < kTcWq; hh++) mbar_init(&hs_bar[hh], 4);
             fence_barrier_init();
             prefetch_tmap(&tmB);
         }
@@ -336,13 +342,22 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
             return true;
         };
         // ---- epilogue of a finished item (deferred: see the group loop)
-        // kLd 16-column loads in flight per wait; a slice covers 16 or 32
-        // columns, whose token scales sit in pd_scl[0] (lane l: column
-        // 32 j + l of the warp's range, j the slices' 32-column block)
-        constexpr int kLd = kAcc == 1 && kTcWq == 2 ? (kEpi >= 32 ? 2 : 1) : 1;
-        static_assert(16 * kLd <= 32, "one scale register per slice");
+        // kLd 16-column loads in flight per wait.  One accumulator buffer:
+        // 32-column slices, all drained at once (the MMAs are idle until the
+        // drain ends).  Two buffers: 16-column slices, one after each of the
+        // next item's groups.  The token scale of the warp's column
+        // cbeg + 32 r + l sits in lane l of pd_scl[r].
+        constexpr int kLd = kDB ? 1 : (kEpi >= 32 ? 2 : 1);
+        static_assert(kEpi % (16 * kLd) == 0, "drain slices");
         constexpr int kSlices = kEpi / (16 * kLd);
         int pd_left = 0;  // slices of the pending item still to drain
+        uint32_t hs_phase = 0;  // completed phases of hs_bar[h]
+        // the four warps of this token range meet (bounded wait)
+        auto group_sync = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&hs_bar[h]);
+            return mbar_wait(&hs_bar[h], hs_phase++ & 1u);
+        };
         int pd_item = 0, pd_row0 = 0, pd_nrows = 0, pd_col = 0, pd_slot = 0;
         float pd_scl[kScl];
 #pragma unroll
@@ -357,12 +372,7 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                     if (tr0) TS_TRACE(6 + 6 * gi_tr);
                     tc_fence_after();
                 }
-                const float cur = pd_scl[0];
-                const int off = (it * 16 * kLd) & 31;  // first column of the slice in cur
-                if ((((it + 1) * 16 * kLd) & 31) == 0) {
-#pragma unroll
-                    for (int i = 0; i + 1 < kScl; i++) pd_scl[i] = pd_scl[i + 1];
-                }
+                const int off = (it * 16 * kLd) & 31;  // slice start within its 32-column block
                 const int c0 = cbeg + it * 16 * kLd;
                 if (cbeg < NTOK && c0 < pd_nrows) {  // columns past the rows: nothing to store
                     // the kAcc accumulators summed one at a time (few live registers)
@@ -396,16 +406,28 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                                 const float a0 = acc[bb][qq], a1 = acc[bb][qq + 1];
                                 const float recv = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
                                 const float gv = odd ? recv : a0, uv = odd ? a1 : recv;
-                                const float sx =
-                                    __shfl_sync(0xffffffffu, cur, off + 16 * bb + qq + odd);
+                                float sreg = pd_scl[0];
+#pragma unroll
+                                for (int i = 1; i < kScl; i++)
+                                    if (((it * 16 * kLd + 16 * bb) >> 5) == i) sreg = pd_scl[i];
+                                const float sx = __shfl_sync(0xffffffffu, sreg,
+                                                             (off + 16 * bb) % 32 + qq + odd);
                                 hv[bb * 8 + qq / 2] = __float2half_rn(silu_mul(gv * sx, uv * sx));
                             }
+                        if (TcHStage<NTOK>::bytes > 0) {
+                            // into this group's tile: token c - cbeg, column t / 2
+                            __half *st = reinterpret_cast<__half *>(hstage + h * (64 * 128));
 #pragma unroll
-                        for (int j = 0; j < kLd * 8; j++) {
-                            const int c = c0 + 2 * j + odd;
-                            if (c < pd_nrows)
-                                L.h_out[(int64_t)(pd_row0 + c) * L.h_row_stride + (pd_col >> 1)] =
-                                    hv[j];
+                            for (int j = 0; j < kLd * 8; j++)
+                                st[(c0 - cbeg + 2 * j + odd) * 64 + (t >> 1)] = hv[j];
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < kLd * 8; j++) {
+                                const int c = c0 + 2 * j + odd;
+                                if (c < pd_nrows)
+                                    L.h_out[(int64_t)(pd_row0 + c) * L.h_row_stride +
+                                            (pd_col >> 1)] = hv[j];
+                            }
                         }
                     } else {
                         float *out = L.out + (int64_t)pd_slot * L.out_split_stride;
@@ -421,6 +443,23 @@ k_lut_tc(const __grid_constant__ CUtensorMap tmB, const LutLaunch L, const LutPl
                     }
                 }
                 if (tr0) TS_TRACE(1401 + 8 * (pd_item % 60) + 2 * it);
+                if (TcHStage<NTOK>::bytes > 0 && L.h_out && pd_left == 1) {
+                    // the four warps of this token range (one per lane quarter)
+                    // have staged their columns: 64 rows of 128 B as 16-byte stores
+                    if (!group_sync()) return false;
+                    const int gt = q * 32 + lane;  // thread within the group
+                    const uint4 *src = reinterpret_cast<const uint4 *>(hstage + h * (64 * 128));
+                    const int n0 = pd_col >> 1 & ~63;  // the tile's first output column
+#pragma unroll
+                    for (int k = gt; k < 64 * 8; k += 128) {
+                        const int r = k >> 3, part = k & 7;
+                        if (cbeg + r < pd_nrows)
+                            *reinterpret_cast<uint4 *>(L.h_out + (int64_t)(pd_row0 + cbeg + r) *
+                                                                     L.h_row_stride +
+                                                       n0 + 8 * part) = src[k];
+                    }
+                    if (!group_sync()) return false;  // the tile is free for the next item
+                }
                 if (--pd_left == 0) {
                     tc_fence_before();
                     __syncwarp();
@@ -680,7 +719,8 @@ LutPlan plan_lut_tc(int N, int K, bool dual, int max_rows_per_group, int64_t est
     const bool pair = ntok <= 16;
     const int nb = ntok <= 64 ? 4 * kTcG : ntok <= 128 ? 8 : 4;  // chunk tiles in the B ring
     P.smem = 1024 + (size_t)nb * ntok * 128 + (pair ? kPairTableBytes : 0) +
-             (size_t)kTcWStages * kTcPieces * kTcExpand * 16 + 512;
+             (size_t)kTcWStages * kTcPieces * kTcExpand * 16 +
+             (ntok == 256 ? TcHStage<256>::bytes : 0) + 512;
     P.tc = 1;
     return P;
 }

@@ -216,7 +216,9 @@ k_rq_x_warp(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log
 // codes and scales are identical; no row buffer, so many rows per SM.
 constexpr int kRegThreads = 512;
 
-template <bool XWARP>  // blocks over 1024: levels across warps
+// XWARP: blocks over 1024 (levels across warps); FULL: blocks of at least 32
+// (all five in-thread levels, unconditional, so no value needs a merge)
+template <bool XWARP, bool FULL>
 __global__ void __launch_bounds__(kRegThreads)
 k_rq_x_reg(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log2b, int bits,
            uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s,
@@ -278,7 +280,7 @@ k_rq_x_reg(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log2
         // index bits 0-4: inside the thread
 #pragma unroll
         for (int L = 0; L < 5; L++) {
-            if (L < log2b) {
+            if (FULL || L < log2b) {
                 const int h = 1 << L;
 #pragma unroll
                 for (int i = 0; i < 32; i++) {
@@ -527,7 +529,9 @@ cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K,
         const int64_t n_groups = (M + rows_per_cta - 1) / rows_per_cta;
         const int grid = (int)std::min<int64_t>(n_groups, 2LL * sm_count());
         count_launch();
-        return launch_pdl(log2b > 10 ? k_rq_x_reg<true> : k_rq_x_reg<false>, dim3((unsigned)grid),
+        auto kern = log2b > 10 ? k_rq_x_reg<true, true>
+                  : log2b >= 5 ? k_rq_x_reg<false, true> : k_rq_x_reg<false, false>;
+        return launch_pdl(kern, dim3((unsigned)grid),
                           dim3(threads), smem, st, 1,
                           reinterpret_cast<const __half *>(x), ldx, M, K, log2b, bits,
                           reinterpret_cast<uint8_t *>(q), ldq, s, sc, perm, rows_per_cta,

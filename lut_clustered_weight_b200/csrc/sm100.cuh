@@ -55,24 +55,36 @@ CQ_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// The same test, but a thread whose phase is not complete is suspended in
+// hardware until the phase completes or about hint_ns nanoseconds pass --
+// no instructions issue while it waits.
+CQ_DEV bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
 CQ_DEV uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
 // Wait for the phase with the given parity to complete.  A thread that has to
-// wait sleeps between polls (16 ns doubling up to max_sleep_ns), so waiting
-// warps leave the issue slots and the shared-memory pipe to the working ones.
-// Gives up after about one second, records kErrWaitTimeout and returns false.
-CQ_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t max_sleep_ns = 256) {
+// wait is suspended in hardware between tests (up to hint_ns each), so waiting
+// warps leave the issue slots and the integer pipe to the working ones and
+// wake when the phase completes.  Gives up after about one second, records
+// kErrWaitTimeout and returns false.
+CQ_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t hint_ns = 10000) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t ns = 16;
     for (uint32_t i = 1;; i++) {
-        __nanosleep(ns);
-        if (mbar_try_wait(bar, parity)) return true;
-        ns = min(2 * ns, max_sleep_ns);
-        if ((i & 63) == 0 && globaltimer_ns() - t0 > 1000000000ull) break;
+        if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+        if ((i & 15) == 0 && globaltimer_ns() - t0 > 1000000000ull) break;
     }
     atomicExch(&g_device_error, kErrWaitTimeout);
     return false;
