@@ -128,7 +128,7 @@ struct MoePlan {
     LutKernel k_r, k_s;                 // kernel of the routed / shared launches
     bool fused;                         // gate/up launches write h (SwiGLU in their epilogue)
     LutPlan gu_r, gu_s, dn_r, dn_s;
-    size_t o_xq, o_sx, o_ids, o_w, o_counts, o_offsets, o_perm, o_inv, o_tiles, o_tgrp;
+    size_t o_xq, o_sx, o_ids, o_w, o_counts, o_offsets, o_perm, o_inv, o_tiles, o_tgrp, o_chist;
     size_t o_pgu_r, o_pgu_s, o_hq, o_sh, o_pdn_r, o_pdn_s;
     size_t o_bx_r, o_bx_s, o_bh_r, o_bh_s;  // fp16 B operands of tensor-core launches
     size_t o_hf;                            // fused: h fp16 [R][Imax]
@@ -211,6 +211,7 @@ MoePlan plan_moe(const cq_moe_desc *d, int64_t T) {
     m.o_inv = take((size_t)m.Rr * 4);
     m.o_tiles = take((size_t)(m.E + 1) * 4);
     m.o_tgrp = take((size_t)m.max_tiles_r * 4);
+    m.o_chist = take(m.E > 0 ? route_scratch_bytes((int)T, (int)m.E, (int)m.k) : 0);
     m.o_pgu_r = take(m.E > 0 && !m.fused ? (size_t)m.gu_r.splits * m.Rr * m.I * 2 * 4 : 0);
     m.o_pgu_s = take(m.ns > 0 && !m.fused ? (size_t)m.gu_s.splits * m.Rs * m.Is * 2 * 4 : 0);
     m.o_hf = take(m.fused ? (size_t)m.R * m.Imax * 2 : 0);
@@ -450,7 +451,8 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
     cudaError_t e = cudaSuccess;
     if (m.E > 0)
         e = launch_route(router_logits, (int)T, (int)m.E, (int)m.k, d->renormalize, m.tile_rows,
-                         ids, tw, counts, offsets, perm, inv, tiles, tgrp, m.max_tiles_r, st);
+                         ids, tw, counts, offsets, perm, inv, tiles, tgrp, m.max_tiles_r,
+                         reinterpret_cast<int32_t *>(ws + m.o_chist), st);
     RqF16 xf{};
     if (m.E > 0 && m.k_r != kKernMma) {
         xf.rows = reinterpret_cast<__half *>(ws + m.o_bx_r);

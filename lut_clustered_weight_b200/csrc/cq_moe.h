@@ -41,10 +41,13 @@ struct CombineArgs {
     float *y_dbg;             // [R][H] or NULL
 };
 
+// Routing: top-k + softmax weights, then the expert grouping.  chist:
+// route_scratch_bytes(T, E, k) bytes of device scratch (per-chunk counts).
+size_t route_scratch_bytes(int T, int E, int k);
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int tile_rows,
                          int32_t *ids, float *w, int32_t *counts, int32_t *offsets, int32_t *perm,
                          int32_t *inv_perm, int32_t *grp_tiles, int32_t *tile_grp,
-                         int max_tiles, cudaStream_t st);
+                         int max_tiles, int32_t *chist, cudaStream_t st);
 cudaError_t launch_swiglu_rq(const SwigluArgs &a, int64_t rows, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 

@@ -1,5 +1,7 @@
 // kernels_moe.cu -- routing / expert grouping and combine kernels of the
 // CodeQuant MoE linear layer (sm_100a).
+#include <algorithm>
+
 #include "cq_common.cuh"
 #include "cq_internal.h"
 #include "cq_moe.h"
@@ -10,10 +12,9 @@ namespace cq {
 // (1) k_topk: one warp per token, the token's logits held in registers:
 //     the k largest in descending order, ties to the lower expert id, and the
 //     softmax weights.
-// (2) k_group: one CTA: per-expert counts and offsets, a stable permutation
-//     of the slots t*k+j grouped by expert (each warp places a contiguous
-//     chunk of slots in slot order), its inverse, and the per-expert prefix of
-//     token tiles used by the grouped GEMM.
+// (2) k_group_hist + k_group_place: per-expert counts and offsets, a stable
+//     permutation of the slots t*k+j grouped by expert, its inverse, and the
+//     per-expert prefix of token tiles used by the grouped GEMM (below).
 constexpr int kTopkWarps = 8;
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
@@ -77,36 +78,71 @@ k_topk(const float *__restrict__ logits, int T, int E, int k, int renorm,
     }
 }
 
-constexpr int kGroupThreads = 1024;
+// Grouping over many CTAs.  The S = T*k slots are cut into contiguous chunks,
+// one CTA each.  k_group_hist: per-chunk expert counts.  k_group_place: the
+// chunk's base per expert (counts of the chunks before it), the global
+// offsets (all chunks' counts, scanned over experts), and a stable placement
+// of the chunk's slots (each warp a contiguous run, in slot order) -- the
+// same permutation a single pass in slot order gives.  CTA 0 also writes the
+// counts, offsets and tile tables.
+constexpr int kGroupThreads = 256;
 constexpr int kGroupWarps = kGroupThreads / 32;
 
 __global__ void __launch_bounds__(kGroupThreads)
-k_group(const int32_t *__restrict__ ids, int T, int E, int k, int tile_rows,
-        int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
-        int32_t *__restrict__ inv_perm, int32_t *__restrict__ grp_tiles,
-        int32_t *__restrict__ tile_grp, int max_tiles) {
+k_group_hist(const int32_t *__restrict__ ids, int S, int E, int chunk, int32_t *__restrict__ chist) {
+    __shared__ int32_t hist[kMaxExperts];
+    griddep_wait();
+    griddep_launch();
+    for (int e = threadIdx.x; e < E; e += kGroupThreads) hist[e] = 0;
+    __syncthreads();
+    const int c0 = blockIdx.x * chunk, c1 = min(S, c0 + chunk);
+    for (int sl = c0 + threadIdx.x; sl < c1; sl += kGroupThreads) atomicAdd(&hist[ids[sl]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kGroupThreads) chist[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(kGroupThreads)
+k_group_place(const int32_t *__restrict__ ids, int S, int E, int tile_rows, int chunk, int nchunk,
+              const int32_t *__restrict__ chist, int32_t *__restrict__ counts,
+              int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+              int32_t *__restrict__ inv_perm, int32_t *__restrict__ grp_tiles,
+              int32_t *__restrict__ tile_grp, int max_tiles) {
     __shared__ int32_t hist[kGroupWarps][kMaxExperts];
     __shared__ int32_t s_off[kMaxExperts + 1];
     __shared__ int32_t s_tiles[kMaxExperts + 1];
+    __shared__ int32_t s_base[kMaxExperts];
     griddep_wait();
     griddep_launch();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int S = T * k;
+    const int cb = blockIdx.x;
     for (int i = tid; i < kGroupWarps * kMaxExperts; i += kGroupThreads) (&hist[0][0])[i] = 0;
     __syncthreads();
-    const int chunk = (S + kGroupWarps - 1) / kGroupWarps;
-    const int c0 = warp * chunk, c1 = min(S, c0 + chunk);
-    for (int sl = c0 + lane; sl < c1; sl += 32) atomicAdd(&hist[warp][ids[sl]], 1);
+    // this chunk's slots: a contiguous run per warp, counted per warp
+    const int c0 = cb * chunk, c1 = min(S, c0 + chunk);
+    const int sub = (c1 - c0 + kGroupWarps - 1) / kGroupWarps;
+    const int w0 = min(c1, c0 + warp * sub), w1 = min(c1, w0 + sub);
+    for (int sl = w0 + lane; sl < w1; sl += 32) atomicAdd(&hist[warp][ids[sl]], 1);
     __syncthreads();
-    if (tid < E) {
-        int c = 0;
-        for (int ww = 0; ww < kGroupWarps; ww++) c += hist[ww][tid];
-        s_off[tid + 1] = c;
-        s_tiles[tid + 1] = (c + tile_rows - 1) / tile_rows;
+    // per expert: slots of the chunks before this one, and of all chunks (one
+    // chunk: this CTA's own counts, no histogram launch)
+    for (int e = tid; e < E; e += kGroupThreads) {
+        int before = 0, total = 0;
+        if (nchunk == 1) {
+            for (int ww = 0; ww < kGroupWarps; ww++) total += hist[ww][e];
+        } else {
+            for (int c = 0; c < nchunk; c++) {
+                const int v = chist[(int64_t)c * E + e];
+                before += c < cb ? v : 0;
+                total += v;
+            }
+        }
+        s_base[e] = before;
+        s_off[e + 1] = total;
+        s_tiles[e + 1] = (total + tile_rows - 1) / tile_rows;
     }
     if (tid == 0) { s_off[0] = 0; s_tiles[0] = 0; }
     __syncthreads();
-    if (warp == 0) {  // inclusive scans over E <= 256 entries, 8 per lane
+    if (warp == 0) {  // inclusive scans over E <= 256 entries
         int base_o = 0, base_t = 0;
         for (int e0 = 0; e0 < E; e0 += 32) {
             const int e = e0 + lane + 1;
@@ -123,26 +159,29 @@ k_group(const int32_t *__restrict__ ids, int T, int E, int k, int tile_rows,
         }
     }
     __syncthreads();
-    if (tid < E) {
-        int base = s_off[tid];
-        counts[tid] = s_off[tid + 1] - s_off[tid];
+    if (cb == 0) {
+        for (int e = tid; e < E; e += kGroupThreads) counts[e] = s_off[e + 1] - s_off[e];
+        for (int e = tid; e <= E; e += kGroupThreads) {
+            offsets[e] = s_off[e];
+            grp_tiles[e] = s_tiles[e];
+        }
+        // tile -> group, so the LUT kernels find a tile's expert with one load
+        for (int e = tid; e < E; e += kGroupThreads)
+            for (int tl = s_tiles[e]; tl < s_tiles[e + 1] && tl < max_tiles; tl++) tile_grp[tl] = e;
+    }
+    // bases of the warps' runs
+    for (int e = tid; e < E; e += kGroupThreads) {
+        int base = s_off[e] + s_base[e];
         for (int ww = 0; ww < kGroupWarps; ww++) {
-            const int h = hist[ww][tid];
-            hist[ww][tid] = base;
+            const int h = hist[ww][e];
+            hist[ww][e] = base;
             base += h;
         }
     }
-    if (tid <= E) {
-        offsets[tid] = s_off[tid];
-        grp_tiles[tid] = s_tiles[tid];
-    }
-    // tile -> group, so the LUT kernels find a tile's expert with one load
-    if (tid < E)
-        for (int tl = s_tiles[tid]; tl < s_tiles[tid + 1] && tl < max_tiles; tl++) tile_grp[tl] = tid;
     __syncthreads();
-    for (int sb = c0; sb < c1; sb += 32) {
+    for (int sb = w0; sb < w1; sb += 32) {
         const int sl = sb + lane;
-        const bool ok = sl < c1;
+        const bool ok = sl < w1;
         const int e = ok ? ids[sl] : -1 - lane;
         const unsigned act = __ballot_sync(0xffffffffu, ok);
         const unsigned peers = __match_any_sync(0xffffffffu, e);
@@ -159,18 +198,37 @@ k_group(const int32_t *__restrict__ ids, int T, int E, int k, int tile_rows,
     }
 }
 
+// Slots per grouping chunk: at least 1024 (decode-sized routings take one
+// CTA and no histogram launch), at most 128 chunks.
+static int group_chunk(int S) { return std::max(1024, (S + 127) / 128); }
+
+size_t route_scratch_bytes(int T, int E, int k) {
+    const int S = T * k;
+    const int chunk = group_chunk(S);
+    return (size_t)((S + chunk - 1) / chunk) * E * sizeof(int32_t);
+}
+
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int tile_rows,
                          int32_t *ids, float *w, int32_t *counts, int32_t *offsets, int32_t *perm,
                          int32_t *inv_perm, int32_t *grp_tiles, int32_t *tile_grp,
-                         int max_tiles, cudaStream_t st) {
+                         int max_tiles, int32_t *chist, cudaStream_t st) {
     TimedScope ts(st, CQ_KERNEL_ROUTE);
-    count_launch(2);
+    const int S = T * k;
+    const int chunk = group_chunk(S);
+    const int nchunk = (S + chunk - 1) / chunk;
+    count_launch(nchunk > 1 ? 3 : 2);
     cudaError_t e = launch_pdl(k_topk, dim3((T + kTopkWarps - 1) / kTopkWarps),
                                dim3(kTopkWarps * 32), 0, st, 1, logits, T, E, k, renorm, ids, w);
     if (e != cudaSuccess) return e;
-    return launch_pdl(k_group, dim3(1), dim3(kGroupThreads), 0, st, 1, (const int32_t *)ids, T, E,
-                      k, tile_rows, counts, offsets, perm, inv_perm, grp_tiles, tile_grp,
-                      max_tiles);
+    if (nchunk > 1) {
+        e = launch_pdl(k_group_hist, dim3(nchunk), dim3(kGroupThreads), 0, st, 1,
+                       (const int32_t *)ids, S, E, chunk, chist);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(k_group_place, dim3(nchunk), dim3(kGroupThreads), 0, st, 1,
+                      (const int32_t *)ids, S, E, tile_rows, chunk, nchunk,
+                      (const int32_t *)chist, counts, offsets, perm, inv_perm, grp_tiles,
+                      tile_grp, max_tiles);
 }
 
 // ------------------------------------------------------------------ combine
