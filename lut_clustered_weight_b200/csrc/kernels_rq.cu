@@ -328,9 +328,22 @@ k_rq_x_reg(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log2
         for (int i = 0; i < 32; i++) mx = fmax(mx, fabs(v[i]));
         tmax[tid] = mx;
         __syncthreads();
+        // the row's first thread reduces its K/32 maxima (four independent
+        // chains) and leaves the row's absmax in the row's first entry
+        if (live && j == 0) {
+            double m4[4] = {0.0, 0.0, 0.0, 0.0};
+            const double *row = tmax + r * K32;
+            int i = 0;
+            for (; i + 4 <= K32; i += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; u++) m4[u] = fmax(m4[u], row[i + u]);
+            }
+            for (; i < K32; i++) m4[0] = fmax(m4[0], row[i]);
+            tmax[r * K32] = fmax(fmax(m4[0], m4[1]), fmax(m4[2], m4[3]));
+        }
+        __syncthreads();
         if (live) {
-            double A = 0.0;
-            for (int i = 0; i < K32; i++) A = fmax(A, tmax[r * K32 + i]);
+            const double A = tmax[r * K32];
             const int qmax = (1 << (bits - 1)) - 1;
             const long long Ai = __double2ll_rn(A * 16777216.0);
             const double R = Ai > 0 ? __ddiv_rn((double)qmax, A) : 0.0;
