@@ -44,7 +44,7 @@ LutKernel pick_kernel(int64_t rows, int64_t N, bool dual, int64_t K, int64_t til
     switch (lut_path()) {
     case kPathMma: return kKernMma;
     case kPathTc: return kKernTc;
-    case kPathTs: return rows <= 32 ? kKernTs : kKernTc;
+    case kPathTs: return kKernTs;  // groups over 32 rows: several 32-token tiles
     default: break;
     }
     if (rows <= 16 && !routed) return kKernMma;
