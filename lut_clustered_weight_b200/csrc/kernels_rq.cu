@@ -10,6 +10,9 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <mutex>
+#include <tuple>
+#include <vector>
 
 #include "cq_common.cuh"
 #include "cq_internal.h"
@@ -491,6 +494,27 @@ static bool use_warp_rows(int64_t rows, int K, int log2b) {
     return log2b <= 8 && K <= 4096 && rows >= 4LL * sm_count();
 }
 
+// CTAs of `kern` resident per SM at this block size and dynamic shared
+// memory (asked once per combination and device).
+static int resident_ctas(const void *kern, int threads, size_t smem) {
+    static std::mutex mu;
+    static std::vector<std::tuple<const void *, int, size_t, int, int>> memo;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(mu);
+    for (const auto &m : memo)
+        if (std::get<0>(m) == kern && std::get<1>(m) == threads && std::get<2>(m) == smem &&
+            std::get<3>(m) == dev)
+            return std::get<4>(m);
+    configure_kernel_once(kern);  // the shared-memory limit the launch will have
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess)
+        n = 1;
+    n = std::max(n, 1);
+    memo.emplace_back(kern, threads, smem, dev, n);
+    return n;
+}
+
 // The register kernel: blocks of at most 8192, whole rows of at most 512
 // threads, 16-byte aligned rows and code rows, and rows enough for the SMs.
 static bool use_reg_rows(int64_t rows, int K, int log2b, int bits, const void *x, int64_t ldx,
@@ -540,10 +564,12 @@ cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K,
         const int threads = (rows_per_cta * K32 + 31) / 32 * 32;
         const size_t smem = (size_t)threads * sizeof(double) * (log2b > 10 ? 33 : 1);
         const int64_t n_groups = (M + rows_per_cta - 1) / rows_per_cta;
-        const int grid = (int)std::min<int64_t>(n_groups, 2LL * sm_count());
-        count_launch();
         auto kern = log2b > 10 ? k_rq_x_reg<true, true>
                   : log2b >= 5 ? k_rq_x_reg<false, true> : k_rq_x_reg<false, false>;
+        // persistent: as many CTAs as are resident at once, each looping
+        const int grid = (int)std::min<int64_t>(
+            n_groups, (int64_t)sm_count() * resident_ctas((const void *)kern, threads, smem));
+        count_launch();
         return launch_pdl(kern, dim3((unsigned)grid),
                           dim3(threads), smem, st, 1,
                           reinterpret_cast<const __half *>(x), ldx, M, K, log2b, bits,
