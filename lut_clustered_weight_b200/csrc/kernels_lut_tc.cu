@@ -5,9 +5,9 @@
 //
 // CodeQuant2 Figure 4 describes the LUT kernel as a one-time LUT precompute
 // held in shared memory followed by table lookups.  Here:
-//  * Two threads per weight row: row t of a 128-row tile is lane t of tensor
-//    memory (TMEM); of the eight "expand" warps, warps w and w + 4 both serve
-//    TMEM lane quarter w, one taking the low and one the high 128 k of every
+//  * Four threads per weight row: row t of a 128-row tile is lane t of tensor
+//    memory (TMEM); of the sixteen "expand" warps, warps w, w + 4, w + 8 and
+//    w + 12 serve TMEM lane quarter w, each taking one 64-k chunk of every
 //    4-chunk (256-k) group.
 //  * PAIR mode (16-token tiles): the one-time precompute is a 256-entry pair
 //    table per row in shared memory -- entry b holds the two fp16 centroids
@@ -24,11 +24,15 @@
 //    exact) are the B operand, 128-byte-swizzled shared tiles loaded by TMA.
 //    The fp32 accumulator lives in TMEM and is read back with tcgen05.ld; the
 //    epilogue writes fp32 partial sums, or fp16 h = silu(s g) (s u) when the
-//    launch has one partial slot per output (SwiGLU fused).
-//  * Roles: warps 0-7 expand (each thread streams its row's index bytes
+//    launch has one partial slot per output (SwiGLU fused; for 256-token
+//    tiles staged in shared memory and written as whole 128-byte rows).  A
+//    finished item is drained after the next item's first group; tiles of up
+//    to 128 tokens keep two accumulators, so the drain overlaps MMAs.
+//  * Roles: warps 0-15 expand (each thread streams its row's index bytes
 //    through a private cp.async ring) and drain the accumulator; lane 0 of
-//    warp 8 issues the MMAs; lane 0 of warp 9 issues the TMA loads of the
-//    activation tiles.  mbarriers connect them; every wait is bounded.
+//    warp 16 issues the MMAs; lane 0 of warp 17 issues the TMA loads of the
+//    activation tiles.  mbarriers connect them (the A ring per slot and
+//    chunk); every wait is bounded.
 //  * Persistent: one CTA per SM works through (128-row tile x token tile)
 //    items cut into 64-k chunks -- contiguous stream-K ranges when there are
 //    few items, else whole (item, split) pieces strided over the CTAs.
