@@ -252,6 +252,10 @@ SMALL_MOE = [
                    act_bits=4, had_block_h=128, had_block_i=64),
     synth.MoEShape("moe_many_rows", H=192, I=128, E=4, top_k=2, n_shared=1, T=320, act_bits=8,
                    had_block_h=64, had_block_i=128, I_shared=256),
+    # 1400 routing slots: the grouping runs as a histogram launch and two
+    # placement CTAs (chunks of 1024 slots)
+    synth.MoEShape("moe_route_chunks", H=128, I=128, E=8, top_k=2, n_shared=0, T=700, act_bits=4,
+                   had_block_h=128, had_block_i=64),
     # gate/up with one partial slot: SwiGLU in the tensor-core epilogue (fp16 h)
     synth.MoEShape("moe_fused_t64", H=384, I=768, E=16, top_k=2, n_shared=0, T=200, act_bits=4,
                    had_block_h=128, had_block_i=256),
