@@ -21,9 +21,12 @@ Per workload:
   value       tokens/s of the whole job (sum over ranks / max time), device
               timed with CUDA events, inputs resident in HBM, the step
               replayed from a CUDA graph
-  e2e         the same metric through the C-ABI calls with host buffers: the
+  e2e         the same metric through the C-ABI calls with host buffers: every
               step's activations (and router logits) copied from pinned host
-              memory and the outputs copied back inside the timed region
+              memory and its outputs copied back inside the timed region, the
+              steps pipelined as a serving loop runs them (the next step's
+              inputs and the previous step's outputs move on two copy streams
+              while a step computes)
   roofline    the dominant LUT GEMM kernel, from its CUDA-event-timed
               launches: the decode kernels (mma.sync, tensor-memory decode)
               as algorithmic bytes against the measured HBM copy peak, the
@@ -381,12 +384,23 @@ class DeviceLayer:
     def run(self):
         self.call(self.x, self.lg, self.out)
 
-    def run_e2e(self):
-        self.x.copy_(self.x_h, non_blocking=True)
+    # e2e: two device buffer sets, so one step's copies overlap another's compute
+    def e2e_buffers(self):
+        import torch
+        self.xb = [self.x, torch.empty_like(self.x)]
+        self.lgb = [self.lg, torch.empty_like(self.lg) if self.lg is not None else None]
+        self.outb = [self.out, torch.empty_like(self.out)]
+
+    def h2d_into(self, b):
+        self.xb[b].copy_(self.x_h, non_blocking=True)
         if self.lg is not None:
-            self.lg.copy_(self.lg_h, non_blocking=True)
-        self.call(self.x, self.lg, self.out)
-        self.out_h.copy_(self.out, non_blocking=True)
+            self.lgb[b].copy_(self.lg_h, non_blocking=True)
+
+    def run_buf(self, b):
+        self.call(self.xb[b], self.lgb[b], self.outb[b])
+
+    def d2h_from(self, b):
+        self.out_h.copy_(self.outb[b], non_blocking=True)
 
     def counts(self, dev):
         """Per-expert token counts of this call (for the byte accounting)."""
@@ -468,6 +482,65 @@ def timed(fn, steps, dist, world):
     return max_over_ranks(e0.elapsed_time(e1), dist, world)
 
 
+def timed_e2e(calls, steps, warmup, dist, world):
+    """Device time (ms) of `steps` end-to-end steps: every step copies its
+    inputs from pinned host memory, runs the calls and copies its outputs back.
+    Steps are pipelined the way a serving loop runs them: step s + 1's inputs
+    go in on one copy stream and step s's outputs come out on another while
+    step s computes (two device buffer sets).  The timed region opens before
+    the first input copy and closes after the last output copy."""
+    import torch
+    for c in calls:
+        c.e2e_buffers()
+    comp = torch.cuda.current_stream()
+    cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+
+    def run(n, e_start=None):
+        inp = [ev(), ev()]      # inputs of buffer set b are on the device
+        done = [None, None]     # compute on buffer set b finished
+        outd = [None, None]     # outputs of buffer set b copied out
+        if e_start is not None:
+            cin.wait_event(e_start)
+        for s in range(n):
+            b = s & 1
+            if done[b] is not None:
+                cin.wait_event(done[b])         # buffer set b's inputs no longer read
+            with torch.cuda.stream(cin):
+                for c in calls:
+                    c.h2d_into(b)
+            inp[b] = ev()
+            inp[b].record(cin)
+            comp.wait_event(inp[b])
+            if outd[b] is not None:
+                comp.wait_event(outd[b])        # buffer set b's outputs copied out
+            for c in calls:
+                c.run_buf(b)
+            done[b] = ev()
+            done[b].record(comp)
+            cout.wait_event(done[b])
+            with torch.cuda.stream(cout):
+                for c in calls:
+                    c.d2h_from(b)
+            outd[b] = ev()
+            outd[b].record(cout)
+        comp.wait_stream(cout)
+        comp.wait_stream(cin)
+
+    run(warmup)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    run(steps, e0)
+    e1.record(comp)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    return max_over_ranks(e0.elapsed_time(e1), dist, world)
+
+
 class LinearCall:
     """One linear call of the single-linear workload (rotate+quantize, then the
     LUT GEMV), every tensor resident, plus pinned host copies for e2e."""
@@ -493,10 +566,22 @@ class LinearCall:
         self.cq.cq_lut_gemm(self.q, self.sx, s.K, s.act_bits, self.w, self.cb, y=self.y,
                             workspace=self.ws)
 
-    def run_e2e(self):
-        self.x.copy_(self.x_h, non_blocking=True)
-        self.run()
-        self.y_h.copy_(self.y, non_blocking=True)
+    def e2e_buffers(self):
+        import torch
+        self.xb = [self.x, torch.empty_like(self.x)]
+        self.yb = [self.y, torch.empty_like(self.y)]
+
+    def h2d_into(self, b):
+        self.xb[b].copy_(self.x_h, non_blocking=True)
+
+    def run_buf(self, b):
+        s = self.s
+        self.cq.cq_rotate_quantize(self.xb[b], s.had_block, s.act_bits, q_out=self.q, s_out=self.sx)
+        self.cq.cq_lut_gemm(self.q, self.sx, s.K, s.act_bits, self.w, self.cb, y=self.yb[b],
+                            workspace=self.ws)
+
+    def d2h_from(self, b):
+        self.y_h.copy_(self.yb[b], non_blocking=True)
 
 
 def lut_timed_launches(cq, step, steps, every_kernel=False):
@@ -781,15 +866,12 @@ def measure(cq, name, args, dev, stream, dist, world, peaks):
                                  args.steps)
 
     # ---- e2e: host buffers through the C-ABI, copies inside the timed region
-    def step_e2e():
-        for c in calls:
-            c.run_e2e()
-    for _ in range(args.warmup):
-        step_e2e()
-    ms_e2e = timed(step_e2e, args.steps, dist, world)
+    ms_e2e = timed_e2e(calls, args.steps, args.warmup, dist, world)
     e2e = {"value": job_throughput(units_per_step, args.steps, world, ms_e2e), "unit": "tokens/s",
            "h2d_bytes_per_step": sum(c.h2d for c in calls),
-           "d2h_bytes_per_step": sum(c.d2h for c in calls), "ms_per_step": ms_e2e / args.steps}
+           "d2h_bytes_per_step": sum(c.d2h for c in calls), "ms_per_step": ms_e2e / args.steps,
+           "pipelining": "step s+1's inputs in and step s's outputs out on two copy streams "
+                         "while step s computes (two device buffer sets)"}
 
     cfg.update({"tokens_per_step": units_per_step, "cuda_graph": use_graph,
                 "l2": "no flush: each step streams "
