@@ -482,6 +482,39 @@ def timed(fn, steps, dist, world):
     return max_over_ranks(e0.elapsed_time(e1), dist, world)
 
 
+class BatchedIO:
+    """The host I/O of many small calls batched the way a caller serving them
+    would: their inputs and outputs as views of one contiguous pinned host
+    buffer and one device buffer per buffer set, so a step copies once each
+    way.  `calls` expose x_h / y_h (host) and take device views through
+    set_views(b, x, y)."""
+
+    def __init__(self, calls):
+        import torch
+        self.calls = calls
+        c0 = calls[0]
+        n = len(calls)
+        self.x_h = torch.stack([c.x_h for c in calls]).pin_memory()
+        self.y_h = torch.empty((n,) + tuple(c0.y_h.shape), dtype=c0.y_h.dtype).pin_memory()
+        dev = c0.x.device
+        self.xd = [torch.empty(self.x_h.shape, dtype=self.x_h.dtype, device=dev) for _ in range(2)]
+        self.yd = [torch.empty(self.y_h.shape, dtype=self.y_h.dtype, device=dev) for _ in range(2)]
+
+    def e2e_buffers(self):
+        for i, c in enumerate(self.calls):
+            c.set_views([self.xd[0][i], self.xd[1][i]], [self.yd[0][i], self.yd[1][i]])
+
+    def h2d_into(self, b):
+        self.xd[b].copy_(self.x_h, non_blocking=True)
+
+    def run_buf(self, b):
+        for c in self.calls:
+            c.run_buf(b)
+
+    def d2h_from(self, b):
+        self.y_h.copy_(self.yd[b], non_blocking=True)
+
+
 def timed_e2e(calls, steps, warmup, dist, world):
     """Device time (ms) of `steps` end-to-end steps: every step copies its
     inputs from pinned host memory, runs the calls and copies its outputs back.
@@ -566,22 +599,14 @@ class LinearCall:
         self.cq.cq_lut_gemm(self.q, self.sx, s.K, s.act_bits, self.w, self.cb, y=self.y,
                             workspace=self.ws)
 
-    def e2e_buffers(self):
-        import torch
-        self.xb = [self.x, torch.empty_like(self.x)]
-        self.yb = [self.y, torch.empty_like(self.y)]
-
-    def h2d_into(self, b):
-        self.xb[b].copy_(self.x_h, non_blocking=True)
+    def set_views(self, xb, yb):
+        self.xb, self.yb = xb, yb
 
     def run_buf(self, b):
         s = self.s
         self.cq.cq_rotate_quantize(self.xb[b], s.had_block, s.act_bits, q_out=self.q, s_out=self.sx)
         self.cq.cq_lut_gemm(self.q, self.sx, s.K, s.act_bits, self.w, self.cb, y=self.yb[b],
                             workspace=self.ws)
-
-    def d2h_from(self, b):
-        self.y_h.copy_(self.yb[b], non_blocking=True)
 
 
 def lut_timed_launches(cq, step, steps, every_kernel=False):
@@ -866,7 +891,8 @@ def measure(cq, name, args, dev, stream, dist, world, peaks):
                                  args.steps)
 
     # ---- e2e: host buffers through the C-ABI, copies inside the timed region
-    ms_e2e = timed_e2e(calls, args.steps, args.warmup, dist, world)
+    io = [BatchedIO(calls)] if name == LINEAR else calls
+    ms_e2e = timed_e2e(io, args.steps, args.warmup, dist, world)
     e2e = {"value": job_throughput(units_per_step, args.steps, world, ms_e2e), "unit": "tokens/s",
            "h2d_bytes_per_step": sum(c.h2d for c in calls),
            "d2h_bytes_per_step": sum(c.d2h for c in calls), "ms_per_step": ms_e2e / args.steps,
