@@ -461,11 +461,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         xf.row_scales = m.fused ? rsc : nullptr;
     }
     if (m.ns > 0 && m.k_s != kKernMma) xf.ident = reinterpret_cast<__half *>(ws + m.o_bx_s);
-    const bool x16 = (xf.ncopy > 0 || xf.ident) &&
-                     rq_writes_f16(T, (int)m.H, ilog2(d->had_block_h), m.bits, x, m.H, xq, ldx);
     if (e == cudaSuccess)
         e = launch_rotate_quantize(x, m.H, T, (int)m.H, ilog2(d->had_block_h), m.bits, xq, ldx,
-                                   sx, st, w->x_scale, w->x_perm, x16 ? &xf : nullptr);
+                                   sx, st, w->x_scale, w->x_perm, &xf);
     // gate / up (dual) -> partial g, u
     if (e == cudaSuccess && m.E > 0) {
         LutLaunch L{};
@@ -482,13 +480,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
             L.h_row_stride = m.Imax;
         }
         if (m.k_r != kKernMma) {
-            void *b = ws + m.o_bx_r;
-            if (!x16)
-                e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, m.Rr, kMapPerm, perm, (int)m.k,
-                                        (int)T, b, st, m.fused ? sx : nullptr, rsc);
-            if (e == cudaSuccess)
-                e = m.k_r == kKernTs ? launch_lut_ts(L, m.gu_r, b, m.Rr, 0, st)
-                                     : launch_lut_tc(L, m.gu_r, b, m.Rr, 0, st);
+            const void *b = ws + m.o_bx_r;  // written by the x rotation
+            e = m.k_r == kKernTs ? launch_lut_ts(L, m.gu_r, b, m.Rr, 0, st)
+                               : launch_lut_tc(L, m.gu_r, b, m.Rr, 0, st);
         } else {
             e = launch_lut(L, m.gu_r, st);
         }
@@ -507,39 +501,32 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
             L.h_row_stride = m.Imax;
         }
         if (m.k_s != kKernMma) {
-            void *b = ws + m.o_bx_s;
-            if (!x16)
-                e = launch_codes_to_f16(xq, ldx, m.bits, (int)m.H, T, kMapIdentity, nullptr, 1,
-                                        (int)T, b, st);
-            if (e == cudaSuccess)
-                e = m.k_s == kKernTs ? launch_lut_ts(L, m.gu_s, b, T, (int)T, st)
-                                     : launch_lut_tc(L, m.gu_s, b, T, (int)T, st);
+            const void *b = ws + m.o_bx_s;  // written by the x rotation
+            e = m.k_s == kKernTs ? launch_lut_ts(L, m.gu_s, b, T, (int)T, st)
+                               : launch_lut_tc(L, m.gu_s, b, T, (int)T, st);
         } else {
             e = launch_lut(L, m.gu_s, st);
         }
     }
-    // SwiGLU + rotate + quantize of h
-    bool h16_r = false, h16_s = false;  // the down projections' B rows written by the rotation
+    // SwiGLU + rotate + quantize of h; the rotation also writes the down
+    // projections' tensor-core B rows
+    __half *bh_r = m.E > 0 && m.k_r != kKernMma ? reinterpret_cast<__half *>(ws + m.o_bh_r) : nullptr;
+    __half *bh_s = m.ns > 0 && m.k_s != kKernMma ? reinterpret_cast<__half *>(ws + m.o_bh_s) : nullptr;
     if (e == cudaSuccess && m.fused) {
         // h was written by the gate/up epilogues: rotate + quantize its rows
         // ... and write the down projections' tensor-core B rows as they go
         if (m.E > 0) {
             RqF16 hf16{};
-            hf16.ident = reinterpret_cast<__half *>(ws + m.o_bh_r);
-            h16_r = m.k_r != kKernMma &&
-                    rq_writes_f16(m.Rr, (int)m.I, ilog2(d->had_block_i), m.bits, hf, m.Imax, hq, ldh);
+            hf16.ident = bh_r;
             e = launch_rotate_quantize(hf, m.Imax, m.Rr, (int)m.I, ilog2(d->had_block_i), m.bits,
-                                       hq, ldh, sh, st, nullptr, nullptr, h16_r ? &hf16 : nullptr);
+                                       hq, ldh, sh, st, nullptr, nullptr, &hf16);
         }
         if (e == cudaSuccess && m.ns > 0) {
             RqF16 hf16{};
-            hf16.ident = reinterpret_cast<__half *>(ws + m.o_bh_s);
-            h16_s = m.k_s != kKernMma &&
-                    rq_writes_f16(m.Rs, (int)m.Is, ilog2(d->had_block_i_shared), m.bits,
-                                  hf + m.Rr * m.Imax, m.Imax, hq + m.Rr * ldh, ldh);
+            hf16.ident = bh_s;
             e = launch_rotate_quantize(hf + m.Rr * m.Imax, m.Imax, m.Rs, (int)m.Is,
                                        ilog2(d->had_block_i_shared), m.bits, hq + m.Rr * ldh, ldh,
-                                       sh + m.Rr, st, nullptr, nullptr, h16_s ? &hf16 : nullptr);
+                                       sh + m.Rr, st, nullptr, nullptr, &hf16);
         }
         if (e == cudaSuccess && dbg && dbg->h)
             e = cudaMemcpyAsync(dbg->h, hf, (size_t)m.R * m.Imax * 2, cudaMemcpyDeviceToDevice, st);
@@ -554,6 +541,8 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         a.perm = perm; a.topk = (int)std::max<int64_t>(m.k, 1); a.T = (int)T;
         a.x_scales = sx; a.bits = m.bits; a.hq = hq; a.ldhq = ldh; a.h_scales = sh;
         a.h_dbg = dbg ? dbg->h : nullptr;
+        a.f16_r = bh_r;
+        a.f16_s = bh_s;
         e = launch_swiglu_rq(a, m.R, st);
     }
     // down -> partial y
@@ -566,13 +555,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.w_stride = m.H * (m.I / 2); L.cb_stride = m.H * 16; L.N = (int)m.H; L.dual = false;
         L.out = pdn_r; L.out_split_stride = m.Rr * m.H; L.out_row_stride = m.H;
         if (m.k_r != kKernMma) {
-            void *b = ws + m.o_bh_r;
-            if (!h16_r)
-                e = launch_codes_to_f16(hq, ldh, m.bits, (int)m.I, m.Rr, kMapIdentity, nullptr, 1,
-                                        1, b, st);
-            if (e == cudaSuccess)
-                e = m.k_r == kKernTs ? launch_lut_ts(L, m.dn_r, b, m.Rr, 0, st)
-                                     : launch_lut_tc(L, m.dn_r, b, m.Rr, 0, st);
+            const void *b = bh_r;  // written by the h rotation
+            e = m.k_r == kKernTs ? launch_lut_ts(L, m.dn_r, b, m.Rr, 0, st)
+                               : launch_lut_tc(L, m.dn_r, b, m.Rr, 0, st);
         } else {
             e = launch_lut(L, m.dn_r, st);
         }
@@ -586,13 +571,9 @@ cq_status cq_moe_ffn(const cq_moe_desc *d, const void *x, const float *router_lo
         L.w_stride = m.H * (m.Is / 2); L.cb_stride = m.H * 16; L.N = (int)m.H; L.dual = false;
         L.out = pdn_s; L.out_split_stride = m.Rs * m.H; L.out_row_stride = m.H;
         if (m.k_s != kKernMma) {
-            void *b = ws + m.o_bh_s;
-            if (!h16_s)
-                e = launch_codes_to_f16(hq + m.Rr * ldh, ldh, m.bits, (int)m.Is, m.Rs,
-                                        kMapIdentity, nullptr, 1, 1, b, st);
-            if (e == cudaSuccess)
-                e = m.k_s == kKernTs ? launch_lut_ts(L, m.dn_s, b, m.Rs, 0, st)
-                                     : launch_lut_tc(L, m.dn_s, b, m.Rs, 0, st);
+            const void *b = bh_s;  // written by the h rotation
+            e = m.k_s == kKernTs ? launch_lut_ts(L, m.dn_s, b, m.Rs, 0, st)
+                               : launch_lut_tc(L, m.dn_s, b, m.Rs, 0, st);
         } else {
             e = launch_lut(L, m.dn_s, st);
         }

@@ -22,10 +22,8 @@ cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K,
                                    int bits, void *q, int64_t ldq_bytes, float *s,
                                    cudaStream_t st, const void *scale = nullptr,
                                    const int32_t *perm = nullptr, const RqF16 *f16 = nullptr);
-bool rq_writes_f16(int64_t M, int K, int log2b, int bits, const void *x, int64_t ldx,
-                   const void *q, int64_t ldq_bytes);
 // fp16 copies of the code rows (the B operand of the tensor-core GEMMs),
-// written by the rotate-quantize kernel itself: copy d (d < ncopy) of row m
+// written by every rotate-quantize kernel itself: copy d (d < ncopy) of row m
 // goes to rows[map[m * ncopy + d]] (rows[m] when map is NULL), with the row's
 // scale at row_scales[that row] when row_scales is non-NULL; ident, when
 // non-NULL, receives one more copy at row m.  Rows of K halves.

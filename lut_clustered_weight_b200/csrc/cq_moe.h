@@ -26,6 +26,8 @@ struct SwigluArgs {
     int64_t ldhq;
     float *h_scales;       // [R]
     void *h_dbg;           // fp16 [R][Imax] or NULL
+    __half *f16_r;         // fp16 copies of the routed h codes [R_routed][I], or NULL
+    __half *f16_s;         // fp16 copies of the shared h codes [R_shared][I_shared], or NULL
 };
 
 struct CombineArgs {

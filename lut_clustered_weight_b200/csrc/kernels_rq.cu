@@ -38,11 +38,11 @@ CQ_DEV RowPart row_part(int K, int log2b, int rank, int csize) {
 }
 
 // Rotate buf[0, n) (complete blocks), reduce the absmax over the row (across
-// the cluster when CLUSTER), quantize and store this CTA's codes; rank 0
-// stores the scale.
+// the cluster when CLUSTER), quantize and store this CTA's codes (and their
+// fp16 copies for row mrow of K positions); rank 0 stores the scale.
 template <bool CLUSTER>
 CQ_DEV void rq_finish(double *buf, RowPart part, int log2b, int bits, uint8_t *qrow,
-                      float *s_out) {
+                      float *s_out, const RqF16 &f16, int64_t mrow, int K) {
     __shared__ double red[33];
     __shared__ double s_amax;
     block_fwht<kRqThreads>(buf, part.n, log2b);
@@ -58,10 +58,12 @@ CQ_DEV void rq_finish(double *buf, RowPart part, int log2b, int bits, uint8_t *q
         cluster.sync();  // every CTA has read every s_amax
         rank0 = cluster.block_rank() == 0;
     }
-    block_quantize_range<kRqThreads>(buf, part.n, part.e0, bits, A, qrow);
+    block_quantize_range<kRqThreads>(buf, part.n, part.e0, bits, A, qrow, f16, mrow, K);
     if (rank0 && threadIdx.x == 0) {
         const int qmax = (1 << (bits - 1)) - 1;
-        *s_out = A > 0.0 ? quant_scale(A, log2b, qmax) : 0.0f;
+        const float sq = A > 0.0 ? quant_scale(A, log2b, qmax) : 0.0f;
+        *s_out = sq;
+        store_copy_scales(f16, mrow, sq);
     }
 }
 
@@ -112,7 +114,7 @@ template <bool CLUSTER>
 __global__ void __launch_bounds__(kRqThreads)
 k_rq_x(const __half *__restrict__ x, int64_t ldx, int K, int log2b, int bits,
        uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s,
-       const __half *__restrict__ scale, const int32_t *__restrict__ perm) {
+       const __half *__restrict__ scale, const int32_t *__restrict__ perm, const RqF16 f16) {
     extern __shared__ __align__(16) double buf[];
     int cs, rank;
     griddep_wait();
@@ -122,7 +124,7 @@ k_rq_x(const __half *__restrict__ x, int64_t ldx, int K, int log2b, int bits,
     const RowPart part = row_part(K, log2b, rank, cs);
     load_x_part(buf, x + m * ldx, part.e0, part.n, K, scale, perm, threadIdx.x, kRqThreads);
     __syncthreads();
-    rq_finish<CLUSTER>(buf, part, log2b, bits, q + m * ldq, s + m);
+    rq_finish<CLUSTER>(buf, part, log2b, bits, q + m * ldq, s + m, f16, m, K);
 }
 
 // ------------------------------------------------------------------ SwiGLU rows
@@ -181,7 +183,9 @@ __global__ void __launch_bounds__(kRqThreads) k_rq_swiglu(const SwigluArgs a) {
         }
     }
     __syncthreads();
-    rq_finish<CLUSTER>(buf, rp, log2b, a.bits, a.hq + p * a.ldhq, a.h_scales + p);
+    RqF16 f16{};
+    f16.ident = routed ? a.f16_r : a.f16_s;
+    rq_finish<CLUSTER>(buf, rp, log2b, a.bits, a.hq + p * a.ldhq, a.h_scales + p, f16, lp, I);
 }
 
 // ------------------------------------------------------------------ one warp per row
@@ -192,7 +196,7 @@ constexpr int kWarpRows = 4;
 __global__ void __launch_bounds__(kWarpRows * 32)
 k_rq_x_warp(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log2b, int bits,
             uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s,
-            const __half *__restrict__ scale, const int32_t *__restrict__ perm) {
+            const __half *__restrict__ scale, const int32_t *__restrict__ perm, const RqF16 f16) {
     extern __shared__ __align__(16) double wbuf[];
     griddep_wait();
     griddep_launch();
@@ -203,7 +207,7 @@ k_rq_x_warp(const __half *__restrict__ x, int64_t ldx, int64_t M, int K, int log
     load_x_part(buf, x + m * ldx, 0, K, K, scale, perm, lane, 32);
     __syncwarp();
     const double A = warp_fwht_absmax(buf, K, log2b);
-    warp_quantize_row(buf, K, log2b, bits, A, q + m * ldq, s + m);
+    warp_quantize_row(buf, K, log2b, bits, A, q + m * ldq, s + m, f16, m);
 }
 
 // ------------------------------------------------------------------ rows in registers
@@ -487,7 +491,9 @@ __global__ void __launch_bounds__(kWarpRows * 32) k_rq_swiglu_warp(const SwigluA
     }
     __syncwarp();
     const double A = warp_fwht_absmax(buf, I, log2b);
-    warp_quantize_row(buf, I, log2b, a.bits, A, a.hq + p * a.ldhq, a.h_scales + p);
+    RqF16 f16{};
+    f16.ident = routed ? a.f16_r : a.f16_s;
+    warp_quantize_row(buf, I, log2b, a.bits, A, a.hq + p * a.ldhq, a.h_scales + p, f16, lp);
 }
 
 static bool use_warp_rows(int64_t rows, int K, int log2b) {
@@ -547,11 +553,6 @@ static cudaError_t launch_clustered(Kern kern, int64_t rows, int cs, size_t smem
     return launch_pdl(kern, dim3((unsigned)(rows * cs)), dim3(kRqThreads), smem, st, cs, args...);
 }
 
-bool rq_writes_f16(int64_t M, int K, int log2b, int bits, const void *x, int64_t ldx,
-                   const void *q, int64_t ldq) {
-    return use_reg_rows(M, K, log2b, bits, x, ldx, q, ldq);
-}
-
 cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K, int log2b,
                                    int bits, void *q, int64_t ldq, float *s, cudaStream_t st,
                                    const void *scale, const int32_t *perm, const RqF16 *f16) {
@@ -576,20 +577,20 @@ cudaError_t launch_rotate_quantize(const void *x, int64_t ldx, int64_t M, int K,
                           reinterpret_cast<uint8_t *>(q), ldq, s, sc, perm, rows_per_cta,
                           (int)n_groups, f16 ? *f16 : RqF16{});
     }
-    if (f16 && (f16->ncopy > 0 || f16->ident)) return cudaErrorNotSupported;
+    const RqF16 f{f16 ? *f16 : RqF16{}};
     if (use_warp_rows(M, K, log2b)) {
         const size_t smem = (size_t)kWarpRows * K * sizeof(double);
         count_launch();
         return launch_pdl(k_rq_x_warp, dim3((unsigned)((M + kWarpRows - 1) / kWarpRows)),
                           dim3(kWarpRows * 32), smem, st, 1, reinterpret_cast<const __half *>(x),
                           ldx, M, K, log2b, bits, reinterpret_cast<uint8_t *>(q), ldq, s, sc,
-                          perm);
+                          perm, f);
     }
     const int cs = cluster_size(M, K, log2b);
     auto kern = cs == 1 ? k_rq_x<false> : k_rq_x<true>;
     return launch_clustered(kern, M, cs, part_smem(K, log2b, cs), st,
                             reinterpret_cast<const __half *>(x), ldx, K, log2b, bits,
-                            reinterpret_cast<uint8_t *>(q), ldq, s, sc, perm);
+                            reinterpret_cast<uint8_t *>(q), ldq, s, sc, perm, f);
 }
 
 cudaError_t launch_swiglu_rq(const SwigluArgs &a, int64_t rows, cudaStream_t st) {

@@ -9,6 +9,7 @@
 #pragma once
 
 #include "cq_common.cuh"
+#include "cq_internal.h"
 
 namespace cq {
 
@@ -180,12 +181,33 @@ CQ_DEV int quantize_round(double v, double R, bool &near_tie) {
     return __double2loint(big);
 }
 
+// The fp16 copies of the codes of row positions (e, e + 1) of row mrow: the
+// tensor-core B rows an RqF16 names (rows of K halves; small integers are
+// exact in fp16).
+CQ_DEV void store_code_copies(const RqF16 &f, int64_t mrow, int K, int e, int q0, int q1) {
+    const __half2 h = __halves2half2(__short2half_rn((short)q0), __short2half_rn((short)q1));
+    for (int d = 0; d < f.ncopy; d++) {
+        const int64_t row = f.map ? (int64_t)f.map[mrow * f.ncopy + d] : mrow;
+        *reinterpret_cast<__half2 *>(f.rows + row * K + e) = h;
+    }
+    if (f.ident) *reinterpret_cast<__half2 *>(f.ident + mrow * K + e) = h;
+}
+// The row's scale beside each routed copy (RqF16::row_scales).
+CQ_DEV void store_copy_scales(const RqF16 &f, int64_t mrow, float sq) {
+    if (!f.row_scales) return;
+    for (int d = 0; d < f.ncopy; d++)
+        f.row_scales[f.map ? (int64_t)f.map[mrow * f.ncopy + d] : mrow] = sq;
+}
+CQ_DEV bool has_copies(const RqF16 &f) { return f.ncopy > 0 || f.ident != nullptr; }
+
 // Quantize buf[0, n) (rotated values of row positions [e0, e0 + n)) and
 // store the codes: bits 4 -> packed bytes (low nibble = even position),
 // bits 8 -> int8.  e0 and n are even.  A is the absmax of the whole row.
+// With copies (f16 non-empty), also the fp16 copies of row mrow's codes.
 template <int THREADS>
 __device__ void block_quantize_range(const double *buf, int n, int e0, int bits, double A,
-                                     uint8_t *qrow) {
+                                     uint8_t *qrow, const RqF16 &f16, int64_t mrow, int K) {
+    const bool copies = has_copies(f16);
     const int qmax = (1 << (bits - 1)) - 1;
     const long long Ai = __double2ll_rn(A * 16777216.0);
     const double R = Ai > 0 ? __ddiv_rn((double)qmax, A) : 0.0;
@@ -205,6 +227,7 @@ __device__ void block_quantize_range(const double *buf, int n, int e0, int bits,
             c.y = (char)q1;
             reinterpret_cast<char2 *>(qrow + e0)[p] = c;
         }
+        if (copies) store_code_copies(f16, mrow, K, e0 + 2 * p, q0, q1);
     }
 }
 
@@ -264,9 +287,11 @@ CQ_DEV double warp_fwht_absmax(double *buf, int K, int log2b) {
     return warp_max_d(amax);
 }
 
-// Quantize a rotated row held by one warp and store codes and scale.
+// Quantize a rotated row held by one warp and store codes and scale (and the
+// fp16 copies of row mrow's codes, when f16 names any).
 CQ_DEV void warp_quantize_row(const double *buf, int K, int log2b, int bits, double A,
-                              uint8_t *qrow, float *s_out) {
+                              uint8_t *qrow, float *s_out, const RqF16 &f16, int64_t mrow) {
+    const bool copies = has_copies(f16);
     const int lane = threadIdx.x & 31;
     const int qmax = (1 << (bits - 1)) - 1;
     const long long Ai = __double2ll_rn(A * 16777216.0);
@@ -287,8 +312,13 @@ CQ_DEV void warp_quantize_row(const double *buf, int K, int log2b, int bits, dou
             c.y = (char)q1;
             reinterpret_cast<char2 *>(qrow)[p] = c;
         }
+        if (copies) store_code_copies(f16, mrow, K, 2 * p, q0, q1);
     }
-    if (lane == 0) *s_out = Ai > 0 ? quant_scale(A, log2b, qmax) : 0.0f;
+    if (lane == 0) {
+        const float sq = Ai > 0 ? quant_scale(A, log2b, qmax) : 0.0f;
+        *s_out = sq;
+        store_copy_scales(f16, mrow, sq);
+    }
 }
 
 }  // namespace cq
