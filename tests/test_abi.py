@@ -123,3 +123,77 @@ def test_timing_record_argument_checks():
     assert f(None, None, -1, ctypes.byref(n)) == cq.CQ_ERR_INVALID_ARGUMENT
     assert f(None, None, 4, ctypes.byref(n)) == cq.CQ_ERR_INVALID_ARGUMENT
     assert cq.cq_timing_read_launches() == []
+
+
+def test_rotate_quantize_ex_argument_checks():
+    f = cq.lib.cq_rotate_quantize_ex
+    ok = dict(x=FAKE, M=2, K=64, b=16, bits=4, scale=FAKE, perm=FAKE, q=FAKE, s=FAKE)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return f(a["x"], a["M"], a["K"], a["b"], a["bits"], a["scale"], a["perm"], a["q"],
+                 a["s"], None)
+
+    assert call(bits=5) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert call(b=12) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert call(scale=FAKE + 2) == cq.CQ_ERR_INVALID_ARGUMENT   # misaligned scale
+    assert call(perm=FAKE + 4) == cq.CQ_ERR_INVALID_ARGUMENT    # misaligned perm
+    assert call(q=None) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert call(K=12, b=4) == cq.CQ_ERR_UNSUPPORTED             # K % 8
+    assert call(M=0) == cq.CQ_OK
+    assert call(M=0, scale=None, perm=None) == cq.CQ_OK         # both optional
+
+
+def test_lut_gemm_ex_argument_checks():
+    f = cq.lib.cq_lut_gemm_ex
+    base = dict(q=FAKE, s=FAKE, M=4, K=256, bits=4, w=FAKE, ib=3, cb=FAKE, N=128, y=FAKE,
+                ws=None, wsb=0)
+
+    def call(**kw):
+        a = {**base, **kw}
+        return f(a["q"], a["s"], a["M"], a["K"], a["bits"], a["w"], a["ib"], a["cb"], a["N"],
+                 a["y"], a["ws"], a["wsb"], None)
+
+    for ib in (0, 2, 6, 8):
+        assert call(ib=ib) == cq.CQ_ERR_UNSUPPORTED
+        assert cq.lib.cq_lut_gemm_ex_workspace_size(4, 128, 256, 4, ib) == 0
+    for ib in (3, 5):
+        assert call(ib=ib, bits=2) == cq.CQ_ERR_INVALID_ARGUMENT
+        assert call(ib=ib, w=None) == cq.CQ_ERR_INVALID_ARGUMENT
+        assert call(ib=ib, cb=FAKE + 8) == cq.CQ_ERR_INVALID_ARGUMENT
+        assert call(ib=ib, K=240) == cq.CQ_ERR_UNSUPPORTED      # K % 32
+        assert call(ib=ib, N=96) == cq.CQ_ERR_UNSUPPORTED       # N % 64
+        assert call(ib=ib, M=0) == cq.CQ_OK
+        need = cq.lib.cq_lut_gemm_ex_workspace_size(4, 128, 256, 4, ib)
+        assert need > 0 and need % 256 == 0                      # split-K partial sums
+        assert call(ib=ib) == cq.CQ_ERR_WORKSPACE
+        assert call(ib=ib, ws=FAKE, wsb=need - 1) == cq.CQ_ERR_WORKSPACE
+    # 4-bit indices are cq_lut_gemm exactly, checks included
+    assert cq.lib.cq_lut_gemm_ex_workspace_size(4, 128, 9728, 4, 4) == \
+        cq.cq_lut_gemm_workspace_size(4, 128, 9728, 4)
+    assert call(ib=4, K=255) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert call(ib=4, K=240) == cq.CQ_ERR_UNSUPPORTED
+    assert call(ib=4, M=0) == cq.CQ_OK
+
+
+def test_lut_gemm_noalloc_argument_checks():
+    f = cq.lib.cq_lut_gemm_noalloc
+    base = dict(q=FAKE, s=FAKE, M=4, K=256, bits=4, w=FAKE, cb=FAKE, N=128, y=FAKE)
+
+    def call(**kw):
+        a = {**base, **kw}
+        return f(a["q"], a["s"], a["M"], a["K"], a["bits"], a["w"], a["cb"], a["N"], a["y"],
+                 None)
+
+    assert call(bits=2) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert call(y=None) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert call(q=FAKE + 1) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert call(K=255) == cq.CQ_ERR_INVALID_ARGUMENT
+    assert call(K=240) == cq.CQ_ERR_UNSUPPORTED
+    assert call(N=96) == cq.CQ_ERR_UNSUPPORTED
+    assert call(M=0) == cq.CQ_OK
+    # a problem whose scratch exceeds the fixed array is refused before any launch
+    M, N, K = 16, 65536, 16384
+    need = cq.cq_lut_gemm_workspace_size(M, N, K, 4)
+    assert need > cq.NOALLOC_SCRATCH_BYTES
+    assert call(M=M, N=N, K=K) == cq.CQ_ERR_UNSUPPORTED
